@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant KV-cache hot path on B200.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+encode every key/value row of the batch into the packed cache (norm,
+rotation, quantization, QJL signs, packing) and run one decode-attention
+step for every query head over it (query preparation, split-K scoring from
+the codes with online softmax and value accumulation, combine).  The
+default workload is the multi-head decode case (batch 8, 32 heads, 4096
+cached tokens, bits 4, fp16 K/V).  Other workloads: --workload gqa_decode |
+shared_prefix | bulk_encode | single_head.
+
+Prints ONE JSON line (rank 0).  `value` = KV tokens scored per second over
+the whole job (sum over ranks of batch*heads*tokens per step / max-over-ranks
+device time per step); for bulk_encode it is input GB/s.  `e2e` is the same
+metric through the public API with host (pinned) inputs copied in and the
+output copied back inside the timed region.  `roofline` is for the kernel
+with the largest share of the step, timed live with CUDA events on the
+launching stream.  `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode: KV tokens scored/s; encode GB/s; % of HBM roofline"
+D = 128
+M = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha_decode",
+                    choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def row_bytes(bits):
+    return (bits - 1) * D // 8 + M // 8 + 8, bits * D // 8 + 4
+
+
+# ------------------------------------------------------------------ workloads
+
+class Workload:
+    """Holds device inputs, caches and the step function of one workload."""
+
+    def __init__(self, name, device, rank=0):
+        import torch
+
+        import kv_cache_vector_10_b200 as tq
+        from kv_cache_vector_10_b200 import workloads as W
+        self.name, self.tq, self.torch = name, tq, torch
+        self.codecs = {}
+        self.launches = 0
+        seed_shift = 1000 * rank
+        if name in ("mha_decode", "gqa_decode", "single_head"):
+            if name == "mha_decode":
+                w = W.mha_decode(device=device, data_seed=2 + seed_shift)
+            elif name == "gqa_decode":
+                w = W.gqa_decode(device=device, data_seed=3 + seed_shift)
+            else:
+                w = W.single_head(device=device, data_seed=1 + seed_shift)
+            self.w = w
+            B, Hkv, T, _ = w["k"].shape
+            Hq = w["q"].shape[1]
+            bits = w["bits"]
+            self.codec = tq.Codec(D, bits, M, w["seed"])
+            self.cache = self.codec.alloc(B, Hkv, (T + 15) // 16 * 16, device)
+            self.segments = [tq.Segment(self.cache, T, b, 1, codes_batch=b) for b in range(B)]
+            self.inputs = dict(k=w["k"], v=w["v"], q=w["q"])
+            self.B, self.Hq, self.Hkv = B, Hq, Hkv
+            self.tokens_scored = B * Hq * T
+            kr, vr = row_bytes(bits)
+            es = w["k"].element_size()
+            self.enc_bytes = B * Hkv * T * (2 * D * es + kr + vr)
+            self.dec_bytes = B * Hkv * T * (kr + vr) + B * Hq * D * 2 * w["q"].element_size()
+            self.desc = (f"{name}: batch {B}, {Hq} query heads over {Hkv} kv heads, {T} tokens, d{D}, "
+                         f"m{M}, bits {bits} (K {bits - 1}+1, V {bits}), {str(w['k'].dtype).split('.')[-1]}")
+        elif name == "shared_prefix":
+            w = W.shared_prefix(device=device, data_seed=5 + seed_shift)
+            self.w = w
+            A, Hq = w["q"].shape[:2]
+            Hkv = w["n_kv_heads"]
+            P, Tt = w["prefix_k"].shape[2], w["tail_k"].shape[2]
+            self.pcodec = tq.Codec(D, w["prefix_bits"], M, w["seed"])
+            self.tcodec = tq.Codec(D, w["tail_bits"], M, w["seed"])
+            self.pcache = self.pcodec.alloc(1, Hkv, P, device)
+            self.tcache = self.tcodec.alloc(A, Hkv, Tt, device)
+            self.segments = [tq.Segment(self.pcache, P, 0, A)] + \
+                            [tq.Segment(self.tcache, Tt, a, 1, codes_batch=a) for a in range(A)]
+            self.inputs = dict(pk=w["prefix_k"], pv=w["prefix_v"], tk=w["tail_k"], tv=w["tail_v"], q=w["q"])
+            self.B, self.Hq, self.Hkv = A, Hq, Hkv
+            self.tokens_scored = A * Hq * (P + Tt)
+            pkr, pvr = row_bytes(w["prefix_bits"])
+            tkr, tvr = row_bytes(w["tail_bits"])
+            es = w["prefix_k"].element_size()
+            self.enc_bytes = Hkv * P * (2 * D * es + pkr + pvr) + A * Hkv * Tt * (2 * D * es + tkr + tvr)
+            self.dec_bytes = Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + A * Hq * D * 4
+            self.desc = (f"shared_prefix: {A} agents, prefix {P} tokens at bits {w['prefix_bits']} read once per "
+                         f"kv head + {A} tails of {Tt} tokens at bits {w['tail_bits']}, {Hq} q heads over {Hkv} kv "
+                         f"heads, d{D}, m{M}, bf16")
+        elif name == "bulk_encode":
+            w = W.bulk_encode(device=device, data_seed=4 + seed_shift)
+            self.w = w
+            L, H, T, _ = w["k"].shape
+            self.c3 = tq.Codec(D, 3, M, w["seed"])
+            self.c4 = tq.Codec(D, 4, M, w["seed"])
+            self.cache3 = self.c3.alloc(28, H, T, device)
+            self.cache4a = self.c4.alloc(2, H, T, device)
+            self.cache4b = self.c4.alloc(2, H, T, device)
+            self.inputs = dict(k=w["k"], v=w["v"])
+            self.B, self.Hq, self.Hkv = L, H, H
+            self.tokens_scored = 0
+            es = w["k"].element_size()
+            k3, v3 = row_bytes(3)
+            k4, v4 = row_bytes(4)
+            self.in_bytes = 2 * L * H * T * D * es
+            self.out_bytes = H * T * (28 * (k3 + v3) + 4 * (k4 + v4))
+            self.enc_bytes = self.in_bytes + self.out_bytes
+            self.dec_bytes = 0
+            self.desc = (f"bulk_encode: {L} layers x {H} kv heads x {T} tokens x d{D}, bf16; bits 3 on layers "
+                         f"2..29, bits 4 on layers 0, 1, 30, 31; m{M}")
+        self.out = None
+        self.ws = None
+
+    # one step with device-resident inputs; returns (encode_events, decode_events)
+    def step(self, inp, ev=None):
+        torch, tq = self.torch, self.tq
+        e = ev or {}
+        if "enc0" in e:
+            e["enc0"].record()
+        n = 0
+        if self.name in ("mha_decode", "gqa_decode", "single_head"):
+            self.codec.encode_kv(inp["k"], inp["v"], self.cache)
+            n += 1
+        elif self.name == "shared_prefix":
+            self.pcodec.encode_kv(inp["pk"], inp["pv"], self.pcache)
+            self.tcodec.encode_kv(inp["tk"], inp["tv"], self.tcache)
+            n += 2
+        else:
+            k, v = inp["k"], inp["v"]
+            self.c4.encode_kv(k[:2], v[:2], self.cache4a)
+            self.c3.encode_kv(k[2:30], v[2:30], self.cache3)
+            self.c4.encode_kv(k[30:], v[30:], self.cache4b)
+            n += 3
+        if "enc1" in e:
+            e["enc1"].record()
+        if self.name != "bulk_encode":
+            if self.out is None:
+                need = tq.tq_decode_workspace_bytes(self.segments, self.B, self.Hq, self.Hkv)
+                self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=inp["q"].device)
+                self.out = torch.empty(self.B, self.Hq, D, dtype=inp["q"].dtype, device=inp["q"].device)
+            tq.tq_decode_attention(self.segments, inp["q"], self.B, self.Hq, self.Hkv, self.out, self.ws)
+            groups = len(set((s.codec.bits) for s in self.segments))
+            n += 2 + groups
+        if "dec1" in e:
+            e["dec1"].record()
+        self.launches = n
+        return self.out
+
+
+def clock_sampler(device_index):
+    """Samples SM clocks and throttle reasons every 200 ms until stopped."""
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+    try:
+        p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200",
+                              "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    except Exception:
+        return None, []
+    rows = []
+
+    def rd():
+        for line in p.stdout:
+            rows.append([x.strip() for x in line.split(",")])
+    t = threading.Thread(target=rd, daemon=True)
+    t.start()
+    return p, rows
+
+
+def summarize_clocks(rows):
+    sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+    mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+    reasons = set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        if len(r) >= 9:
+            for i, nm in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(nm)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    sm.sort()
+    return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+def oracle_unit(wl_name, rank_seed=0):
+    """One bounded CPU-oracle unit of the workload: returns (seconds, units, unit_name, sample_desc).
+
+    Units are KV tokens scored (decode workloads) or input bytes (bulk_encode)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from kv_cache_vector_10_b200 import workloads as W
+    if wl_name == "bulk_encode":
+        w = W.bulk_encode(device="cpu", layers=1, heads=1, n_tokens=1024)
+        oc = oracle.Codec(D, 3, M, 42)
+        k = w["k"][0, 0].double().numpy()
+        v = w["v"][0, 0].double().numpy()
+        t0 = time.perf_counter()
+        oc.encode(k, 0, True)
+        oc.encode(v, 0, False)
+        dt = time.perf_counter() - t0
+        return dt, 2 * 1024 * D * 2, "bytes", "1 layer x 1 head x 1024 tokens, bits 3, K+V encode"
+    if wl_name == "shared_prefix":
+        w = W.shared_prefix(device="cpu", agents=1, prefix_tokens=1024, tail_tokens=256)
+        pc, tc = oracle.Codec(D, 2, M, 42), oracle.Codec(D, 4, M, 42)
+        t0 = time.perf_counter()
+        ekp = pc.encode(w["prefix_k"][0, 0].double().numpy(), 0, True)
+        evp = pc.encode(w["prefix_v"][0, 0].double().numpy(), 0, False)
+        ekt = tc.encode(w["tail_k"][0, 0].double().numpy(), 0, True)
+        evt = tc.encode(w["tail_v"][0, 0].double().numpy(), 0, False)
+        for j in range(4):
+            oracle.attention(w["q"][0, j].double().numpy(),
+                             [(pc, 0, ekp["rows"], evp["rows"]), (tc, 0, ekt["rows"], evt["rows"])])
+        dt = time.perf_counter() - t0
+        return dt, 4 * (1024 + 256), "tokens", "1 agent x 1 kv head (4 q heads), prefix 1024 + tail 256 tokens"
+    if wl_name == "mha_decode":
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024)
+        G = 1
+    elif wl_name == "gqa_decode":
+        w = W.gqa_decode(device="cpu", batch=1, q_heads=4, kv_heads=1, n_tokens=1024)
+        G = 4
+    else:
+        w = W.single_head(device="cpu")
+        G = 4
+    oc = oracle.Codec(D, w["bits"], M, w["seed"])
+    T = w["k"].shape[2]
+    t0 = time.perf_counter()
+    ek = oc.encode(w["k"][0, 0].double().numpy(), 0, True)
+    ev = oc.encode(w["v"][0, 0].double().numpy(), 0, False)
+    for j in range(G):
+        oracle.attention(w["q"][0, j].double().numpy(), [(oc, 0, ek["rows"], ev["rows"])])
+    dt = time.perf_counter() - t0
+    return dt, G * T, "tokens", f"1 kv head x {G} query head(s) x {T} tokens: encode K+V + decode"
+
+
+def cpu_baseline(wl_name, seconds):
+    tot_t, tot_u, n = 0.0, 0, 0
+    unit = desc = None
+    while tot_t < seconds or n == 0:
+        dt, u, unit, desc = oracle_unit(wl_name)
+        tot_t += dt
+        tot_u += u
+        n += 1
+    val = tot_u / tot_t
+    if unit == "bytes":
+        return {"value": val / 1e9, "unit": "GB/s in", "cores": 1, "kind": "oracle",
+                "sample": f"{n} x ({desc}), {tot_t:.1f} s single-threaded fp64 C oracle"}
+    return {"value": val, "unit": "KV tokens scored/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} x ({desc}), {tot_t:.1f} s single-threaded fp64 C oracle"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_unit(args.workload)
+    tot_t, tot_u, unit, desc = 0.0, 0, None, None
+    for _ in range(args.steps):
+        dt, u, unit, desc = oracle_unit(args.workload)
+        tot_t += dt
+        tot_u += u
+    val = tot_u / tot_t
+    unit_name = "GB/s in" if unit == "bytes" else "KV tokens scored/s"
+    if unit == "bytes":
+        val /= 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit_name, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample": desc},
+            "cpu_baseline": {"value": val, "unit": unit_name, "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} timed steps, each {desc}"},
+            "e2e": {"value": val, "unit": unit_name, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    wl = Workload(args.workload, dev, rank)
+    inp = wl.inputs
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        wl.step(inp)
+    torch.cuda.synchronize()
+    # timed region
+    evs = [dict(enc0=torch.cuda.Event(enable_timing=True), enc1=torch.cuda.Event(enable_timing=True),
+                dec1=torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    smi, rows = clock_sampler(dev.index)
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        wl.step(inp, evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    if smi is not None:
+        time.sleep(0.25)
+        smi.terminate()
+    total_ms = t_start.elapsed_time(t_end)
+    enc_ms = sum(e["enc0"].elapsed_time(e["enc1"]) for e in evs) / args.steps
+    dec_ms = (sum(e["enc1"].elapsed_time(e["dec1"]) for e in evs) / args.steps) if wl.dec_bytes else 0.0
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    clocks = summarize_clocks(rows)
+
+    # end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.cpu().pin_memory() for k, v in inp.items()}
+        dev_bufs = {k: torch.empty_like(v) for k, v in inp.items()}
+        out_host = torch.empty(wl.B, wl.Hq, D, dtype=inp["q"].dtype).pin_memory() if "q" in inp else None
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = out_host.numel() * out_host.element_size() if out_host is not None else 0
+
+        def e2e_step():
+            for k2, v2 in host.items():
+                dev_bufs[k2].copy_(v2, non_blocking=True)
+            o = wl.step(dev_bufs)
+            if out_host is not None:
+                out_host.copy_(o, non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        a.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        if wl.name == "bulk_encode":
+            ev, eu = world * wl.in_bytes / (e_ms * 1e-3) / 1e9, "GB/s in"
+        else:
+            ev, eu = world * wl.tokens_scored / (e_ms * 1e-3), "KV tokens scored/s"
+        e2e = {"value": ev, "unit": eu, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    hbm, peak_kind = peaks()
+    if wl.name == "bulk_encode":
+        value, unit = world * wl.in_bytes / (ms_step * 1e-3) / 1e9, "GB/s in"
+    else:
+        value, unit = world * wl.tokens_scored / (ms_step * 1e-3), "KV tokens scored/s"
+    enc_gbs = wl.enc_bytes / (enc_ms * 1e-3) / 1e9 if enc_ms > 0 else None
+    dec_gbs = wl.dec_bytes / (dec_ms * 1e-3) / 1e9 if dec_ms > 0 else None
+    kernels = {"encode": {"ms": enc_ms, "algorithmic_bytes": wl.enc_bytes, "achieved_gbs": enc_gbs,
+                          "frac_of_" + peak_kind + "_hbm": enc_gbs / hbm if enc_gbs else None}}
+    if wl.dec_bytes:
+        kernels["decode"] = {"ms": dec_ms, "algorithmic_bytes": wl.dec_bytes, "achieved_gbs": dec_gbs,
+                             "frac_of_" + peak_kind + "_hbm": dec_gbs / hbm if dec_gbs else None,
+                             "kv_tokens_scored_per_s": wl.tokens_scored / (dec_ms * 1e-3)}
+    dom = "encode" if enc_ms >= dec_ms else "decode"
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": dk["achieved_gbs"] / hbm, "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)",
+                "traffic": None}
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.desc, "l2": "inputs larger than L2 (no flush needed)",
+                       "step": "encode all K/V rows + one decode step per query head"},
+            "roofline": roofline, "kernels": kernels, "gpu_launches": wl.launches * args.steps,
+            "clocks": clocks, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant KV-cache compression and attention over
+ * the compressed cache, on one NVIDIA B200 (sm_100a).
+ *
+ * The method (turboquant-plus-rs 0.1.0 README, "Architecture" and "Key
+ * ideas"): every key/value head vector is rotated by a seeded random
+ * rotation (fast Walsh-Hadamard with random signs), scalar-quantized per
+ * coordinate against the Lloyd-Max codebook of the post-rotation Gaussian
+ * with norm extraction and correction (PolarQuant: b-1 bits for keys, b bits
+ * MSE-only for values), and for keys the residual gets a 1-bit QJL sign
+ * sketch.  Attention scores are estimated from the packed codes.  The call
+ * shapes follow bitpolar 0.3.3 src/kv_cache.rs (KvCacheConfig {head_dim,
+ * bits, projections, seed}; KvCacheCompressor::push, attention_scores,
+ * decode_values; MultiHeadKvCache with seed + h per head).
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers owned by the caller, on the
+ *    device that was current when the context was created.  The library
+ *    never frees or keeps them past the call.  A context owns only its small
+ *    device tables (signs, QJL matrix, codebooks) and a status word.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call enqueues its kernels on that stream and returns
+ *    without synchronizing, except tq_get_status and tq_ensure_heads.
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and returned as tq_status; nothing runs in that case.
+ *  - There is no CPU fallback: if the device is not an sm_100 GPU or the
+ *    kernels cannot launch, the call returns TQ_ERR_DEVICE / TQ_ERR_CUDA.
+ *  - d = head_dim, m = projections, b = bits, B_K = b-1, B_V = b.
+ *
+ * Packed row formats (the pages give no layout; this is the library's):
+ *  K row (k_row_bytes = B_K*d/8 + m/8 + 8):
+ *    B_K index bit planes of d/8 bytes (plane p holds bit p of the index of
+ *    coordinate j at byte j/8, bit j%8), then the m-bit QJL sign plane
+ *    (projection i at byte i/8, bit i%8; 1 = non-negative), then n_s
+ *    (float32, the corrected norm), then gamma (float32, the residual norm).
+ *  V row (v_row_bytes = B_V*d/8 + 4):
+ *    B_V-bit index fields, coordinate j at bit B_V*j of a little-endian bit
+ *    stream, then n_s (float32).
+ *  Indices count the codebook boundaries at or below z = sqrt(d)*Pi*x/|x|.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_NULL = 1,          /* a required pointer is NULL */
+    TQ_ERR_ZERO_DIM = 2,      /* head_dim == 0 (bitpolar ZeroDimension) */
+    TQ_ERR_DIM = 3,           /* head_dim not 64 or 128 (bitpolar OddDimension, generalized) */
+    TQ_ERR_BITS = 4,          /* bits not in 2..5 (bitpolar InvalidBitWidth) */
+    TQ_ERR_ZERO_PROJ = 5,     /* projections == 0 (bitpolar ZeroProjections) */
+    TQ_ERR_PROJ = 6,          /* projections not a multiple of 32 in [32, 256] */
+    TQ_ERR_EMPTY = 7,         /* zero heads or zero batch (bitpolar EmptyInput) */
+    TQ_ERR_DIM_MISMATCH = 8,  /* shapes disagree: H_q % H_kv, tokens beyond capacity,
+                                 capacity not a multiple of 16 (bitpolar DimensionMismatch) */
+    TQ_ERR_WORKSPACE = 9,     /* workspace NULL or smaller than tq_decode_workspace_bytes */
+    TQ_ERR_ALIGN = 10,        /* a pointer or stride breaks the stated alignment */
+    TQ_ERR_CUDA = 11,         /* a CUDA runtime call failed (see tq_last_cuda_error) */
+    TQ_ERR_DEVICE = 12,       /* current device is not compute capability 10.0 */
+    TQ_ERR_LIMIT = 13         /* a count exceeds a documented maximum (segments, heads) */
+} tq_status;
+
+typedef enum tq_dtype { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
+typedef enum tq_which { TQ_KEYS = 0, TQ_VALUES = 1, TQ_BOTH = 2 } tq_which;
+
+typedef struct tq_ctx tq_ctx;
+
+/* A packed cache: two device buffers laid out [batch][n_kv_heads][capacity]
+ * rows of k_row_bytes / v_row_bytes.  Either pointer may be NULL when the
+ * call does not touch it.  capacity must be a multiple of 16 and the
+ * buffers 16-byte aligned, so every (batch, head) block starts 16-byte
+ * aligned.  Sized by tq_packed_bytes. */
+typedef struct tq_codes {
+    void *k;
+    void *v;
+    int32_t batch;
+    int32_t n_kv_heads;
+    int64_t capacity;
+} tq_codes;
+
+/* One segment of compressed keys/values that a contiguous range of
+ * sequences attends to (shared prefixes appear once with n_seqs > 1; a
+ * sequence's private tail has n_seqs = 1).  Tokens [0, n_tokens) of batch
+ * slot `codes_batch` of `codes` are read.  Different segments may use
+ * different contexts (bit widths, seeds). */
+typedef struct tq_segment {
+    const tq_ctx *ctx;
+    tq_codes codes;
+    int32_t codes_batch;
+    int32_t first_seq;
+    int32_t n_seqs;
+    int32_t reserved;
+    int64_t n_tokens;
+} tq_segment;
+
+#define TQ_MAX_SEGMENTS 64
+#define TQ_MAX_HEADS 1024
+
+/* Create a codec context on the current CUDA device: KvCacheConfig {head_dim,
+ * bits, projections, seed} of bitpolar src/kv_cache.rs, where `bits` is the
+ * total TurboQuant width b (keys: b-1 PolarQuant bits + 1 QJL bit; values: b
+ * MSE bits; turboquant-plus-rs "Architecture").  Builds the Lloyd-Max
+ * codebooks on the host and uploads them.  Head tables are built by
+ * tq_ensure_heads (or on first use).  head_dim in {64, 128}; bits in 2..5;
+ * projections a multiple of 32 in [32, 256].  On success *out owns device
+ * memory released by tq_destroy.  Synchronous. */
+tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_ctx **out);
+
+/* Release a context and its device tables (synchronizes the device). NULL is a no-op. */
+void tq_destroy(tq_ctx *ctx);
+
+/* Build and upload the tables of heads 0..n_heads-1 (head h uses seed + h,
+ * bitpolar MultiHeadKvCache::new): random signs of the rotation and the
+ * m x d QJL matrix (binary16 entries).  Synchronous; idempotent.  Calls that
+ * use more heads than built call this themselves, so make the first such
+ * call before capturing a CUDA graph.  n_heads <= TQ_MAX_HEADS. */
+tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads);
+
+/* Packed bytes per token-head row: K, V, or K+V for TQ_BOTH; 0 if ctx is NULL. */
+int64_t tq_row_bytes(const tq_ctx *ctx, tq_which which);
+
+/* Device bytes of a tq_codes buffer pair (or one side) for the given shape
+ * (turboquant-plus-rs "Modules": memory footprint). */
+size_t tq_packed_bytes(const tq_ctx *ctx, int batch, int n_kv_heads, int64_t capacity, tq_which which);
+
+/* Encode n_tokens keys and/or values per (batch, head) into tokens
+ * [token_offset, token_offset + n_tokens) of `codes` (bitpolar
+ * KvCacheCompressor::push; MultiHeadKvCache::push_token).
+ *  k, v   : device input, element (b, h, t, j) at base[b*stride_b + h*stride_h
+ *           + t*stride_t + j] in `dtype`; either may be NULL to skip that side.
+ *           Rows must be 16-byte aligned (strides multiples of 16 bytes).
+ *  codes  : batch and n_kv_heads must equal the call's; token_offset +
+ *           n_tokens <= capacity.  n_tokens == 0 is a no-op (k, v may be NULL).
+ * Keys get PolarQuant at b-1 bits plus QJL signs (computed on tcgen05
+ * tensor cores); values get PolarQuant at b bits.  Non-finite rows are
+ * encoded as zero vectors and counted in the context's status word
+ * (bitpolar NonFiniteInput), read with tq_get_status. */
+tq_status tq_encode_kv(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch,
+                       int n_kv_heads, int64_t n_tokens, int64_t stride_b, int64_t stride_h,
+                       int64_t stride_t, const tq_codes *codes, int64_t token_offset, void *stream);
+
+/* Pre-softmax scores of every query head against tokens [0, n_tokens) of its
+ * kv head, estimated from the packed keys and scaled by 1/sqrt(d) (bitpolar
+ * KvCacheCompressor::attention_scores):
+ *   s = [n_s <Pi q, C[idx]>/sqrt(d) + sqrt(pi/2)/m gamma <S Pi q, 2 bit - 1>] / sqrt(d).
+ *  q      : device float32 [codes->batch][n_q_heads][d].
+ *  scores : device float32 [codes->batch][n_q_heads][n_tokens].
+ * Query head j reads kv head j / (n_q_heads / n_kv_heads). */
+tq_status tq_attention_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, int n_q_heads,
+                              int64_t n_tokens, float *scores, void *stream);
+
+/* Reconstruct tokens [0, n_tokens) (bitpolar decode_values):
+ *   v_hat = n_s Pi^T C[idx]/sqrt(d),
+ *   k_hat = Pi^T (n_s C[idx]/sqrt(d) + sqrt(pi/2)/m gamma S^T (2 bit - 1)).
+ *  k_hat, v_hat : device float32 [batch][n_kv_heads][n_tokens][d]; either may be NULL. */
+tq_status tq_dequantize(tq_ctx *ctx, const tq_codes *codes, int64_t n_tokens, float *k_hat,
+                        float *v_hat, void *stream);
+
+/* Workspace bytes tq_decode_attention needs for this segment list. */
+size_t tq_decode_workspace_bytes(const tq_segment *segs, int n_segs, int batch, int n_q_heads,
+                                 int n_kv_heads);
+
+/* One decode step: for every sequence b and query head j,
+ *   out[b][j] = sum_t softmax_t(s_t) v_hat_t
+ * over the concatenation of all segments that sequence b attends to, with
+ * s_t the score of tq_attention_scores.  Split-K over tokens: each work item
+ * stages packed K/V tiles in shared memory, scores them through per-query
+ * lookup tables, keeps an online softmax and the value sum in registers,
+ * and shares each tile across the query heads of its kv-head group (GQA)
+ * and across all sequences of a shared segment; a second kernel merges the
+ * partials by log-sum-exp.
+ *  segs      : HOST array of n_segs (<= TQ_MAX_SEGMENTS) segments; every
+ *              sequence in [0, batch) must be covered by at least one.
+ *  q         : device [batch][n_q_heads][d] in q_dtype.
+ *  out       : device [batch][n_q_heads][d] in out_dtype.
+ *  workspace : device, >= tq_decode_workspace_bytes(...), 16-byte aligned;
+ *              contents on entry are ignored. */
+tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype,
+                              int batch, int n_q_heads, int n_kv_heads, void *out,
+                              tq_dtype out_dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronize `stream` and read the context's status word: the number of
+ * non-finite rows encoded so far, and device error flags (bit 0: a bounded
+ * wait inside a kernel gave up; its outputs for that tile are invalid). */
+tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags);
+
+/* Zero the status word (enqueued on `stream`). */
+tq_status tq_reset_status(tq_ctx *ctx, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *tq_status_string(tq_status s);
+
+/* Message of the last CUDA error seen by this thread's libtq calls (static storage). */
+const char *tq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H */

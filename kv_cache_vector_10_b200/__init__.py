@@ -1,0 +1,278 @@
+"""kv_cache_vector_10_b200 -- TurboQuant KV-cache codec and compressed-KV
+decode attention on NVIDIA B200 (sm_100a).
+
+This module is a thin ctypes binding over ``lib/libtq.so`` (C ABI declared in
+``include/tq.h``).  It only marshals arguments: tensors are passed as device
+pointers (``tensor.data_ptr()``) together with torch's current CUDA stream;
+every step of encode, scoring, dequantization and decode runs in the
+library's kernels.  There is no CPU fallback: importing on a machine without
+the built library raises, and calls on a non-sm_100 device fail with
+``TQ_ERR_DEVICE``.
+
+Names follow the C ABI (``tq_create``, ``tq_encode_kv``,
+``tq_attention_scores``, ``tq_decode_attention``, ``tq_dequantize``).  The
+``Codec`` / ``PackedCache`` / ``Segment`` classes are conveniences on top.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libtq.so")
+
+TQ_OK = 0
+TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
+TQ_KEYS, TQ_VALUES, TQ_BOTH = 0, 1, 2
+TQ_MAX_SEGMENTS = 64
+
+STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_DIM", 4: "TQ_ERR_BITS",
+                5: "TQ_ERR_ZERO_PROJ", 6: "TQ_ERR_PROJ", 7: "TQ_ERR_EMPTY", 8: "TQ_ERR_DIM_MISMATCH",
+                9: "TQ_ERR_WORKSPACE", 10: "TQ_ERR_ALIGN", 11: "TQ_ERR_CUDA", 12: "TQ_ERR_DEVICE",
+                13: "TQ_ERR_LIMIT"}
+
+EXPORTED = ["tq_create", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
+            "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
+            "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error"]
+
+
+class TQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = f"{where}: {STATUS_NAMES.get(code, code)}"
+        if code == 11 and _lib is not None:
+            msg += f" ({_lib.tq_last_cuda_error().decode()})"
+        super().__init__(msg)
+
+
+class tq_codes(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("batch", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("capacity", ctypes.c_int64)]
+
+
+class tq_segment(ctypes.Structure):
+    _fields_ = [("ctx", ctypes.c_void_p), ("codes", tq_codes), ("codes_batch", ctypes.c_int32),
+                ("first_seq", ctypes.c_int32), ("n_seqs", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_tokens", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_10_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    V, I, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
+    sig = {
+        "tq_create": (I, [I, I, I, U64, ctypes.POINTER(V)]),
+        "tq_destroy": (None, [V]),
+        "tq_ensure_heads": (I, [V, I]),
+        "tq_row_bytes": (I64, [V, I]),
+        "tq_packed_bytes": (SZ, [V, I, I, I64, I]),
+        "tq_encode_kv": (I, [V, V, V, I, I, I, I64, I64, I64, I64, ctypes.POINTER(tq_codes), I64, V]),
+        "tq_attention_scores": (I, [V, ctypes.POINTER(tq_codes), V, I, I64, V, V]),
+        "tq_dequantize": (I, [V, ctypes.POINTER(tq_codes), I64, V, V, V]),
+        "tq_decode_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
+        "tq_decode_attention": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V, SZ, V]),
+        "tq_get_status": (I, [V, V, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32)]),
+        "tq_reset_status": (I, [V, V]),
+        "tq_status_string": (ctypes.c_char_p, [I]),
+        "tq_last_cuda_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+lib = _lib
+
+
+def _check(code: int, where: str):
+    if code != TQ_OK:
+        raise TQError(code, where)
+
+
+def _stream(stream=None):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(dt) -> int:
+    import torch
+    return {torch.float32: TQ_F32, torch.float16: TQ_F16, torch.bfloat16: TQ_BF16}[dt]
+
+
+# ---------------------------------------------------------------- C ABI names
+
+def tq_create(head_dim: int, bits: int, projections: int, seed: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.tq_create(head_dim, bits, projections, seed & 0xFFFFFFFFFFFFFFFF, ctypes.byref(out)), "tq_create")
+    return out.value
+
+
+def tq_destroy(ctx: int) -> None:
+    _lib.tq_destroy(ctx)
+
+
+def tq_ensure_heads(ctx: int, n_heads: int) -> None:
+    _check(_lib.tq_ensure_heads(ctx, n_heads), "tq_ensure_heads")
+
+
+def tq_row_bytes(ctx: int, which: int) -> int:
+    return _lib.tq_row_bytes(ctx, which)
+
+
+def tq_packed_bytes(ctx: int, batch: int, n_kv_heads: int, capacity: int, which: int) -> int:
+    return _lib.tq_packed_bytes(ctx, batch, n_kv_heads, capacity, which)
+
+
+def tq_encode_kv(ctx: int, k, v, batch: int, n_kv_heads: int, n_tokens: int, codes: "PackedCache",
+                 token_offset: int = 0, stream=None) -> None:
+    """k, v: CUDA tensors [batch, n_kv_heads, n_tokens, d] (any strides with a
+    contiguous last dim); either may be None."""
+    ref = k if k is not None else v
+    sb, sh, st, sd = ref.stride()
+    if sd != 1:
+        raise ValueError("last dimension must be contiguous")
+    if k is not None and v is not None and (k.stride() != v.stride() or k.dtype != v.dtype):
+        raise ValueError("k and v must share dtype and strides")
+    c = codes.struct()
+    _check(_lib.tq_encode_kv(ctx, k.data_ptr() if k is not None else None, v.data_ptr() if v is not None else None,
+                             _dtype_code(ref.dtype), batch, n_kv_heads, n_tokens, sb, sh, st, ctypes.byref(c),
+                             token_offset, _stream(stream)), "tq_encode_kv")
+
+
+def tq_attention_scores(ctx: int, codes: "PackedCache", q, n_q_heads: int, n_tokens: int, scores, stream=None):
+    c = codes.struct()
+    _check(_lib.tq_attention_scores(ctx, ctypes.byref(c), q.data_ptr(), n_q_heads, n_tokens, scores.data_ptr(),
+                                    _stream(stream)), "tq_attention_scores")
+
+
+def tq_dequantize(ctx: int, codes: "PackedCache", n_tokens: int, k_hat=None, v_hat=None, stream=None):
+    c = codes.struct()
+    _check(_lib.tq_dequantize(ctx, ctypes.byref(c), n_tokens, k_hat.data_ptr() if k_hat is not None else None,
+                              v_hat.data_ptr() if v_hat is not None else None, _stream(stream)), "tq_dequantize")
+
+
+def _segment_array(segments):
+    arr = (tq_segment * len(segments))()
+    for i, s in enumerate(segments):
+        arr[i].ctx = s.codec.ctx
+        arr[i].codes = s.cache.struct()
+        arr[i].codes_batch = s.codes_batch
+        arr[i].first_seq = s.first_seq
+        arr[i].n_seqs = s.n_seqs
+        arr[i].n_tokens = s.n_tokens
+    return arr
+
+
+def tq_decode_workspace_bytes(segments, batch: int, n_q_heads: int, n_kv_heads: int) -> int:
+    arr = _segment_array(segments)
+    return _lib.tq_decode_workspace_bytes(arr, len(segments), batch, n_q_heads, n_kv_heads)
+
+
+def tq_decode_attention(segments, q, batch: int, n_q_heads: int, n_kv_heads: int, out, workspace, stream=None):
+    arr = _segment_array(segments)
+    _check(_lib.tq_decode_attention(arr, len(segments), q.data_ptr(), _dtype_code(q.dtype), batch, n_q_heads,
+                                    n_kv_heads, out.data_ptr(), _dtype_code(out.dtype), workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tq_decode_attention")
+
+
+def tq_get_status(ctx: int, stream=None):
+    n = ctypes.c_uint64()
+    f = ctypes.c_uint32()
+    _check(_lib.tq_get_status(ctx, _stream(stream), ctypes.byref(n), ctypes.byref(f)), "tq_get_status")
+    return n.value, f.value
+
+
+def tq_reset_status(ctx: int, stream=None):
+    _check(_lib.tq_reset_status(ctx, _stream(stream)), "tq_reset_status")
+
+
+# -------------------------------------------------------------- conveniences
+
+class Codec:
+    """A codec context: KvCacheConfig {head_dim, bits, projections, seed}."""
+
+    def __init__(self, head_dim: int, bits: int, projections: int, seed: int):
+        self.head_dim, self.bits, self.projections, self.seed = head_dim, bits, projections, seed
+        self.ctx = tq_create(head_dim, bits, projections, seed)
+        self.k_row_bytes = tq_row_bytes(self.ctx, TQ_KEYS)
+        self.v_row_bytes = tq_row_bytes(self.ctx, TQ_VALUES)
+
+    def close(self):
+        if self.ctx:
+            tq_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def alloc(self, batch: int, n_kv_heads: int, capacity: int, device="cuda") -> "PackedCache":
+        return PackedCache(self, batch, n_kv_heads, capacity, device)
+
+    def encode_kv(self, k, v, cache: "PackedCache", token_offset: int = 0, stream=None):
+        ref = k if k is not None else v
+        B, H, T, _ = ref.shape
+        tq_encode_kv(self.ctx, k, v, B, H, T, cache, token_offset, stream)
+
+    def attention_scores(self, cache, q, n_tokens: int, stream=None):
+        import torch
+        B, Hq, _ = q.shape
+        scores = torch.empty(B, Hq, n_tokens, dtype=torch.float32, device=q.device)
+        tq_attention_scores(self.ctx, cache, q.float().contiguous(), Hq, n_tokens, scores, stream)
+        return scores
+
+    def dequantize(self, cache, n_tokens: int, keys: bool = True, values: bool = True, stream=None):
+        import torch
+        shp = (cache.batch, cache.n_kv_heads, n_tokens, self.head_dim)
+        kh = torch.empty(shp, dtype=torch.float32, device=cache.k.device) if keys else None
+        vh = torch.empty(shp, dtype=torch.float32, device=cache.k.device) if values else None
+        tq_dequantize(self.ctx, cache, n_tokens, kh, vh, stream)
+        return kh, vh
+
+    def status(self, stream=None):
+        return tq_get_status(self.ctx, stream)
+
+
+class PackedCache:
+    """Device buffers of packed K and V rows, [batch][n_kv_heads][capacity][row bytes]."""
+
+    def __init__(self, codec: Codec, batch: int, n_kv_heads: int, capacity: int, device="cuda"):
+        import torch
+        if capacity % 16:
+            raise ValueError("capacity must be a multiple of 16")
+        self.codec, self.batch, self.n_kv_heads, self.capacity = codec, batch, n_kv_heads, capacity
+        self.k = torch.zeros(batch, n_kv_heads, capacity, codec.k_row_bytes, dtype=torch.uint8, device=device)
+        self.v = torch.zeros(batch, n_kv_heads, capacity, codec.v_row_bytes, dtype=torch.uint8, device=device)
+
+    def struct(self) -> tq_codes:
+        return tq_codes(self.k.data_ptr(), self.v.data_ptr(), self.batch, self.n_kv_heads, self.capacity)
+
+
+class Segment:
+    """Tokens [0, n_tokens) of batch slot `codes_batch` of `cache`, attended by
+    sequences [first_seq, first_seq + n_seqs)."""
+
+    def __init__(self, cache: PackedCache, n_tokens: int, first_seq: int, n_seqs: int = 1, codes_batch: int = 0):
+        self.cache, self.codec = cache, cache.codec
+        self.n_tokens, self.first_seq, self.n_seqs, self.codes_batch = n_tokens, first_seq, n_seqs, codes_batch
+
+
+def decode_attention(segments, q, n_kv_heads: int, out_dtype=None, workspace=None, stream=None):
+    """One decode step; q: [batch, n_q_heads, d] CUDA tensor."""
+    import torch
+    B, Hq, d = q.shape
+    out = torch.empty(B, Hq, d, dtype=out_dtype or q.dtype, device=q.device)
+    need = tq_decode_workspace_bytes(segments, B, Hq, n_kv_heads)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    tq_decode_attention(segments, q.contiguous(), B, Hq, n_kv_heads, out, workspace, stream)
+    return out

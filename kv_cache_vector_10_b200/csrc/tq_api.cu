@@ -1,0 +1,333 @@
+// tq_api.cu -- the C ABI of libtq: argument validation, context lifetime,
+// table upload and kernel dispatch.  No computation on the data path
+// happens on the host; every step runs in the kernels of tq_encode.cu,
+// tq_decode.cu and tq_aux.cu.
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "tq_internal.cuh"
+
+extern "C" void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t *sign_words,
+                                    uint16_t *S_bits);
+extern "C" int tq_host_codebook(int B, float *c, float *beta);
+
+tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch, int H,
+                           int64_t T, int64_t sb, int64_t sh, int64_t st, const tq_codes *codes,
+                           int64_t token_offset, cudaStream_t stream, int n_sms);
+tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, int Hq, int64_t T,
+                           float *scores, cudaStream_t stream);
+tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float *k_hat, float *v_hat,
+                            cudaStream_t stream);
+size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
+tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,
+                           int Hq, int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes,
+                           cudaStream_t stream, int n_sms);
+
+static thread_local char g_cuda_msg[256] = "no error";
+
+tq_status tq_check_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return TQ_OK;
+    snprintf(g_cuda_msg, sizeof(g_cuda_msg), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return TQ_ERR_CUDA;
+}
+
+static int device_sms(int dev) {
+    static int cached[64] = {0};
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+tq_status tq_check_device(const tq_ctx *ctx) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (ctx && dev != ctx->device) return TQ_ERR_DEVICE;
+    return TQ_OK;
+}
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_tiled() {
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+extern "C" {
+
+const char *tq_status_string(tq_status s) {
+    switch (s) {
+        case TQ_OK: return "TQ_OK";
+        case TQ_ERR_NULL: return "TQ_ERR_NULL";
+        case TQ_ERR_ZERO_DIM: return "TQ_ERR_ZERO_DIM";
+        case TQ_ERR_DIM: return "TQ_ERR_DIM";
+        case TQ_ERR_BITS: return "TQ_ERR_BITS";
+        case TQ_ERR_ZERO_PROJ: return "TQ_ERR_ZERO_PROJ";
+        case TQ_ERR_PROJ: return "TQ_ERR_PROJ";
+        case TQ_ERR_EMPTY: return "TQ_ERR_EMPTY";
+        case TQ_ERR_DIM_MISMATCH: return "TQ_ERR_DIM_MISMATCH";
+        case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE";
+        case TQ_ERR_ALIGN: return "TQ_ERR_ALIGN";
+        case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+        case TQ_ERR_DEVICE: return "TQ_ERR_DEVICE";
+        case TQ_ERR_LIMIT: return "TQ_ERR_LIMIT";
+    }
+    return "TQ_ERR_UNKNOWN";
+}
+
+const char *tq_last_cuda_error(void) { return g_cuda_msg; }
+
+tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_ctx **out) {
+    if (!out) return TQ_ERR_NULL;
+    *out = nullptr;
+    if (head_dim == 0) return TQ_ERR_ZERO_DIM;
+    if (head_dim != 64 && head_dim != 128) return TQ_ERR_DIM;
+    if (bits < 2 || bits > 5) return TQ_ERR_BITS;
+    if (projections == 0) return TQ_ERR_ZERO_PROJ;
+    if (projections < 32 || projections > 256 || projections % 32) return TQ_ERR_PROJ;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (prop.major != 10 || prop.minor != 0) return TQ_ERR_DEVICE;
+    tq_ctx *c = new tq_ctx();
+    std::memset(c, 0, sizeof(*c));
+    c->d = head_dim;
+    c->bits = bits;
+    c->m = projections;
+    c->BK = bits - 1;
+    c->BV = bits;
+    c->seed = seed;
+    c->device = dev;
+    c->LK = tq_host_codebook(c->BK, c->ck, c->bk);
+    c->LV = tq_host_codebook(c->BV, c->cv, c->bv);
+    tq_status st = tq_check_cuda(cudaMalloc(&c->d_status, 2 * sizeof(unsigned long long)));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMemset(c->d_status, 0, 2 * sizeof(unsigned long long)));
+    if (st != TQ_OK) {
+        tq_destroy(c);
+        return st;
+    }
+    *out = c;
+    return TQ_OK;
+}
+
+void tq_destroy(tq_ctx *ctx) {
+    if (!ctx) return;
+    cudaDeviceSynchronize();
+    cudaFree(ctx->d_signs);
+    cudaFree(ctx->d_S);
+    cudaFree(ctx->d_status);
+    delete ctx;
+}
+
+tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
+    if (!ctx) return TQ_ERR_NULL;
+    if (n_heads <= 0) return TQ_ERR_EMPTY;
+    if (n_heads > TQ_MAX_HEADS) return TQ_ERR_LIMIT;
+    if (n_heads <= ctx->heads_built) return TQ_OK;
+    tq_status st = tq_check_device(ctx);
+    if (st != TQ_OK) return st;
+    const int d = ctx->d, m = ctx->m;
+    std::vector<uint32_t> signs((size_t)n_heads * (d / 32));
+    std::vector<uint16_t> S((size_t)n_heads * m * d);
+    for (int h = 0; h < n_heads; ++h)
+        tq_host_head_tables(d, m, ctx->seed, h, &signs[(size_t)h * (d / 32)], &S[(size_t)h * m * d]);
+    uint32_t *nsig = nullptr;
+    __half *nS = nullptr;
+    st = tq_check_cuda(cudaMalloc(&nsig, signs.size() * 4));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMalloc(&nS, S.size() * 2));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nsig, signs.data(), signs.size() * 4, cudaMemcpyHostToDevice));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nS, S.data(), S.size() * 2, cudaMemcpyHostToDevice));
+    CUtensorMap map;
+    if (st == TQ_OK) {
+        PFN_encodeTiled enc = get_encode_tiled();
+        if (!enc) st = TQ_ERR_CUDA;
+        else {
+            cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n_heads * m};
+            cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+            cuuint32_t box[2] = {64, (cuuint32_t)m};
+            cuuint32_t es[2] = {1, 1};
+            CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, nS, dims, strides, box, es,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                snprintf(g_cuda_msg, sizeof(g_cuda_msg), "cuTensorMapEncodeTiled failed: %d", (int)r);
+                st = TQ_ERR_CUDA;
+            }
+        }
+    }
+    if (st != TQ_OK) {
+        cudaFree(nsig);
+        cudaFree(nS);
+        return st;
+    }
+    cudaDeviceSynchronize();   // no kernel may still read the old tables
+    cudaFree(ctx->d_signs);
+    cudaFree(ctx->d_S);
+    ctx->d_signs = nsig;
+    ctx->d_S = nS;
+    ctx->tmap_S = map;
+    ctx->heads_built = n_heads;
+    return TQ_OK;
+}
+
+int64_t tq_row_bytes(const tq_ctx *ctx, tq_which which) {
+    if (!ctx) return 0;
+    const int64_t kb = (int64_t)ctx->BK * ctx->d / 8 + ctx->m / 8 + 8;
+    const int64_t vb = (int64_t)ctx->BV * ctx->d / 8 + 4;
+    return which == TQ_KEYS ? kb : which == TQ_VALUES ? vb : kb + vb;
+}
+
+size_t tq_packed_bytes(const tq_ctx *ctx, int batch, int n_kv_heads, int64_t capacity, tq_which which) {
+    if (!ctx || batch < 0 || n_kv_heads < 0 || capacity < 0) return 0;
+    return (size_t)batch * n_kv_heads * capacity * tq_row_bytes(ctx, which);
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static tq_status check_codes(const tq_ctx *ctx, const tq_codes *codes, bool need_k, bool need_v) {
+    if (!codes) return TQ_ERR_NULL;
+    if ((need_k && !codes->k) || (need_v && !codes->v)) return TQ_ERR_NULL;
+    if (codes->batch <= 0 || codes->n_kv_heads <= 0) return TQ_ERR_EMPTY;
+    if (codes->capacity < 0 || codes->capacity % 16) return TQ_ERR_DIM_MISMATCH;
+    if ((need_k && !aligned16(codes->k)) || (need_v && !aligned16(codes->v))) return TQ_ERR_ALIGN;
+    (void)ctx;
+    return TQ_OK;
+}
+
+tq_status tq_encode_kv(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch, int n_kv_heads,
+                       int64_t n_tokens, int64_t stride_b, int64_t stride_h, int64_t stride_t,
+                       const tq_codes *codes, int64_t token_offset, void *stream) {
+    if (!ctx || !codes) return TQ_ERR_NULL;
+    if (batch <= 0 || n_kv_heads <= 0) return TQ_ERR_EMPTY;
+    if (n_tokens == 0 && token_offset >= 0 && token_offset <= codes->capacity) return TQ_OK;   // nothing to encode
+    if (!k && !v) return TQ_ERR_NULL;
+    if (dtype != TQ_F32 && dtype != TQ_F16 && dtype != TQ_BF16) return TQ_ERR_DIM_MISMATCH;
+    tq_status st = check_codes(ctx, codes, k != nullptr, v != nullptr);
+    if (st != TQ_OK) return st;
+    if (codes->batch != batch || codes->n_kv_heads != n_kv_heads) return TQ_ERR_DIM_MISMATCH;
+    if (n_tokens < 0 || token_offset < 0 || token_offset + n_tokens > codes->capacity) return TQ_ERR_DIM_MISMATCH;
+    const int64_t es = dtype == TQ_F32 ? 4 : 2;
+    if (stride_t < ctx->d || stride_b < 0 || stride_h < 0) return TQ_ERR_DIM_MISMATCH;
+    if ((stride_b * es) % 16 || (stride_h * es) % 16 || (stride_t * es) % 16) return TQ_ERR_ALIGN;
+    if ((k && !aligned16(k)) || (v && !aligned16(v))) return TQ_ERR_ALIGN;
+    if ((st = tq_check_device(ctx)) != TQ_OK) return st;
+    if ((st = tq_ensure_heads(ctx, n_kv_heads)) != TQ_OK) return st;
+    if (n_tokens == 0) return TQ_OK;
+    return tq_launch_encode(ctx, k, v, dtype, batch, n_kv_heads, n_tokens, stride_b, stride_h, stride_t, codes,
+                            token_offset, static_cast<cudaStream_t>(stream), device_sms(ctx->device));
+}
+
+tq_status tq_attention_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, int n_q_heads, int64_t n_tokens,
+                              float *scores, void *stream) {
+    if (!ctx || !q || !scores) return TQ_ERR_NULL;
+    tq_status st = check_codes(ctx, codes, true, false);
+    if (st != TQ_OK) return st;
+    if (n_q_heads <= 0) return TQ_ERR_EMPTY;
+    if (n_q_heads % codes->n_kv_heads) return TQ_ERR_DIM_MISMATCH;
+    if (n_tokens < 0 || n_tokens > codes->capacity) return TQ_ERR_DIM_MISMATCH;
+    if ((st = tq_check_device(ctx)) != TQ_OK) return st;
+    if ((st = tq_ensure_heads(ctx, codes->n_kv_heads)) != TQ_OK) return st;
+    if (n_tokens == 0) return TQ_OK;
+    return tq_launch_scores(ctx, codes, q, n_q_heads, n_tokens, scores, static_cast<cudaStream_t>(stream));
+}
+
+tq_status tq_dequantize(tq_ctx *ctx, const tq_codes *codes, int64_t n_tokens, float *k_hat, float *v_hat,
+                        void *stream) {
+    if (!ctx) return TQ_ERR_NULL;
+    if (!k_hat && !v_hat) return TQ_ERR_NULL;
+    tq_status st = check_codes(ctx, codes, k_hat != nullptr, v_hat != nullptr);
+    if (st != TQ_OK) return st;
+    if (n_tokens < 0 || n_tokens > codes->capacity) return TQ_ERR_DIM_MISMATCH;
+    if ((st = tq_check_device(ctx)) != TQ_OK) return st;
+    if ((st = tq_ensure_heads(ctx, codes->n_kv_heads)) != TQ_OK) return st;
+    if (n_tokens == 0) return TQ_OK;
+    return tq_launch_dequant(ctx, codes, n_tokens, k_hat, v_hat, static_cast<cudaStream_t>(stream));
+}
+
+static tq_status check_segments(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv) {
+    if (!segs) return TQ_ERR_NULL;
+    if (n_segs <= 0 || batch <= 0 || Hq <= 0 || Hkv <= 0) return TQ_ERR_EMPTY;
+    if (n_segs > TQ_MAX_SEGMENTS) return TQ_ERR_LIMIT;
+    if (Hq % Hkv) return TQ_ERR_DIM_MISMATCH;
+    std::vector<int> covered(batch, 0);
+    const int d = segs[0].ctx ? segs[0].ctx->d : 0;
+    for (int s = 0; s < n_segs; ++s) {
+        const tq_segment &g = segs[s];
+        if (!g.ctx) return TQ_ERR_NULL;
+        if (g.ctx->d != d) return TQ_ERR_DIM_MISMATCH;
+        tq_status st = check_codes(g.ctx, &g.codes, true, true);
+        if (st != TQ_OK) return st;
+        if (g.codes.n_kv_heads != Hkv) return TQ_ERR_DIM_MISMATCH;
+        if (g.codes_batch < 0 || g.codes_batch >= g.codes.batch) return TQ_ERR_DIM_MISMATCH;
+        if (g.n_tokens < 0 || g.n_tokens > g.codes.capacity) return TQ_ERR_DIM_MISMATCH;
+        if (g.n_seqs <= 0 || g.first_seq < 0 || g.first_seq + g.n_seqs > batch) return TQ_ERR_DIM_MISMATCH;
+        for (int b = g.first_seq; b < g.first_seq + g.n_seqs; ++b) covered[b] = 1;
+    }
+    for (int b = 0; b < batch; ++b)
+        if (!covered[b]) return TQ_ERR_DIM_MISMATCH;
+    return TQ_OK;
+}
+
+size_t tq_decode_workspace_bytes(const tq_segment *segs, int n_segs, int batch, int n_q_heads, int n_kv_heads) {
+    if (check_segments(segs, n_segs, batch, n_q_heads, n_kv_heads) != TQ_OK) return 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return tq_decode_ws(segs, n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
+}
+
+tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,
+                              int n_q_heads, int n_kv_heads, void *out, tq_dtype out_dtype, void *workspace,
+                              size_t ws_bytes, void *stream) {
+    if (!q || !out) return TQ_ERR_NULL;
+    tq_status st = check_segments(segs, n_segs, batch, n_q_heads, n_kv_heads);
+    if (st != TQ_OK) return st;
+    if ((q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) ||
+        (out_dtype != TQ_F32 && out_dtype != TQ_F16 && out_dtype != TQ_BF16))
+        return TQ_ERR_DIM_MISMATCH;
+    for (int s = 0; s < n_segs; ++s) {
+        tq_ctx *c = const_cast<tq_ctx *>(segs[s].ctx);
+        if ((st = tq_check_device(c)) != TQ_OK) return st;
+        if ((st = tq_ensure_heads(c, n_kv_heads)) != TQ_OK) return st;
+    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const size_t need = tq_decode_ws(segs, n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
+    if (!workspace || ws_bytes < need) return TQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return TQ_ERR_ALIGN;
+    return tq_launch_decode(segs, n_segs, q, q_dtype, batch, n_q_heads, n_kv_heads, out, out_dtype, workspace,
+                            ws_bytes, static_cast<cudaStream_t>(stream), device_sms(dev));
+}
+
+tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags) {
+    if (!ctx) return TQ_ERR_NULL;
+    unsigned long long h[2] = {0, 0};
+    tq_status st = tq_check_cuda(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(h, ctx->d_status, sizeof(h), cudaMemcpyDeviceToHost));
+    if (st != TQ_OK) return st;
+    if (nonfinite_rows) *nonfinite_rows = h[0];
+    if (error_flags) *error_flags = (uint32_t)h[1];
+    return TQ_OK;
+}
+
+tq_status tq_reset_status(tq_ctx *ctx, void *stream) {
+    if (!ctx) return TQ_ERR_NULL;
+    return tq_check_cuda(
+        cudaMemsetAsync(ctx->d_status, 0, 2 * sizeof(unsigned long long), static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

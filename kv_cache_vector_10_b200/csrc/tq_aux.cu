@@ -1,0 +1,367 @@
+// tq_aux.cu -- exact-path scores, dequantization, decode query preparation
+// and the log-sum-exp combine of split-K partials (sm_100a).
+//
+//  * Scores (bitpolar src/kv_cache.rs, KvCacheCompressor::attention_scores;
+//    pre-softmax, scaled by 1/sqrt(head_dim)), estimated from the codes:
+//      s = [n_s <q_rot, C[idx]>/sqrt(d) + sqrt(pi/2)/m gamma <S q_rot, 2b-1>] / sqrt(d),
+//    q_rot = Pi q (turboquant-plus-rs README, Architecture: TurboQuant
+//    inner-product estimator; QJL removes the bias).
+//  * Dequantization (bitpolar decode_values):
+//      v_hat = n_s Pi^T C[idx]/sqrt(d),
+//      k_hat = Pi^T (n_s C[idx]/sqrt(d) + sqrt(pi/2)/m gamma S^T (2b-1)).
+//  * Decode query preparation: q_rot and S q_rot per (segment, sequence,
+//    head), consumed by the split-K kernel's per-query lookup tables.
+//  * Combine: partials (running max, sum, unnormalised output) of all
+//    splits and segments of a (sequence, head) merged by log-sum-exp.
+#include "tq_decode.cuh"
+
+namespace {
+
+constexpr int AUX_THREADS = 128;
+
+// Block-wide: q_rot = H (D q) / sqrt(d) and sq = S q_rot, in shared memory.
+template <int D>
+__device__ void prep_query(const float *sq_in, const uint32_t *signs, const __half *S, int M, float *s_qr,
+                           float *s_sq) {
+    const int tid = threadIdx.x;
+    for (int j = tid; j < D; j += blockDim.x) {
+        const float x = sq_in[j];
+        s_qr[j] = ((signs[j / 32] >> (j % 32)) & 1) ? -x : x;
+    }
+    __syncthreads();
+    for (int len = 1; len < D; len <<= 1) {
+        for (int i = tid; i < D / 2; i += blockDim.x) {
+            const int j = (i / len) * 2 * len + (i % len);
+            const float a = s_qr[j], b = s_qr[j + len];
+            s_qr[j] = a + b;
+            s_qr[j + len] = a - b;
+        }
+        __syncthreads();
+    }
+    const float sc = rsqrtf((float)D);
+    for (int j = tid; j < D; j += blockDim.x) s_qr[j] *= sc;
+    __syncthreads();
+    for (int i = tid; i < M; i += blockDim.x) {
+        const __half *row = S + (int64_t)i * D;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D; ++j) acc = fmaf(__half2float(row[j]), s_qr[j], acc);
+        s_sq[i] = acc;
+    }
+    __syncthreads();
+}
+
+struct ScoresParams {
+    const uint8_t *kc;
+    const float *q;
+    float *scores;
+    const uint32_t *signs;
+    const __half *S;
+    int64_t capacity, T;
+    int Hq, Hkv, M, krow, bk;
+    float ck[16];
+};
+
+template <int D>
+__global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_constant__ ScoresParams p) {
+    __shared__ float s_qr[D];
+    __shared__ float s_sq[256];
+    const int j = blockIdx.y, b = blockIdx.z;
+    const int h = j / (p.Hq / p.Hkv);
+    prep_query<D>(p.q + ((int64_t)b * p.Hq + j) * D, p.signs + (int64_t)h * (D / 32), p.S + (int64_t)h * p.M * D,
+                  p.M, s_qr, s_sq);
+    const int64_t t = (int64_t)blockIdx.x * AUX_THREADS + threadIdx.x;
+    if (t >= p.T) return;
+    const uint8_t *row = p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) * p.krow;
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
+    float a = 0.f;
+    for (int jj = 0; jj < D; ++jj) {
+        int idx = 0;
+        for (int q = 0; q < p.bk; ++q) idx |= ((w[q * (D / 32) + jj / 32] >> (jj % 32)) & 1) << q;
+        a = fmaf(s_qr[jj], p.ck[idx], a);
+    }
+    const uint32_t *sg = w + p.bk * (D / 32);
+    float bq = 0.f;
+    for (int i = 0; i < p.M; ++i) bq += ((sg[i / 32] >> (i % 32)) & 1) ? s_sq[i] : -s_sq[i];
+    const float ns = __uint_as_float(sg[p.M / 32]);
+    const float gamma = __uint_as_float(sg[p.M / 32 + 1]);
+    const float isd = rsqrtf((float)D);
+    const float cq = 1.2533141373155003f / (float)p.M;   // sqrt(pi/2) / m
+    p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (ns * a * isd + cq * gamma * bq) * isd;
+}
+
+struct DequantParams {
+    const uint8_t *kc;
+    const uint8_t *vc;
+    float *kh;
+    float *vh;
+    const uint32_t *signs;
+    const __half *S;
+    int64_t capacity, T;
+    int H, M, krow, vrow, bk, bv;
+    float ck[16];
+    float cv[32];
+};
+
+template <int D>
+__device__ __forceinline__ void unrotate_store(float (&w)[D], const uint32_t *sg, float *dst) {
+#pragma unroll
+    for (int len = 1; len < D; len <<= 1)
+#pragma unroll
+        for (int i = 0; i < D; i += 2 * len)
+#pragma unroll
+            for (int j = i; j < i + len; ++j) {
+                const float a = w[j], b = w[j + len];
+                w[j] = a + b;
+                w[j + len] = a - b;
+            }
+    const float sc = rsqrtf((float)D);
+#pragma unroll
+    for (int j = 0; j < D; j += 4) {
+        float4 o;
+        o.x = ((sg[j / 32] >> (j % 32)) & 1) ? -w[j] * sc : w[j] * sc;
+        o.y = ((sg[(j + 1) / 32] >> ((j + 1) % 32)) & 1) ? -w[j + 1] * sc : w[j + 1] * sc;
+        o.z = ((sg[(j + 2) / 32] >> ((j + 2) % 32)) & 1) ? -w[j + 2] * sc : w[j + 2] * sc;
+        o.w = ((sg[(j + 3) / 32] >> ((j + 3) % 32)) & 1) ? -w[j + 3] * sc : w[j + 3] * sc;
+        *reinterpret_cast<float4 *>(dst + j) = o;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(AUX_THREADS) tq_dequant_kernel(const __grid_constant__ DequantParams p) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __half *sS = reinterpret_cast<__half *>(dsm);
+    const int h = blockIdx.y, b = blockIdx.z;
+    uint32_t sg[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) sg[i] = p.signs[(int64_t)h * (D / 32) + i];
+    if (p.kh) {
+        const __half *src = p.S + (int64_t)h * p.M * D;
+        for (int i = threadIdx.x; i < p.M * D / 8; i += blockDim.x)
+            reinterpret_cast<uint4 *>(sS)[i] = reinterpret_cast<const uint4 *>(src)[i];
+        __syncthreads();
+    }
+    const int64_t t = (int64_t)blockIdx.x * AUX_THREADS + threadIdx.x;
+    if (t >= p.T) return;
+    const int64_t rowi = ((int64_t)b * p.H + h) * p.capacity + t;
+    const int64_t outi = (((int64_t)b * p.H + h) * p.T + t) * D;
+    const float isd = rsqrtf((float)D);
+    if (p.vh) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(p.vc + rowi * p.vrow);
+        float x[D];
+        const float ns = __uint_as_float(w[p.bv * D / 32]);
+#pragma unroll
+        for (int j = 0; j < D; ++j) {
+            const int bit = p.bv * j;
+            uint32_t v = w[bit / 32] >> (bit % 32);
+            if ((bit % 32) + p.bv > 32) v |= w[bit / 32 + 1] << (32 - bit % 32);
+            x[j] = ns * p.cv[v & ((1u << p.bv) - 1)] * isd;
+        }
+        unrotate_store<D>(x, sg, p.vh + outi);
+    }
+    if (p.kh) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(p.kc + rowi * p.krow);
+        const uint32_t *sgn = w + p.bk * (D / 32);
+        const float ns = __uint_as_float(sgn[p.M / 32]);
+        const float gamma = __uint_as_float(sgn[p.M / 32 + 1]);
+        const float cq = 1.2533141373155003f / (float)p.M * gamma;
+        float x[D];
+#pragma unroll
+        for (int j = 0; j < D; ++j) {
+            int idx = 0;
+            for (int q = 0; q < p.bk; ++q) idx |= ((w[q * (D / 32) + j / 32] >> (j % 32)) & 1) << q;
+            x[j] = ns * p.ck[idx] * isd;
+        }
+        for (int i = 0; i < p.M; ++i) {
+            const float s = ((sgn[i / 32] >> (i % 32)) & 1) ? cq : -cq;
+            const __half2 *srow = reinterpret_cast<const __half2 *>(sS + i * D);
+#pragma unroll
+            for (int j = 0; j < D / 2; ++j) {
+                const float2 f = __half22float2(srow[j]);
+                x[2 * j] = fmaf(s, f.x, x[2 * j]);
+                x[2 * j + 1] = fmaf(s, f.y, x[2 * j + 1]);
+            }
+        }
+        unrotate_store<D>(x, sg, p.kh + outi);
+    }
+}
+
+// --------------------------------------------------------- decode helpers
+template <typename T>
+__device__ __forceinline__ float load_as_float(const void *p, int64_t i);
+template <>
+__device__ __forceinline__ float load_as_float<float>(const void *p, int64_t i) {
+    return static_cast<const float *>(p)[i];
+}
+template <>
+__device__ __forceinline__ float load_as_float<__half>(const void *p, int64_t i) {
+    return __half2float(static_cast<const __half *>(p)[i]);
+}
+template <>
+__device__ __forceinline__ float load_as_float<__nv_bfloat16>(const void *p, int64_t i) {
+    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+// One block per (segment, seq_local, head): prepared query [q_rot | S q_rot].
+template <int D, typename Tq>
+__global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
+    __shared__ float s_in[D];
+    __shared__ float s_qr[D];
+    __shared__ float s_sq[256];
+    int s = 0;
+    int64_t blk = blockIdx.x;
+    for (; s < P.n_segs; ++s) {
+        const int64_t n = (int64_t)P.seg[s].n_seqs * P.Hq;
+        if (blk < n) break;
+        blk -= n;
+    }
+    const SegDesc &g = P.seg[s];
+    const int seq_local = (int)(blk / P.Hq), j = (int)(blk % P.Hq);
+    const int seq = g.first_seq + seq_local;
+    const int h = j / P.G;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) s_in[i] = load_as_float<Tq>(q, ((int64_t)seq * P.Hq + j) * D + i);
+    __syncthreads();
+    prep_query<D>(s_in, g.signs + (int64_t)h * (D / 32), g.S + (int64_t)h * g.m * D, g.m, s_qr, s_sq);
+    float *dst = P.qprep + g.qprep_base + ((int64_t)seq_local * P.Hq + j) * (D + g.m);
+    for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = s_qr[i];
+    for (int i = threadIdx.x; i < g.m; i += blockDim.x) dst[D + i] = s_sq[i];
+}
+
+template <typename To>
+__device__ __forceinline__ void store_out(void *p, int64_t i, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(void *p, int64_t i, float v) {
+    static_cast<float *>(p)[i] = v;
+}
+template <>
+__device__ __forceinline__ void store_out<__half>(void *p, int64_t i, float v) {
+    static_cast<__half *>(p)[i] = __float2half_rn(v);
+}
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(void *p, int64_t i, float v) {
+    static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+}
+
+// One block of d threads per (sequence, head).
+template <int D, typename To>
+__global__ void __launch_bounds__(D) tq_combine_kernel(const __grid_constant__ DecodePlan P, void *out) {
+    const int b = blockIdx.x / P.Hq, j = blockIdx.x % P.Hq;
+    const int PF = tq_part_floats(D);
+    float mx = -INFINITY;
+    for (int s = 0; s < P.n_segs; ++s) {
+        const SegDesc &g = P.seg[s];
+        if (b < g.first_seq || b >= g.first_seq + g.n_seqs || g.T == 0) continue;
+        for (int sp = 0; sp < g.n_splits; ++sp) {
+            const float *pp = P.part + (g.part_base + ((int64_t)sp * g.n_seqs + (b - g.first_seq)) * P.Hq + j) * PF;
+            mx = fmaxf(mx, pp[0]);
+        }
+    }
+    float l = 0.f, o = 0.f;
+    if (mx != -INFINITY) {
+        for (int s = 0; s < P.n_segs; ++s) {
+            const SegDesc &g = P.seg[s];
+            if (b < g.first_seq || b >= g.first_seq + g.n_seqs || g.T == 0) continue;
+            for (int sp = 0; sp < g.n_splits; ++sp) {
+                const float *pp =
+                    P.part + (g.part_base + ((int64_t)sp * g.n_seqs + (b - g.first_seq)) * P.Hq + j) * PF;
+                if (pp[0] == -INFINITY) continue;
+                const float w = __expf(pp[0] - mx);
+                l = fmaf(w, pp[1], l);
+                o = fmaf(w, pp[4 + threadIdx.x], o);
+            }
+        }
+    }
+    store_out<To>(out, ((int64_t)b * P.Hq + j) * D + threadIdx.x, l > 0.f ? o / l : 0.f);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launches
+tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, int Hq, int64_t T, float *scores,
+                           cudaStream_t stream) {
+    ScoresParams p{};
+    p.kc = static_cast<const uint8_t *>(codes->k);
+    p.q = q;
+    p.scores = scores;
+    p.signs = ctx->d_signs;
+    p.S = ctx->d_S;
+    p.capacity = codes->capacity;
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = codes->n_kv_heads;
+    p.M = ctx->m;
+    p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
+    p.bk = ctx->BK;
+    for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
+    dim3 grid((unsigned)((T + AUX_THREADS - 1) / AUX_THREADS), (unsigned)Hq, (unsigned)codes->batch);
+    if (ctx->d == 128) tq_scores_kernel<128><<<grid, AUX_THREADS, 0, stream>>>(p);
+    else tq_scores_kernel<64><<<grid, AUX_THREADS, 0, stream>>>(p);
+    return tq_check_cuda(cudaGetLastError());
+}
+
+tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float *k_hat, float *v_hat,
+                            cudaStream_t stream) {
+    DequantParams p{};
+    p.kc = static_cast<const uint8_t *>(codes->k);
+    p.vc = static_cast<const uint8_t *>(codes->v);
+    p.kh = k_hat;
+    p.vh = v_hat;
+    p.signs = ctx->d_signs;
+    p.S = ctx->d_S;
+    p.capacity = codes->capacity;
+    p.T = T;
+    p.H = codes->n_kv_heads;
+    p.M = ctx->m;
+    p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
+    p.vrow = (int)tq_row_bytes(ctx, TQ_VALUES);
+    p.bk = ctx->BK;
+    p.bv = ctx->BV;
+    for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
+    for (int i = 0; i < ctx->LV; ++i) p.cv[i] = ctx->cv[i];
+    dim3 grid((unsigned)((T + AUX_THREADS - 1) / AUX_THREADS), (unsigned)codes->n_kv_heads, (unsigned)codes->batch);
+    const size_t smem = k_hat ? (size_t)ctx->m * ctx->d * 2 : 0;
+    cudaError_t e;
+    if (ctx->d == 128) {
+        e = cudaFuncSetAttribute(tq_dequant_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) tq_dequant_kernel<128><<<grid, AUX_THREADS, smem, stream>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(tq_dequant_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) tq_dequant_kernel<64><<<grid, AUX_THREADS, smem, stream>>>(p);
+    }
+    if (e != cudaSuccess) return tq_check_cuda(e);
+    return tq_check_cuda(cudaGetLastError());
+}
+
+cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cudaStream_t stream) {
+    int64_t blocks = 0;
+    for (int s = 0; s < P.n_segs; ++s) blocks += (int64_t)P.seg[s].n_seqs * P.Hq;
+    if (blocks == 0) return cudaSuccess;
+#define TQ_QPREP(DD, TT) tq_qprep_kernel<DD, TT><<<(unsigned)blocks, AUX_THREADS, 0, stream>>>(P, q)
+    if (P.d == 128) {
+        if (dt == TQ_F32) TQ_QPREP(128, float);
+        else if (dt == TQ_F16) TQ_QPREP(128, __half);
+        else TQ_QPREP(128, __nv_bfloat16);
+    } else {
+        if (dt == TQ_F32) TQ_QPREP(64, float);
+        else if (dt == TQ_F16) TQ_QPREP(64, __half);
+        else TQ_QPREP(64, __nv_bfloat16);
+    }
+#undef TQ_QPREP
+    return cudaGetLastError();
+}
+
+cudaError_t tq_launch_combine(const DecodePlan &P, void *out, tq_dtype dt, cudaStream_t stream) {
+    const unsigned blocks = (unsigned)(P.batch * P.Hq);
+#define TQ_COMB(DD, TT) tq_combine_kernel<DD, TT><<<blocks, DD, 0, stream>>>(P, out)
+    if (P.d == 128) {
+        if (dt == TQ_F32) TQ_COMB(128, float);
+        else if (dt == TQ_F16) TQ_COMB(128, __half);
+        else TQ_COMB(128, __nv_bfloat16);
+    } else {
+        if (dt == TQ_F32) TQ_COMB(64, float);
+        else if (dt == TQ_F16) TQ_COMB(64, __half);
+        else TQ_COMB(64, __nv_bfloat16);
+    }
+#undef TQ_COMB
+    return cudaGetLastError();
+}

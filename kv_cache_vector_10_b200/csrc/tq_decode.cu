@@ -1,0 +1,586 @@
+// tq_decode.cu -- split-K decode attention over the packed cache (sm_100a).
+//
+// For each (segment, kv-head, token split, query chunk) one CTA of 8 warps:
+//   * builds per-query lookup tables in shared memory.  Key scores need
+//     <q_rot, C[idx]> and <S q_rot, 2b-1> (turboquant-plus-rs README,
+//     Architecture: TurboQuant inner-product estimate).  The codebook is
+//     antisymmetric, so C[idx] is a sum over odd subsets A of the index bits
+//     of alpha_A * sigma_A with sigma_A = +-1 the parity of the bits in A
+//     (Walsh expansion).  Each sigma-plane, like the QJL sign plane, is a
+//     +-1 pattern, so its inner product with a vector is a sum of 16 byte
+//     lookups into a table LUT[g][byte] = sum_{i<8} v[8g+i] (2 bit_i - 1).
+//   * streams 32-token chunks of packed key and value rows into shared
+//     memory with bulk async copies (two buffers per warp);
+//   * scores two tokens per warp step (16 lanes per token, one byte group
+//     per lane), reduces the 16 partial sums by a transposing butterfly,
+//     keeps an online softmax per query, and accumulates the value sum in
+//     the rotated frame (4 coordinates per lane, centroid table lookups);
+//   * merges its warps, rotates the partial output back (Pi^T) and writes
+//     (max, sum, output) for the combine kernel.
+// Every query of a kv-head group (GQA) and every sequence of a shared
+// segment reads the same staged tile.
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "tq_decode.cuh"
+
+cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cudaStream_t stream);
+cudaError_t tq_launch_combine(const DecodePlan &P, void *out, tq_dtype dt, cudaStream_t stream);
+
+namespace {
+
+template <int QC>
+struct Vec;
+template <>
+struct Vec<1> {
+    using T = float;
+    __device__ static float get(const float &v, int) { return v; }
+    __device__ static void set(float &v, int, float x) { v = x; }
+};
+template <>
+struct Vec<2> {
+    using T = float2;
+    __device__ static float get(const float2 &v, int i) { return i == 0 ? v.x : v.y; }
+    __device__ static void set(float2 &v, int i, float x) { (i == 0 ? v.x : v.y) = x; }
+};
+template <>
+struct Vec<4> {
+    using T = float4;
+    __device__ static float get(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+    __device__ static void set(float4 &v, int i, float x) { (i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w) = x; }
+};
+
+// Odd subsets of BK index bits: XOR masks of the sigma-planes.
+__host__ __device__ constexpr int n_sigma_planes(int bk) { return bk == 1 ? 1 : bk == 2 ? 2 : bk == 3 ? 4 : 8; }
+__host__ __device__ constexpr uint32_t sigma_set(int bk, int s) {
+    // singletons first, then triples
+    return s < bk ? (1u << s)
+                  : (bk == 3 ? 7u : (s == 4 ? 7u : s == 5 ? 11u : s == 6 ? 13u : 14u));
+}
+
+// Table slot of (round, byte, half, slot): QC == 1 keeps one copy per half
+// warp so 32 lanes read 32 distinct banks; wider entries are read in
+// half/quarter-warp phases and need no copy.
+template <int QC>
+__device__ __forceinline__ int lut_slot(int round, int byte, int half, int slot) {
+    if constexpr (QC == 1) return ((round * 256 + byte) * 2 + half) * 16 + slot;
+    else return (round * 256 + byte) * 16 + slot;
+}
+template <int QC>
+__host__ __device__ constexpr int lut_entries(int rounds) {
+    return rounds * 256 * 16 * (QC == 1 ? 2 : 1);
+}
+
+template <int D, int BK, int BV, int QC>
+__global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const __grid_constant__ DecodePlan P) {
+    using VT = typename Vec<QC>::T;
+    constexpr int NGK = D / 8;                    // byte groups of an index plane
+    constexpr int RK = (NGK + 15) / 16;
+    constexpr int NP = n_sigma_planes(BK);
+    constexpr int CPL = D / 32;                   // value coordinates per lane
+    constexpr int LV = 1 << BV;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+
+    // ---- locate the work item
+    int s = 0;
+    int64_t item = blockIdx.x;
+    for (; s < P.n_segs; ++s) {
+        const SegDesc &g0 = P.seg[s];
+        const int64_t n = (int64_t)P.Hkv * g0.n_splits * g0.n_qchunks;
+        if (g0.bk == BK && item >= g0.item_base && item < g0.item_base + n) break;
+    }
+    if (s >= P.n_segs) return;
+    const SegDesc &g = P.seg[s];
+    const int64_t local = item - g.item_base;
+    const int qchunk = (int)(local % g.n_qchunks);
+    const int split = (int)((local / g.n_qchunks) % g.n_splits);
+    const int h = (int)(local / ((int64_t)g.n_qchunks * g.n_splits));
+    const int M = g.m;
+    const int NGS = M / 8, RS = (NGS + 15) / 16;
+    const int krow = g.krow, vrow = g.vrow;
+    const int64_t t_begin = (int64_t)split * g.split_len;
+    const int64_t t_end = std::min<int64_t>(g.T, t_begin + g.split_len);
+    const int nq = g.n_seqs * P.G;
+
+    // ---- shared memory carve-up
+    VT *lutq = reinterpret_cast<VT *>(smem_raw);
+    VT *luts = lutq + lut_entries<QC>(RK);
+    float *vtab = reinterpret_cast<float *>(luts + lut_entries<QC>(RS));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(vtab + 32);
+    uint8_t *stage = reinterpret_cast<uint8_t *>(bars + 2 * TQ_DEC_WARPS);
+    const int chunk_bytes = TQ_DEC_CHUNK * (krow + vrow);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = lane >> 4, slot = lane & 15;
+
+    if (tid < 32) vtab[tid] = g.vtab[tid < LV ? tid : 0];
+    if (tid == 0) {
+        for (int i = 0; i < 2 * TQ_DEC_WARPS; ++i) tqdev::mbar_init(&bars[i], 1);
+        tqdev::fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int64_t n_chunks = t_end > t_begin ? (t_end - t_begin + TQ_DEC_CHUNK - 1) / TQ_DEC_CHUNK : 0;
+    const uint8_t *kbase = g.kc + (int64_t)h * g.capacity * krow;
+    const uint8_t *vbase = g.vc + (int64_t)h * g.capacity * vrow;
+    auto issue = [&](int64_t ci, int buf) {
+        const int64_t tb = t_begin + ci * TQ_DEC_CHUNK;
+        const int64_t ntok = std::min<int64_t>(TQ_DEC_CHUNK, g.capacity - tb);
+        uint8_t *dk = stage + (warp * 2 + buf) * chunk_bytes;
+        uint8_t *dv = dk + TQ_DEC_CHUNK * krow;
+        tqdev::mbar_expect_tx(&bars[warp * 2 + buf], (uint32_t)(ntok * (krow + vrow)));
+        tqdev::bulk_load(dk, kbase + tb * krow, (uint32_t)(ntok * krow), &bars[warp * 2 + buf]);
+        tqdev::bulk_load(dv, vbase + tb * vrow, (uint32_t)(ntok * vrow), &bars[warp * 2 + buf]);
+    };
+    if (lane == 0) {
+        if (warp < n_chunks) issue(warp, 0);
+        if (warp + TQ_DEC_WARPS < n_chunks) issue(warp + TQ_DEC_WARPS, 1);
+    }
+
+    // ---- per-query lookup tables
+    const float *qp_base = P.qprep + g.qprep_base;
+    auto qvec = [&](int qq) -> const float * {
+        const int qi = qchunk * QC + qq;
+        if (qi >= nq) return nullptr;
+        const int seq_local = qi / P.G, j = h * P.G + qi % P.G;
+        return qp_base + ((int64_t)seq_local * P.Hq + j) * (D + M);
+    };
+    {
+        const int gslot = tid % 16, lo = tid / 16;   // fixed low nibble per thread
+        for (int kind = 0; kind < 2; ++kind) {
+            const int NG = kind == 0 ? NGK : NGS, R = kind == 0 ? RK : RS;
+            VT *lut = kind == 0 ? lutq : luts;
+            for (int r = 0; r < R; ++r) {
+                const int gg = r * 16 + gslot;
+                float lo_v[QC], hi_v[QC], hv[QC][4];
+#pragma unroll
+                for (int qq = 0; qq < QC; ++qq) {
+                    const float *v = qvec(qq);
+                    float vals[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) vals[i] = (v && gg < NG) ? v[(kind == 0 ? 0 : D) + 8 * gg + i] : 0.f;
+                    float a = 0.f, b = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        a += ((lo >> i) & 1) ? vals[i] : -vals[i];
+                        b -= vals[4 + i];
+                        hv[qq][i] = 2.f * vals[4 + i];
+                    }
+                    lo_v[qq] = a;
+                    hi_v[qq] = b;
+                }
+                int gray = 0;
+                for (int k = 0; k < 16; ++k) {
+                    if (k > 0) {
+                        const int f = __ffs(k) - 1;
+                        const bool up = !((gray >> f) & 1);
+                        gray ^= 1 << f;
+#pragma unroll
+                        for (int qq = 0; qq < QC; ++qq) hi_v[qq] += up ? hv[qq][f] : -hv[qq][f];
+                    }
+                    const int byte = lo | (gray << 4);
+                    VT e;
+#pragma unroll
+                    for (int qq = 0; qq < QC; ++qq) Vec<QC>::set(e, qq, lo_v[qq] + hi_v[qq]);
+                    lut[lut_slot<QC>(r, byte, 0, gslot)] = e;
+                    if constexpr (QC == 1) lut[lut_slot<QC>(r, byte, 1, gslot)] = e;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- main loop
+    float alpha[NP];
+#pragma unroll
+    for (int sp = 0; sp < NP; ++sp) alpha[sp] = g.alpha[sp];
+    const float inv_d = 1.f / (float)D;
+    const float cqs = 1.2533141373155003f / (float)M * rsqrtf((float)D);   // sqrt(pi/2)/m/sqrt(d)
+    const int off_sign = BK * (D / 8);
+    const int off_ns = off_sign + M / 8;
+    const int voff_ns = BV * D / 8;
+
+    float m_run[QC], l_lane[QC], o[QC][CPL];
+#pragma unroll
+    for (int qq = 0; qq < QC; ++qq) {
+        m_run[qq] = -INFINITY;
+        l_lane[qq] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) o[qq][c] = 0.f;
+    }
+    bool aborted = false;
+    for (int64_t k = 0;; ++k) {
+        const int64_t ci = warp + k * TQ_DEC_WARPS;
+        if (ci >= n_chunks) break;
+        const int buf = (int)(k & 1);
+        if (!tqdev::mbar_wait_bounded(&bars[warp * 2 + buf], (uint32_t)((k >> 1) & 1))) {
+            aborted = true;
+            break;
+        }
+        const uint8_t *sK = stage + (warp * 2 + buf) * chunk_bytes;
+        const uint8_t *sV = sK + TQ_DEC_CHUNK * krow;
+        const int64_t t0 = t_begin + ci * TQ_DEC_CHUNK;
+
+        float part[QC][16];
+#pragma unroll
+        for (int st = 0; st < 16; ++st) {
+            const uint8_t *kr = sK + (2 * st + half) * krow;
+            float am[QC], as[QC];
+#pragma unroll
+            for (int qq = 0; qq < QC; ++qq) am[qq] = as[qq] = 0.f;
+#pragma unroll
+            for (int r = 0; r < RK; ++r) {
+                const int gg = r * 16 + slot;
+                if (gg < NGK) {
+                    uint32_t pb[BK];
+#pragma unroll
+                    for (int pl = 0; pl < BK; ++pl) pb[pl] = kr[pl * (D / 8) + gg];
+#pragma unroll
+                    for (int sp = 0; sp < NP; ++sp) {
+                        uint32_t x = 0;
+#pragma unroll
+                        for (int pl = 0; pl < BK; ++pl)
+                            if ((sigma_set(BK, sp) >> pl) & 1) x ^= pb[pl];
+                        const VT e = lutq[lut_slot<QC>(r, (int)x, half, slot)];
+#pragma unroll
+                        for (int qq = 0; qq < QC; ++qq) am[qq] = fmaf(alpha[sp], Vec<QC>::get(e, qq), am[qq]);
+                    }
+                }
+            }
+            for (int r = 0; r < RS; ++r) {
+                const int gg = r * 16 + slot;
+                if (gg < NGS) {
+                    const VT e = luts[lut_slot<QC>(r, kr[off_sign + gg], half, slot)];
+#pragma unroll
+                    for (int qq = 0; qq < QC; ++qq) as[qq] += Vec<QC>::get(e, qq);
+                }
+            }
+            const float ns = *reinterpret_cast<const float *>(kr + off_ns);
+            const float gm = *reinterpret_cast<const float *>(kr + off_ns + 4);
+            const float a1 = ns * inv_d, a2 = gm * cqs;
+#pragma unroll
+            for (int qq = 0; qq < QC; ++qq) part[qq][st] = fmaf(a1, am[qq], a2 * as[qq]);
+        }
+        // transposing butterfly over the 16 lanes of each half-warp
+#pragma unroll
+        for (int qq = 0; qq < QC; ++qq) {
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1) {
+                const bool up = (slot & w) != 0;
+#pragma unroll
+                for (int i = 0; i < w; ++i) {
+                    const float send = up ? part[qq][i] : part[qq][i + w];
+                    const float keep = up ? part[qq][i + w] : part[qq][i];
+                    part[qq][i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                }
+            }
+        }
+        // this lane now holds the score of token 2*slot + half
+        const int tok = 2 * slot + half;
+        const bool valid = t0 + tok < t_end;
+        const float nsv = *reinterpret_cast<const float *>(sV + tok * vrow + voff_ns);
+        float w_tok[QC];
+#pragma unroll
+        for (int qq = 0; qq < QC; ++qq) {
+            const float sc = valid ? part[qq][0] : -INFINITY;
+            float cm = sc;
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, w));
+            const float mn = fmaxf(m_run[qq], cm);
+            const float corr = (mn == -INFINITY) ? 1.f : __expf(m_run[qq] - mn);
+            const float pr = valid ? __expf(sc - mn) : 0.f;
+            l_lane[qq] = fmaf(l_lane[qq], corr, pr);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[qq][c] *= corr;
+            m_run[qq] = mn;
+            w_tok[qq] = valid ? pr * nsv : 0.f;
+        }
+        // value accumulation, lane owns coordinates CPL*lane .. CPL*lane+CPL-1
+        const int vbit = BV * CPL * lane;
+        const int vw0 = vbit / 32, vsh = vbit % 32;
+#pragma unroll 4
+        for (int tau = 0; tau < TQ_DEC_CHUNK; ++tau) {
+            const int src = (tau & 1) * 16 + (tau >> 1);
+            const uint32_t *vr = reinterpret_cast<const uint32_t *>(sV + tau * vrow);
+            const uint32_t raw = __funnelshift_r(vr[vw0], vr[vw0 + 1], vsh);
+            float wq[QC];
+#pragma unroll
+            for (int qq = 0; qq < QC; ++qq) wq[qq] = __shfl_sync(0xffffffffu, w_tok[qq], src);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const float val = vtab[(raw >> (BV * c)) & (LV - 1)];
+#pragma unroll
+                for (int qq = 0; qq < QC; ++qq) o[qq][c] = fmaf(wq[qq], val, o[qq][c]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && ci + 2 * TQ_DEC_WARPS < n_chunks) {
+            tqdev::fence_proxy_async_smem();
+            issue(ci + 2 * TQ_DEC_WARPS, buf);
+        }
+    }
+    if (aborted && lane == 0)
+        atomicOr(reinterpret_cast<unsigned int *>(g.status + 1), TQ_FLAG_WAIT_TIMEOUT);
+
+    // ---- merge warps, rotate back, write partials
+    __syncthreads();
+    float *scr = reinterpret_cast<float *>(stage);              // [warp][QC][D + 2]
+#pragma unroll
+    for (int qq = 0; qq < QC; ++qq) {
+        float lt = l_lane[qq];
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, w);
+        float *row = scr + (warp * QC + qq) * (D + 2);
+        if (lane == 0) {
+            row[0] = aborted ? -INFINITY : m_run[qq];
+            row[1] = aborted ? 0.f : lt;
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) row[2 + CPL * lane + c] = aborted ? 0.f : o[qq][c];
+    }
+    __syncthreads();
+    float *acc = scr + TQ_DEC_WARPS * QC * (D + 2);             // [QC][D]
+    float *ml = acc + QC * D;                                    // [QC][2]
+    for (int i = tid; i < QC * D; i += blockDim.x) {
+        const int qq = i / D, j = i % D;
+        float mx = -INFINITY;
+        for (int w = 0; w < TQ_DEC_WARPS; ++w) mx = fmaxf(mx, scr[(w * QC + qq) * (D + 2)]);
+        float a = 0.f, l = 0.f;
+        if (mx != -INFINITY)
+            for (int w = 0; w < TQ_DEC_WARPS; ++w) {
+                const float *row = scr + (w * QC + qq) * (D + 2);
+                if (row[0] == -INFINITY) continue;
+                const float f = __expf(row[0] - mx);
+                a = fmaf(f, row[2 + j], a);
+                l = fmaf(f, row[1], l);
+            }
+        acc[qq * D + j] = a;
+        if (j == 0) {
+            ml[2 * qq] = mx;
+            ml[2 * qq + 1] = l;
+        }
+    }
+    __syncthreads();
+    // Pi^T with the 1/sqrt(d) of the value scale: out = D H acc / d
+    for (int len = 1; len < D; len <<= 1) {
+        for (int i = tid; i < QC * D / 2; i += blockDim.x) {
+            const int qq = i / (D / 2), ii = i % (D / 2);
+            const int j = (ii / len) * 2 * len + (ii % len);
+            float *a = acc + qq * D;
+            const float x = a[j], y = a[j + len];
+            a[j] = x + y;
+            a[j + len] = x - y;
+        }
+        __syncthreads();
+    }
+    const uint32_t *sg = g.signs + (int64_t)h * (D / 32);
+    for (int i = tid; i < QC * D; i += blockDim.x) {
+        const int qq = i / D, j = i % D;
+        const int qi = qchunk * QC + qq;
+        if (qi >= nq) continue;
+        const int seq_local = qi / P.G, jh = h * P.G + qi % P.G;
+        float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
+        float v = acc[qq * D + j] * inv_d;
+        if ((sg[j / 32] >> (j % 32)) & 1) v = -v;
+        dst[4 + j] = v;
+        if (j == 0) {
+            dst[0] = ml[2 * qq];
+            dst[1] = ml[2 * qq + 1];
+            dst[2] = 0.f;
+            dst[3] = 0.f;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ planning
+struct SegPlan {
+    int qc;
+    int n_qchunks, n_splits, split_len;
+    int64_t part_floats, qprep_floats;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sms, std::vector<SegPlan> &out) {
+    const int G = Hq / Hkv;
+    out.resize(n_segs);
+    int64_t work = 0;
+    for (int s = 0; s < n_segs; ++s) {
+        const int nq = segs[s].n_seqs * G;
+        SegPlan &p = out[s];
+        p.qc = nq >= 4 ? 4 : nq >= 2 ? 2 : 1;
+        p.n_qchunks = (nq + p.qc - 1) / p.qc;
+        work += segs[s].n_tokens * (int64_t)Hkv * p.n_qchunks;
+    }
+    const int64_t target_items = 2 * (int64_t)n_sms;
+    int64_t L = (work + target_items - 1) / std::max<int64_t>(target_items, 1);
+    L = std::max<int64_t>(L, TQ_DEC_SPLIT_UNIT);
+    const int d = segs[0].ctx->d;
+    for (int s = 0; s < n_segs; ++s) {
+        SegPlan &p = out[s];
+        const int64_t T = segs[s].n_tokens;
+        int64_t ns = std::max<int64_t>(1, (T + L - 1) / L);
+        int64_t sl = (T + ns - 1) / ns;
+        sl = std::max<int64_t>(TQ_DEC_SPLIT_UNIT, (sl + TQ_DEC_SPLIT_UNIT - 1) / TQ_DEC_SPLIT_UNIT * TQ_DEC_SPLIT_UNIT);
+        ns = std::max<int64_t>(1, (T + sl - 1) / sl);
+        p.n_splits = (int)ns;
+        p.split_len = (int)sl;
+        p.part_floats = (int64_t)ns * segs[s].n_seqs * Hq * tq_part_floats(d);
+        p.qprep_floats = (int64_t)segs[s].n_seqs * Hq * (d + segs[s].ctx->m);
+    }
+}
+
+template <int D, int BK, int BV, int QC>
+size_t decode_smem(int krow, int vrow, int M) {
+    using VT = typename Vec<QC>::T;
+    const int RK = (D / 8 + 15) / 16, RS = (M / 8 + 15) / 16;
+    size_t b = (size_t)(lut_entries<QC>(RK) + lut_entries<QC>(RS)) * sizeof(VT);
+    b += 32 * 4 + 2 * TQ_DEC_WARPS * 8;
+    const size_t stage = (size_t)TQ_DEC_WARPS * 2 * TQ_DEC_CHUNK * (krow + vrow);
+    const size_t merge = ((size_t)TQ_DEC_WARPS * QC * (D + 2) + QC * D + 2 * QC) * 4;
+    return b + std::max(stage, merge);
+}
+
+template <int D, int BK, int BV, int QC>
+cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vrow, int M, cudaStream_t stream) {
+    const size_t smem = decode_smem<D, BK, BV, QC>(krow, vrow, M);
+    auto kern = tq_decode_kernel<D, BK, BV, QC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)items, TQ_DEC_WARPS * 32, smem, stream>>>(P);
+    return cudaGetLastError();
+}
+
+template <int D, int QC>
+cudaError_t launch_decode_bits(int bits, const DecodePlan &P, int64_t items, int krow, int vrow, int M,
+                               cudaStream_t st) {
+    switch (bits) {
+        case 2: return launch_decode_t<D, 1, 2, QC>(P, items, krow, vrow, M, st);
+        case 3: return launch_decode_t<D, 2, 3, QC>(P, items, krow, vrow, M, st);
+        case 4: return launch_decode_t<D, 3, 4, QC>(P, items, krow, vrow, M, st);
+        case 5: return launch_decode_t<D, 4, 5, QC>(P, items, krow, vrow, M, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_decode_dim(int bits, int qc, const DecodePlan &P, int64_t items, int krow, int vrow, int M,
+                              cudaStream_t st) {
+    if (qc == 1) return launch_decode_bits<D, 1>(bits, P, items, krow, vrow, M, st);
+    if (qc == 2) return launch_decode_bits<D, 2>(bits, P, items, krow, vrow, M, st);
+    return launch_decode_bits<D, 4>(bits, P, items, krow, vrow, M, st);
+}
+
+// Walsh coefficients of an antisymmetric codebook over its index bits:
+// alpha_A = 2^-B sum_idx c[idx] prod_{p in A} (2 bit_p(idx) - 1).
+void sigma_alphas(const tq_ctx *ctx, float *alpha) {
+    const int B = ctx->BK, L = 1 << B;
+    const int NP = n_sigma_planes(B);
+    for (int sp = 0; sp < NP; ++sp) {
+        const uint32_t set = sigma_set(B, sp);
+        double a = 0.0;
+        for (int idx = 0; idx < L; ++idx) {
+            double prod = 1.0;
+            for (int p = 0; p < B; ++p)
+                if ((set >> p) & 1) prod *= ((idx >> p) & 1) ? 1.0 : -1.0;
+            a += (double)ctx->ck[idx] * prod;
+        }
+        alpha[sp] = (float)(a / L);
+    }
+}
+
+}  // namespace
+
+size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms) {
+    (void)batch;
+    std::vector<SegPlan> pl;
+    plan_segments(segs, n_segs, Hq, Hkv, n_sms, pl);
+    size_t q = 0, p = 0;
+    for (auto &x : pl) {
+        q += x.qprep_floats;
+        p += x.part_floats;
+    }
+    return align256(q * 4) + align256(p * 4);
+}
+
+tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch, int Hq,
+                           int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes, cudaStream_t stream,
+                           int n_sms) {
+    (void)ws_bytes;
+    std::vector<SegPlan> pl;
+    plan_segments(segs, n_segs, Hq, Hkv, n_sms, pl);
+    static DecodePlan P;   // large; filled per call on the host
+    P = DecodePlan{};
+    P.n_segs = n_segs;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.G = Hq / Hkv;
+    P.d = segs[0].ctx->d;
+    P.batch = batch;
+    size_t qtot = 0;
+    for (auto &x : pl) qtot += x.qprep_floats;
+    P.qprep = static_cast<float *>(ws);
+    P.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align256(qtot * 4));
+    int64_t qoff = 0, poff = 0;
+    for (int s = 0; s < n_segs; ++s) {
+        const tq_segment &sg = segs[s];
+        const tq_ctx *c = sg.ctx;
+        SegDesc &d = P.seg[s];
+        const int64_t krow = tq_row_bytes(c, TQ_KEYS), vrow = tq_row_bytes(c, TQ_VALUES);
+        d.kc = static_cast<const uint8_t *>(sg.codes.k) + (int64_t)sg.codes_batch * Hkv * sg.codes.capacity * krow;
+        d.vc = static_cast<const uint8_t *>(sg.codes.v) + (int64_t)sg.codes_batch * Hkv * sg.codes.capacity * vrow;
+        d.signs = c->d_signs;
+        d.S = c->d_S;
+        d.status = c->d_status;
+        d.capacity = sg.codes.capacity;
+        d.T = sg.n_tokens;
+        d.part_base = poff / tq_part_floats(P.d);
+        d.qprep_base = qoff;
+        d.first_seq = sg.first_seq;
+        d.n_seqs = sg.n_seqs;
+        d.krow = (int)krow;
+        d.vrow = (int)vrow;
+        d.m = c->m;
+        d.bk = c->BK;
+        d.bv = c->BV;
+        d.n_splits = pl[s].n_splits;
+        d.split_len = pl[s].split_len;
+        d.n_qchunks = pl[s].n_qchunks;
+        d.n_planes = n_sigma_planes(c->BK);
+        for (int i = 0; i < d.n_planes; ++i) d.plane_sets[i] = sigma_set(c->BK, i);
+        sigma_alphas(c, d.alpha);
+        for (int i = 0; i < 32; ++i) d.vtab[i] = i < c->LV ? c->cv[i] : 0.f;
+        qoff += pl[s].qprep_floats;
+        poff += pl[s].part_floats;
+    }
+    cudaError_t e = tq_launch_qprep(P, q, q_dtype, stream);
+    if (e != cudaSuccess) return tq_check_cuda(e);
+    // one launch per (bits, queries per CTA) group
+    std::vector<int> done(n_segs, 0);
+    for (int s0 = 0; s0 < n_segs; ++s0) {
+        if (done[s0]) continue;
+        const int bk = P.seg[s0].bk, qc = pl[s0].qc, m = P.seg[s0].m;
+        int64_t items = 0;
+        for (int s = 0; s < n_segs; ++s) {
+            SegDesc &d = P.seg[s];
+            if (!done[s] && d.bk == bk && pl[s].qc == qc && d.m == m) {
+                d.item_base = items;
+                items += (int64_t)Hkv * d.n_splits * d.n_qchunks;
+            } else if (!done[s]) {
+                d.item_base = -(int64_t)1 << 62;   // not in this launch
+            }
+        }
+        DecodePlan Pg = P;
+        for (int s = 0; s < n_segs; ++s)
+            if (done[s]) Pg.seg[s].item_base = -(int64_t)1 << 62;
+        for (int s = 0; s < n_segs; ++s)
+            if (!done[s] && P.seg[s].bk == bk && pl[s].qc == qc && P.seg[s].m == m) done[s] = 1;
+        if (items == 0) continue;
+        e = P.d == 128 ? launch_decode_dim<128>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
+                       : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);
+        if (e != cudaSuccess) return tq_check_cuda(e);
+    }
+    e = tq_launch_combine(P, out, out_dtype, stream);
+    return tq_check_cuda(e);
+}

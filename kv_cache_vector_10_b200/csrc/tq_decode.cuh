@@ -1,0 +1,43 @@
+// tq_decode.cuh -- work plan of the split-K decode, shared by the query
+// preparation, split-K and combine kernels.
+#pragma once
+
+#include "tq_internal.cuh"
+
+#define TQ_DEC_CHUNK 32       // tokens per warp chunk
+#define TQ_DEC_WARPS 8        // warps per CTA
+#define TQ_DEC_SPLIT_UNIT (TQ_DEC_CHUNK * TQ_DEC_WARPS)
+
+// One segment as the kernels see it.  Codes pointers already point at the
+// segment's batch slot: row (h, t) is at base + (h * capacity + t) * row.
+struct SegDesc {
+    const uint8_t *kc;
+    const uint8_t *vc;
+    const uint32_t *signs;     // [H_kv][d/32]
+    const __half *S;           // [H_kv][m][d]
+    unsigned long long *status;  // the segment context's status word
+    int64_t capacity;
+    int64_t T;
+    int64_t part_base;         // first partial slot of this segment
+    int64_t qprep_base;        // first float of this segment's prepared queries
+    int64_t item_base;         // first work item of this segment in its launch
+    int first_seq, n_seqs;
+    int krow, vrow, m, bk, bv;
+    int n_splits, split_len, n_qchunks;
+    int n_planes;              // odd subsets of the key index bits
+    uint32_t plane_sets[8];    // bit mask of index planes XOR-ed into sigma-plane s
+    float alpha[8];            // Walsh coefficient of sigma-plane s
+    float vtab[32];            // value centroids, indexed by code
+};
+
+struct DecodePlan {
+    SegDesc seg[TQ_MAX_SEGMENTS];
+    int n_segs;
+    int Hq, Hkv, G, d;
+    int batch;
+    float *qprep;              // prepared queries: [q_rot (d) | S q_rot (m)] per (segment, seq, head)
+    float *part;               // partial slots: [m, l, pad, pad, o (d)]
+};
+
+// Floats per partial slot.
+__host__ __device__ constexpr int tq_part_floats(int d) { return d + 4; }

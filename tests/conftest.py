@@ -25,3 +25,17 @@ def pytest_collection_modifyitems(config, items):
         for it in items:
             if "gpu" in it.keywords:
                 it.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # Build (or refresh) the in-tree CUDA library and the C oracle before any
+    # test module imports them.  Both are no-ops when up to date.
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("_tq_build", os.path.join(ROOT, "kv_cache_vector_10_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import oracle
+
+    oracle.build()
