@@ -50,18 +50,25 @@ struct EncodeParams {
     TqBook book;
 };
 
+// Row loaders.  The rotation's random signs are applied while converting:
+// `sm` holds, per 32-bit input word, a mask with the sign bit of every
+// element that D flips (bits 15/31 for 16-bit types, bit 31 for fp32).
 template <typename Tin>
 struct Loader;
 
 template <>
 struct Loader<float> {
     template <int D>
-    __device__ static void load(const float *src, float (&x)[D]) {
-        const float4 *p = reinterpret_cast<const float4 *>(src);
+    __device__ static void load(const float *src, const uint32_t *sm, float (&x)[D]) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src);
+        const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
         for (int i = 0; i < D / 4; ++i) {
-            float4 q = __ldg(p + i);
-            x[4 * i] = q.x; x[4 * i + 1] = q.y; x[4 * i + 2] = q.z; x[4 * i + 3] = q.w;
+            const uint4 q = __ldg(p + i), f = m[i];
+            x[4 * i] = __uint_as_float(q.x ^ f.x);
+            x[4 * i + 1] = __uint_as_float(q.y ^ f.y);
+            x[4 * i + 2] = __uint_as_float(q.z ^ f.z);
+            x[4 * i + 3] = __uint_as_float(q.w ^ f.w);
         }
     }
 };
@@ -69,18 +76,19 @@ struct Loader<float> {
 template <>
 struct Loader<__half> {
     template <int D>
-    __device__ static void load(const __half *src, float (&x)[D]) {
+    __device__ static void load(const __half *src, const uint32_t *sm, float (&x)[D]) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src);
+        const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
-            uint4 q = __ldg(p + i);
-            uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            const uint4 q = __ldg(p + i), f = m[i];
+            const uint32_t w[4] = {q.x ^ f.x, q.y ^ f.y, q.z ^ f.z, q.w ^ f.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                __half2 h2 = *reinterpret_cast<__half2 *>(&w[e]);
-                float2 f = __half22float2(h2);
-                x[8 * i + 2 * e] = f.x;
-                x[8 * i + 2 * e + 1] = f.y;
+                const float2 v = __half22float2(__halves2half2(__ushort_as_half((unsigned short)(w[e] & 0xFFFFu)),
+                                                               __ushort_as_half((unsigned short)(w[e] >> 16))));
+                x[8 * i + 2 * e] = v.x;
+                x[8 * i + 2 * e + 1] = v.y;
             }
         }
     }
@@ -89,12 +97,13 @@ struct Loader<__half> {
 template <>
 struct Loader<__nv_bfloat16> {
     template <int D>
-    __device__ static void load(const __nv_bfloat16 *src, float (&x)[D]) {
+    __device__ static void load(const __nv_bfloat16 *src, const uint32_t *sm, float (&x)[D]) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src);
+        const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
-            uint4 q = __ldg(p + i);
-            uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            const uint4 q = __ldg(p + i), f = m[i];
+            const uint32_t w[4] = {q.x ^ f.x, q.y ^ f.y, q.z ^ f.z, q.w ^ f.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 x[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
@@ -103,6 +112,23 @@ struct Loader<__nv_bfloat16> {
         }
     }
 };
+
+template <typename Tin>
+constexpr int mask_words(int D) { return sizeof(Tin) == 4 ? D : D / 2; }
+
+// Per-head input sign masks: word w covers the elements stored in input
+// word w.
+template <typename Tin, int D>
+__device__ void build_sign_masks(const uint32_t *signs, uint32_t *sm) {
+    for (int w = threadIdx.x; w < mask_words<Tin>(D); w += blockDim.x) {
+        if constexpr (sizeof(Tin) == 4) {
+            sm[w] = ((signs[w / 32] >> (w % 32)) & 1u) << 31;
+        } else {
+            const int j = 2 * w;
+            sm[w] = (((signs[j / 32] >> (j % 32)) & 1u) << 15) | (((signs[(j + 1) / 32] >> ((j + 1) % 32)) & 1u) << 31);
+        }
+    }
+}
 
 // Norm of a row held in registers.  Returns -1 for a row with a non-finite
 // value, 0 for an all-zero row.  Rows whose sum of squares over- or
@@ -132,16 +158,9 @@ __device__ __forceinline__ float row_norm(const float (&x)[D]) {
     return mx * sqrtf(acc);
 }
 
-// u <- H (D x) in place: sign flip from bit masks, then the butterflies.
+// u <- H u in place (the signs were applied by the loader).
 template <int D>
-__device__ __forceinline__ void rotate_unnormalised(float (&x)[D], const uint32_t *sw) {
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) {
-        const uint32_t m = sw[w];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            x[32 * w + i] = __uint_as_float(__float_as_uint(x[32 * w + i]) ^ ((m << (31 - i)) & 0x80000000u));
-    }
+__device__ __forceinline__ void fwht_inplace(float (&x)[D]) {
 #pragma unroll
     for (int len = 1; len < D; len <<= 1) {
 #pragma unroll
@@ -156,32 +175,55 @@ __device__ __forceinline__ void rotate_unnormalised(float (&x)[D], const uint32_
     }
 }
 
-// Number of positive boundaries at or below |u| (boundaries pre-scaled by n)
-// and the magnitude of the selected centroid.
+// Magnitude index of a = |u| among the HB cells of the positive half of the
+// codebook: the number of positive boundaries nb[k] (pre-scaled by n) with
+// a >= nb[k], found by a branchless binary search (bit k of the result is
+// decided at level k from the top).
 template <int HB>
-__device__ __forceinline__ int quant_mag(float a, const float (&nb)[16], const float *mag, float &cm) {
-    int cnt = 0;
-    cm = mag[0];
-#pragma unroll
-    for (int k = 0; k < HB - 1; ++k) {
-        const bool t = a >= nb[k];
-        cnt += t ? 1 : 0;
-        cm = t ? mag[k + 1] : cm;
+__device__ __forceinline__ uint32_t mag_index(float a, const float (&nb)[16]) {
+    if constexpr (HB == 1) {
+        return 0u;
+    } else if constexpr (HB == 2) {
+        return a >= nb[0] ? 1u : 0u;
+    } else if constexpr (HB == 4) {
+        const bool t1 = a >= nb[1];
+        const bool t0 = a >= (t1 ? nb[2] : nb[0]);
+        return (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    } else if constexpr (HB == 8) {
+        const bool t2 = a >= nb[3];
+        const bool t1 = a >= (t2 ? nb[5] : nb[1]);
+        const float b0 = t2 ? (t1 ? nb[6] : nb[4]) : (t1 ? nb[2] : nb[0]);
+        const bool t0 = a >= b0;
+        return (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+    } else {
+        const bool t3 = a >= nb[7];
+        const bool t2 = a >= (t3 ? nb[11] : nb[3]);
+        const bool t1 = a >= (t3 ? (t2 ? nb[13] : nb[9]) : (t2 ? nb[5] : nb[1]));
+        const float b0 = t3 ? (t2 ? (t1 ? nb[14] : nb[12]) : (t1 ? nb[10] : nb[8]))
+                            : (t2 ? (t1 ? nb[6] : nb[4]) : (t1 ? nb[2] : nb[0]));
+        const bool t0 = a >= b0;
+        return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
     }
-    return cnt;
 }
 
 template <int D, int BK, int BV, typename Tin>
 __global__ void __launch_bounds__(ENC_GROUP, 1)
     tq_encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmapS) {
-    constexpr int LK = 1 << BK, HK = LK / 2;
-    constexpr int LV = 1 << BV, HV = LV / 2;
+    constexpr int HK = (1 << BK) / 2;
+    constexpr int HV = (1 << BV) / 2;
     constexpr int NW = D / 32;                 // 32-bit words per bit plane
     constexpr int ATOM = ENC_GROUP * 128;      // bytes of one 128-row x 128-byte swizzle column
     constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
-    (void)LK; (void)LV;
+    constexpr int MW = mask_words<Tin>(D);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // misc region [0, 1024): sign masks, centroid magnitudes, barriers
+    uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // [MW] (<= 512 B)
+    float *s_mag = reinterpret_cast<float *>(smem + 512);                   // [16] magnitudes
+    float *s_mag2 = s_mag + 16;                                             // [16] squared
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);              // [0] S loaded, [1] MMA done
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
+    int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
     const int tid = threadIdx.x, warp = tid / 32;
     // Blocks [0, k_blocks) encode keys, the rest encode values.
     const bool is_key = blockIdx.x < p.k_blocks;
@@ -190,19 +232,23 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
     const int head = (int)(bh % p.H);
     const int64_t b = bh / p.H;
     const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_GROUP;
-    uint32_t sw[NW];
-#pragma unroll
-    for (int w = 0; w < NW; ++w) sw[w] = __ldg(p.signs + (int64_t)head * NW + w);
+    build_sign_masks<Tin, D>(p.signs + (int64_t)head * NW, s_mask);
+    if (tid < 16) {
+        const float mg = is_key ? (tid < HK ? p.book.kmag[tid] : 0.f) : (tid < HV ? p.book.vmag[tid] : 0.f);
+        s_mag[tid] = mg;
+        s_mag2[tid] = mg * mg;
+    }
     const Tin *src = reinterpret_cast<const Tin *>(is_key ? p.k : p.v) + b * p.sb + (int64_t)head * p.sh;
 
     if (!is_key) {
+        __syncthreads();
         // ------------------------------------------------------- values
         constexpr int VW = BV * D / 32;
         for (int tile = 0; tile < ENC_TILES; ++tile) {
             const int64_t t = tb0 + tile * ENC_GROUP + tid;
             if (t >= p.T) break;
             float x[D];
-            Loader<Tin>::template load<D>(src + t * p.st, x);
+            Loader<Tin>::template load<D>(src + t * p.st, s_mask, x);
             const float n = row_norm<D>(x);
             if (n < 0.f) atomicAdd(&p.status[0], 1ull);
             uint32_t f[VW];
@@ -217,17 +263,16 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
                     if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= (uint32_t)HV >> (32 - bit % 32);
                 }
             } else {
-                rotate_unnormalised<D>(x, sw);
+                fwht_inplace<D>(x);
                 float nb[16];
 #pragma unroll
                 for (int k2 = 0; k2 < HV - 1; ++k2) nb[k2] = n * p.book.vpb[k2];
                 float c2 = 0.f;
 #pragma unroll
                 for (int j = 0; j < D; ++j) {
-                    float cm;
-                    const int cnt = quant_mag<HV>(fabsf(x[j]), nb, p.book.vmag, cm);
-                    const uint32_t idx = (uint32_t)(x[j] >= 0.f ? HV + cnt : HV - 1 - cnt);
-                    c2 = fmaf(cm, cm, c2);
+                    const uint32_t cnt = mag_index<HV>(fabsf(x[j]), nb);
+                    const uint32_t idx = x[j] < 0.f ? (uint32_t)(HV - 1) - cnt : (uint32_t)HV + cnt;
+                    c2 += s_mag2[cnt];
                     const int bit = BV * j;
                     f[bit / 32] |= idx << (bit % 32);
                     if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
@@ -244,11 +289,8 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
 
     // ------------------------------------------------------------- keys
     const int M = p.M;
-    uint8_t *sS = smem;                                   // [D/64][M rows][128 B]
-    uint8_t *sA = smem + (D / 64) * M * 128;              // [pass][D/64][128 rows][128 B]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sA + 2 * A_BYTES);  // [0] S loaded, [1] MMA done
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
-    int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
+    uint8_t *sS = smem + 1024;                            // [D/64][M rows][128 B]
+    uint8_t *sA = sS + (D / 64) * M * 128;                // [pass][D/64][128 rows][128 B]
     const uint32_t tmem_cols = M <= 128 ? 128u : 256u;
     if (tid == 0) {
         tqdev::mbar_init(&bars[0], 1);
@@ -278,7 +320,7 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
             float x[D];
             float n = 0.f;
             if (valid) {
-                Loader<Tin>::template load<D>(src + t * p.st, x);
+                Loader<Tin>::template load<D>(src + t * p.st, s_mask, x);
                 n = row_norm<D>(x);
                 if (n < 0.f) atomicAdd(&p.status[0], 1ull);
             }
@@ -298,41 +340,53 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
                         for (int w = 0; w < NW; ++w) dst[q * NW + w] = ((HK >> q) & 1) ? 0xFFFFFFFFu : 0u;
                 }
             } else {
-                rotate_unnormalised<D>(x, sw);
+                fwht_inplace<D>(x);
                 float nb[16];
 #pragma unroll
                 for (int k2 = 0; k2 < HK - 1; ++k2) nb[k2] = n * p.book.kpb[k2];
-                // pass 1: squared norm of the selected centroids
+                // pass 1: magnitude and sign bits of every index, squared centroid norm
                 float c2 = 0.f;
-#pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    float cm;
-                    quant_mag<HK>(fabsf(x[j]), nb, p.book.kmag, cm);
-                    c2 = fmaf(cm, cm, c2);
-                }
-                ns = n * sqrtf((float)D / c2);
-                // pass 2: index planes and the residual u - n_s C[idx]
-                float e2 = 0.f;
+                uint32_t *dst = reinterpret_cast<uint32_t *>(rowp);
+                uint32_t mb[BK > 1 ? BK - 1 : 1][NW];
 #pragma unroll
                 for (int w = 0; w < NW; ++w) {
-                    uint32_t pl[BK];
+                    uint32_t negw = 0u;
 #pragma unroll
-                    for (int q = 0; q < BK; ++q) pl[q] = 0u;
+                    for (int q = 0; q < BK - 1; ++q) mb[q][w] = 0u;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int j = 32 * w + i;
-                        float cm;
-                        const int cnt = quant_mag<HK>(fabsf(x[j]), nb, p.book.kmag, cm);
-                        const bool pos = x[j] >= 0.f;
-                        const int idx = pos ? HK + cnt : HK - 1 - cnt;
+                        const float u = x[32 * w + i];
+                        const uint32_t cnt = mag_index<HK>(fabsf(u), nb);
+                        negw |= (__float_as_uint(u) >> 31) << i;
 #pragma unroll
-                        for (int q = 0; q < BK; ++q) pl[q] |= (uint32_t)((idx >> q) & 1) << i;
-                        x[j] = fmaf(-ns, pos ? cm : -cm, x[j]);
-                        e2 = fmaf(x[j], x[j], e2);
+                        for (int q = 0; q < BK - 1; ++q) mb[q][w] |= ((cnt >> q) & 1u) << i;
+                        c2 += s_mag2[cnt];
                     }
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(rowp);
+                    // ascending index: top bit = non-negative, low bits = magnitude
+                    // index, complemented for negative values
 #pragma unroll
-                    for (int q = 0; q < BK; ++q) dst[q * NW + w] = pl[q];
+                    for (int q = 0; q < BK - 1; ++q) dst[q * NW + w] = mb[q][w] ^ negw;
+                    dst[(BK - 1) * NW + w] = ~negw;
+                }
+                ns = n * sqrtf((float)D / c2);
+                // Hide the packed words' provenance so the compiler re-extracts
+                // the bits instead of keeping 128 indices live across passes.
+#pragma unroll
+                for (int q = 0; q < BK - 1; ++q)
+#pragma unroll
+                    for (int w = 0; w < NW; ++w) asm volatile("" : "+r"(mb[q][w]));
+                // pass 2: residual u - n_s C[idx], the magnitude index read back
+                // from the packed bits
+                float e2 = 0.f;
+#pragma unroll
+                for (int j = 0; j < D; ++j) {
+                    const float u = x[j];
+                    uint32_t cnt = 0u;
+#pragma unroll
+                    for (int q = 0; q < BK - 1; ++q) cnt |= ((mb[q][j / 32] >> (j % 32)) & 1u) << q;
+                    const float c = copysignf(s_mag[cnt], u);
+                    x[j] = fmaf(-ns, c, u);
+                    e2 = fmaf(x[j], x[j], e2);
                 }
                 gamma = sqrtf(e2) * inv_sqrt_d;
                 // pass 3: |e| = sqrt(d) scaled residual as binary16 hi + lo, swizzled K-major
@@ -420,7 +474,7 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
 
 template <int D, int BK, int BV, typename Tin>
 cudaError_t launch_t(const EncodeParams &p, const CUtensorMap &map, int grid, cudaStream_t s) {
-    const size_t smem = 1024 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_GROUP * 128 + 64;
+    const size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_GROUP * 128;
     auto kern = tq_encode_kernel<D, BK, BV, Tin>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
