@@ -328,7 +328,10 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
         e = cudaFuncSetAttribute(tq_dequant_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess) tq_dequant_kernel<64><<<grid, AUX_THREADS, smem, stream>>>(p);
     }
-    if (e != cudaSuccess) return tq_check_cuda(e);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return tq_check_cuda(e);
+    }
     return tq_check_cuda(cudaGetLastError());
 }
 

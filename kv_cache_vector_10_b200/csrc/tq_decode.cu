@@ -14,7 +14,9 @@
 //   * scores two tokens per warp step (16 lanes per token, one byte group
 //     per lane), reduces the 16 partial sums by a transposing butterfly,
 //     keeps an online softmax per query, and accumulates the value sum in
-//     the rotated frame (4 coordinates per lane, centroid table lookups);
+//     the rotated frame with the same layout (8 coordinates of one token per
+//     lane per step; two codes per lookup in a replicated pair table; packed
+//     fp32x2 multiply-adds);
 //   * merges its warps, rotates the partial output back (Pi^T) and writes
 //     (max, sum, output) for the combine kernel.
 // Every query of a kv-head group (GQA) and every sequence of a shared
@@ -72,14 +74,23 @@ __host__ __device__ constexpr int lut_entries(int rounds) {
     return rounds * 256 * 16 * (QC == 1 ? 2 : 1);
 }
 
+// Value pair table: entry e = two consecutive B_V-bit codes (low code in the
+// low bits) -> the two centroids.  VCOPIES copies, indexed by the lane's slot,
+// keep every half-warp access conflict-free.
+template <int BV>
+__host__ __device__ constexpr int vpair_copies() { return BV <= 4 ? 16 : 1; }
+template <int BV>
+__host__ __device__ constexpr int vpair_entries() { return 1 << (2 * BV); }
+
 template <int D, int BK, int BV, int QC>
 __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const __grid_constant__ DecodePlan P) {
     using VT = typename Vec<QC>::T;
-    constexpr int NGK = D / 8;                    // byte groups of an index plane
+    constexpr int NGK = D / 8;                    // byte groups of an index plane = value slots
     constexpr int RK = (NGK + 15) / 16;
     constexpr int NP = n_sigma_planes(BK);
-    constexpr int CPL = D / 32;                   // value coordinates per lane
-    constexpr int LV = 1 << BV;
+    constexpr int VPB = 2 * BV;                   // bits of a value pair
+    constexpr int VCOP = vpair_copies<BV>();
+    static_assert(D == 64 || D == 128, "head_dim");
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
     // ---- locate the work item
@@ -106,15 +117,18 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     // ---- shared memory carve-up
     VT *lutq = reinterpret_cast<VT *>(smem_raw);
     VT *luts = lutq + lut_entries<QC>(RK);
-    float *vtab = reinterpret_cast<float *>(luts + lut_entries<QC>(RS));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(vtab + 32);
+    float2 *vlut = reinterpret_cast<float2 *>(luts + lut_entries<QC>(RS));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(vlut + vpair_entries<BV>() * VCOP);
     uint8_t *stage = reinterpret_cast<uint8_t *>(bars + 2 * TQ_DEC_WARPS);
     const int chunk_bytes = TQ_DEC_CHUNK * (krow + vrow);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int half = lane >> 4, slot = lane & 15;
 
-    if (tid < 32) vtab[tid] = g.vtab[tid < LV ? tid : 0];
+    for (int i = tid; i < vpair_entries<BV>() * VCOP; i += blockDim.x) {
+        const int e = i / VCOP;
+        vlut[i] = make_float2(g.vtab[e & ((1 << BV) - 1)], g.vtab[e >> BV]);
+    }
     if (tid == 0) {
         for (int i = 0; i < 2 * TQ_DEC_WARPS; ++i) tqdev::mbar_init(&bars[i], 1);
         tqdev::fence_barrier_init();
@@ -200,17 +214,23 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int off_sign = BK * (D / 8);
     const int off_ns = off_sign + M / 8;
     const int voff_ns = BV * D / 8;
+    // value bits of this lane's 8 coordinates: [8*BV*slot, 8*BV*slot + 8*BV)
+    const int vbit = 8 * BV * slot;
+    const int vw0 = vbit / 32, vsh = vbit % 32;
+    const bool vslot = slot < NGK;
+    const int vcopy = VCOP > 1 ? slot : 0;
 
-    float m_run[QC], l_lane[QC], o[QC][CPL];
+    float m_run[QC], l_lane[QC];
+    float2 o[QC][4];   // coordinates 8*slot + 2p, +1 (tokens of parity `half`)
 #pragma unroll
     for (int qq = 0; qq < QC; ++qq) {
         m_run[qq] = -INFINITY;
         l_lane[qq] = 0.f;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) o[qq][c] = 0.f;
+        for (int c = 0; c < 4; ++c) o[qq][c] = make_float2(0.f, 0.f);
     }
-    bool aborted = false;
-    for (int64_t k = 0;; ++k) {
+    bool aborted = tqdev::status_aborted(g.status);
+    for (int64_t k = 0; !aborted; ++k) {
         const int64_t ci = warp + k * TQ_DEC_WARPS;
         if (ci >= n_chunks) break;
         const int buf = (int)(k & 1);
@@ -222,6 +242,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         const uint8_t *sV = sK + TQ_DEC_CHUNK * krow;
         const int64_t t0 = t_begin + ci * TQ_DEC_CHUNK;
 
+        // scores: step st covers tokens 2*st (lanes 0-15) and 2*st+1 (16-31),
+        // one byte group (8 coordinates / 8 projections) per lane
         float part[QC][16];
 #pragma unroll
         for (int st = 0; st < 16; ++st) {
@@ -291,27 +313,43 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             const float corr = (mn == -INFINITY) ? 1.f : __expf(m_run[qq] - mn);
             const float pr = valid ? __expf(sc - mn) : 0.f;
             l_lane[qq] = fmaf(l_lane[qq], corr, pr);
+            const float2 c2 = make_float2(corr, corr);
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) o[qq][c] *= corr;
+            for (int c = 0; c < 4; ++c) o[qq][c] = __fmul2_rn(o[qq][c], c2);
             m_run[qq] = mn;
             w_tok[qq] = valid ? pr * nsv : 0.f;
         }
-        // value accumulation, lane owns coordinates CPL*lane .. CPL*lane+CPL-1
-        const int vbit = BV * CPL * lane;
-        const int vw0 = vbit / 32, vsh = vbit % 32;
+        // values: step st again covers tokens 2*st + half; lane slot g owns
+        // coordinates 8g..8g+7 (four value pairs)
 #pragma unroll 4
-        for (int tau = 0; tau < TQ_DEC_CHUNK; ++tau) {
-            const int src = (tau & 1) * 16 + (tau >> 1);
-            const uint32_t *vr = reinterpret_cast<const uint32_t *>(sV + tau * vrow);
-            const uint32_t raw = __funnelshift_r(vr[vw0], vr[vw0 + 1], vsh);
-            float wq[QC];
+        for (int st = 0; st < 16; ++st) {
+            const uint32_t *vr = reinterpret_cast<const uint32_t *>(sV + (2 * st + half) * vrow);
+            float2 wq[QC];
 #pragma unroll
-            for (int qq = 0; qq < QC; ++qq) wq[qq] = __shfl_sync(0xffffffffu, w_tok[qq], src);
+            for (int qq = 0; qq < QC; ++qq) {
+                const float wv = __shfl_sync(0xffffffffu, w_tok[qq], half * 16 + st);
+                wq[qq] = make_float2(wv, wv);
+            }
+            if (vslot) {
+                uint32_t raw;
+                if constexpr (BV == 4) raw = vr[vw0];
+                else raw = __funnelshift_r(vr[vw0], vr[vw0 + 1], vsh);
+                uint32_t raw_hi = 0;
+                if constexpr (BV == 5) raw_hi = __funnelshift_r(vr[vw0 + 1], vr[vw0 + 2], vsh);
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const float val = vtab[(raw >> (BV * c)) & (LV - 1)];
+                for (int pp = 0; pp < 4; ++pp) {
+                    uint32_t e;
+                    if constexpr (BV == 5) {
+                        const int sh = VPB * pp;
+                        e = (sh >= 32 ? raw_hi >> (sh - 32) : (sh + VPB > 32 ? (raw >> sh) | (raw_hi << (32 - sh)) : raw >> sh)) &
+                            ((1u << VPB) - 1);
+                    } else {
+                        e = (raw >> (VPB * pp)) & ((1u << VPB) - 1);
+                    }
+                    const float2 cv = vlut[e * VCOP + vcopy];
 #pragma unroll
-                for (int qq = 0; qq < QC; ++qq) o[qq][c] = fmaf(wq[qq], val, o[qq][c]);
+                    for (int qq = 0; qq < QC; ++qq) o[qq][pp] = __ffma2_rn(wq[qq], cv, o[qq][pp]);
+                }
             }
         }
         __syncwarp();
@@ -320,10 +358,9 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             issue(ci + 2 * TQ_DEC_WARPS, buf);
         }
     }
-    if (aborted && lane == 0)
-        atomicOr(reinterpret_cast<unsigned int *>(g.status + 1), TQ_FLAG_WAIT_TIMEOUT);
+    if (aborted && lane == 0) atomicOr(reinterpret_cast<unsigned int *>(g.status + 1), TQ_FLAG_WAIT_TIMEOUT);
 
-    // ---- merge warps, rotate back, write partials
+    // ---- merge token parities, then warps; rotate back; write partials
     __syncthreads();
     float *scr = reinterpret_cast<float *>(stage);              // [warp][QC][D + 2]
 #pragma unroll
@@ -337,7 +374,15 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             row[1] = aborted ? 0.f : lt;
         }
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) row[2 + CPL * lane + c] = aborted ? 0.f : o[qq][c];
+        for (int c = 0; c < 4; ++c) {
+            float2 v = o[qq][c];
+            v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
+            v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
+            if (half == 0 && vslot) {
+                row[2 + 8 * slot + 2 * c] = aborted ? 0.f : v.x;
+                row[2 + 8 * slot + 2 * c + 1] = aborted ? 0.f : v.y;
+            }
+        }
     }
     __syncthreads();
     float *acc = scr + TQ_DEC_WARPS * QC * (D + 2);             // [QC][D]
@@ -402,6 +447,19 @@ struct SegPlan {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Shared memory of one decode CTA (must match tq_decode_kernel's carve-up).
+size_t decode_smem_bytes(int d, int bv, int qc, int krow, int vrow, int M) {
+    const int RK = (d / 8 + 15) / 16, RS = (M / 8 + 15) / 16;
+    const size_t vt = qc == 1 ? 4 : qc == 2 ? 8 : 16;
+    const size_t lut = (size_t)(RK + RS) * 256 * 16 * (qc == 1 ? 2 : 1) * vt;
+    const size_t vpair = (size_t)(1 << (2 * bv)) * (bv <= 4 ? 16 : 1) * 8;
+    const size_t stage = (size_t)TQ_DEC_WARPS * 2 * TQ_DEC_CHUNK * (krow + vrow);
+    const size_t merge = ((size_t)TQ_DEC_WARPS * qc * (d + 2) + qc * d + 2 * qc) * 4;
+    return lut + vpair + 2 * TQ_DEC_WARPS * 8 + std::max(stage, merge);
+}
+
+constexpr size_t kMaxDynSmem = 232448;   // 227 KB per block on sm_100
+
 void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sms, std::vector<SegPlan> &out) {
     const int G = Hq / Hkv;
     out.resize(n_segs);
@@ -409,7 +467,10 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
     for (int s = 0; s < n_segs; ++s) {
         const int nq = segs[s].n_seqs * G;
         SegPlan &p = out[s];
+        const tq_ctx *c = segs[s].ctx;
+        const int krow = (int)tq_row_bytes(c, TQ_KEYS), vrow = (int)tq_row_bytes(c, TQ_VALUES);
         p.qc = nq >= 4 ? 4 : nq >= 2 ? 2 : 1;
+        while (p.qc > 1 && decode_smem_bytes(c->d, c->BV, p.qc, krow, vrow, c->m) > kMaxDynSmem) p.qc /= 2;
         p.n_qchunks = (nq + p.qc - 1) / p.qc;
         work += segs[s].n_tokens * (int64_t)Hkv * p.n_qchunks;
     }
@@ -432,22 +493,14 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
 }
 
 template <int D, int BK, int BV, int QC>
-size_t decode_smem(int krow, int vrow, int M) {
-    using VT = typename Vec<QC>::T;
-    const int RK = (D / 8 + 15) / 16, RS = (M / 8 + 15) / 16;
-    size_t b = (size_t)(lut_entries<QC>(RK) + lut_entries<QC>(RS)) * sizeof(VT);
-    b += 32 * 4 + 2 * TQ_DEC_WARPS * 8;
-    const size_t stage = (size_t)TQ_DEC_WARPS * 2 * TQ_DEC_CHUNK * (krow + vrow);
-    const size_t merge = ((size_t)TQ_DEC_WARPS * QC * (D + 2) + QC * D + 2 * QC) * 4;
-    return b + std::max(stage, merge);
-}
-
-template <int D, int BK, int BV, int QC>
 cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vrow, int M, cudaStream_t stream) {
-    const size_t smem = decode_smem<D, BK, BV, QC>(krow, vrow, M);
+    const size_t smem = decode_smem_bytes(D, BV, QC, krow, vrow, M);
     auto kern = tq_decode_kernel<D, BK, BV, QC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+        cudaGetLastError();   // do not leave the failure as the thread's sticky last error
+        return e;
+    }
     kern<<<(unsigned)items, TQ_DEC_WARPS * 32, smem, stream>>>(P);
     return cudaGetLastError();
 }

@@ -310,7 +310,9 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
     }
     const float inv_sqrt_d = rsqrtf((float)D);
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
-    for (int tile = 0; tile < ENC_TILES; ++tile) {
+    if (tid == 0 && tqdev::status_aborted(p.status)) *s_abort = 1;
+    __syncthreads();
+    for (int tile = 0; tile < ENC_TILES && !*s_abort; ++tile) {
         const int64_t tt0 = tb0 + tile * ENC_GROUP;
         if (tt0 >= p.T) break;
         const int64_t t = tt0 + tid;
@@ -477,7 +479,10 @@ cudaError_t launch_t(const EncodeParams &p, const CUtensorMap &map, int grid, cu
     const size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_GROUP * 128;
     auto kern = tq_encode_kernel<D, BK, BV, Tin>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+        cudaGetLastError();   // do not leave the failure as the thread's sticky last error
+        return e;
+    }
     kern<<<grid, ENC_GROUP, smem, s>>>(p, map);
     return cudaGetLastError();
 }

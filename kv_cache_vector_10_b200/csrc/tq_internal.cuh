@@ -70,14 +70,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase.  Returns false if the bound was hit.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on an mbarrier phase: gives up after timeout_ns of wall time
+// (default 200 ms) and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase,
-                                                  uint32_t max_polls = (1u << 24)) {
-    for (uint32_t i = 0; i < max_polls; ++i) {
-        if (mbar_try_wait(bar, phase)) return true;
-        if (i > 64) __nanosleep(32);
+                                                  uint64_t timeout_ns = 200000000ull) {
+    if (mbar_try_wait(bar, phase)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, phase)) {
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
-    return false;
+    return true;
+}
+
+// True once any kernel of this context recorded a timed-out wait; later
+// CTAs then skip their work instead of waiting again.
+__device__ __forceinline__ bool status_aborted(const unsigned long long *status) {
+    return (*reinterpret_cast<const volatile unsigned long long *>(status + 1) & TQ_FLAG_WAIT_TIMEOUT) != 0;
 }
 
 __device__ __forceinline__ void fence_barrier_init() {

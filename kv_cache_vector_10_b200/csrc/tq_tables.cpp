@@ -43,7 +43,7 @@ double upper_tail(double x) { return 0.5 * std::erfc(x * 0.707106781186547524400
 
 }  // namespace
 
-extern "C" void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t *sign_words,
+extern "C" __attribute__((visibility("hidden"))) void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t *sign_words,
                                     uint16_t *S_bits) {
     SplitMix64 g{seed + (uint64_t)(int64_t)h};
     for (int w = 0; w < d / 32; ++w) sign_words[w] = 0;
@@ -63,7 +63,7 @@ extern "C" void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t
 
 // Centroids c[L] (ascending) and boundaries beta[L-1] of the 2^B-level
 // Lloyd-Max quantizer of N(0,1), rounded to float.  Returns L (0 on bad B).
-extern "C" int tq_host_codebook(int B, float *c, float *beta) {
+extern "C" __attribute__((visibility("hidden"))) int tq_host_codebook(int B, float *c, float *beta) {
     if (B < 1 || B > 5) return 0;
     const int L = 1 << B, H = L / 2;
     double mag[16], edge[17];
