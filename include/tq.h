@@ -185,6 +185,37 @@ tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q,
                               int batch, int n_q_heads, int n_kv_heads, void *out,
                               tq_dtype out_dtype, void *workspace, size_t ws_bytes, void *stream);
 
+/* Bytes of the scratch array compiled into the library for
+ * tq_decode_attention_static (8 MiB). */
+#define TQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* Decode attention that allocates nothing.  The paper has no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc -- for
+ * example a plug-in living inside a host application that owns all device
+ * memory through its own allocator and gives the plug-in no allocation
+ * hook, or a serving loop that must not allocate on the decode path because
+ * cudaMalloc may synchronize the device.  It computes exactly what
+ * tq_decode_attention computes, with the same arguments minus the
+ * workspace: the scratch (prepared queries and split-K partials) lives in a
+ * fixed array of TQ_STATIC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library holds until the process exits.
+ *  - Returns TQ_ERR_LIMIT if the call needs more scratch than
+ *    TQ_STATIC_SCRATCH_BYTES (tq_decode_workspace_bytes gives the need), or
+ *    if a segment's context has no tables yet for n_kv_heads heads (building
+ *    them allocates; call tq_ensure_heads first).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and it keeps the last
+ *    call's contents; nothing in it needs clearing, because the decode writes
+ *    every scratch value it later reads.  Calls that overlap on the GPU
+ *    (unordered streams) race on the array and must be serialized by the
+ *    caller.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine. */
+tq_status tq_decode_attention_static(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype,
+                                     int batch, int n_q_heads, int n_kv_heads, void *out,
+                                     tq_dtype out_dtype, void *stream);
+
 /* Synchronize `stream` and read the context's status word: the number of
  * non-finite rows encoded so far, and device error flags (bit 0: a bounded
  * wait inside a kernel gave up; its outputs for that tile are invalid). */

@@ -33,7 +33,8 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
 
 EXPORTED = ["tq_create", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
-            "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error"]
+            "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
+            "tq_decode_attention_static"]
 
 
 class TQError(RuntimeError):
@@ -58,7 +59,7 @@ class tq_segment(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_vector_10_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python kv_cache_vector_10_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     V, I, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
     sig = {
@@ -72,6 +73,7 @@ def _load():
         "tq_dequantize": (I, [V, ctypes.POINTER(tq_codes), I64, V, V, V]),
         "tq_decode_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
         "tq_decode_attention": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V, SZ, V]),
+        "tq_decode_attention_static": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V]),
         "tq_get_status": (I, [V, V, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32)]),
         "tq_reset_status": (I, [V, V]),
         "tq_status_string": (ctypes.c_char_p, [I]),
@@ -180,6 +182,15 @@ def tq_decode_attention(segments, q, batch: int, n_q_heads: int, n_kv_heads: int
                                     n_kv_heads, out.data_ptr(), _dtype_code(out.dtype), workspace.data_ptr(),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
            "tq_decode_attention")
+
+
+def tq_decode_attention_static(segments, q, batch: int, n_q_heads: int, n_kv_heads: int, out, stream=None):
+    """Decode attention with the library's built-in scratch array (no allocation,
+    no workspace argument); see include/tq.h for its limits and sharing rules."""
+    arr = _segment_array(segments)
+    _check(_lib.tq_decode_attention_static(arr, len(segments), q.data_ptr(), _dtype_code(q.dtype), batch, n_q_heads,
+                                           n_kv_heads, out.data_ptr(), _dtype_code(out.dtype), _stream(stream)),
+           "tq_decode_attention_static")
 
 
 def tq_get_status(ctx: int, stream=None):

@@ -3,7 +3,8 @@
 nvcc compiles the CUDA translation units for compute_100a/sm_100a; the host
 table generator (tq_tables.cpp) is compiled by g++ with FP contraction off;
 everything is linked into ``kv_cache_vector_10_b200/lib/libtq.so`` with the
-CUDA runtime linked statically.  Run ``python -m kv_cache_vector_10_b200.build``.
+CUDA runtime linked statically.  Run ``python kv_cache_vector_10_b200/build.py`` (as a script, so the package
+__init__ -- which loads the library -- is not imported first).
 """
 from __future__ import annotations
 
@@ -19,7 +20,7 @@ OBJ_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libtq.so")
 ROOT = os.path.dirname(HERE)
 
-CU_SOURCES = ["tq_api.cu", "tq_encode.cu", "tq_decode.cu", "tq_aux.cu"]
+CU_SOURCES = ["tq_api.cu", "tq_encode.cu", "tq_decode.cu", "tq_aux.cu", "tq_static.cu"]
 CPP_SOURCES = ["tq_tables.cpp"]
 HEADERS = ["tq_internal.cuh", "tq_decode.cuh"]
 

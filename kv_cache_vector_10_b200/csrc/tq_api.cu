@@ -331,3 +331,30 @@ tq_status tq_reset_status(tq_ctx *ctx, void *stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free decode support
+// Used only by tq_decode_attention_static (tq_static.cu): the same argument
+// checks as tq_decode_attention, except that head tables are never built
+// here (building allocates); a context without tables for n_kv_heads heads
+// is rejected with TQ_ERR_LIMIT.
+int tq_device_sms(int dev) { return device_sms(dev); }
+
+tq_status tq_validate_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch, int Hq,
+                             int Hkv, const void *out, tq_dtype out_dtype, bool build_tables) {
+    if (!q || !out) return TQ_ERR_NULL;
+    tq_status st = check_segments(segs, n_segs, batch, Hq, Hkv);
+    if (st != TQ_OK) return st;
+    if ((q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) ||
+        (out_dtype != TQ_F32 && out_dtype != TQ_F16 && out_dtype != TQ_BF16))
+        return TQ_ERR_DIM_MISMATCH;
+    for (int s = 0; s < n_segs; ++s) {
+        tq_ctx *c = const_cast<tq_ctx *>(segs[s].ctx);
+        if ((st = tq_check_device(c)) != TQ_OK) return st;
+        if (build_tables) {
+            if ((st = tq_ensure_heads(c, Hkv)) != TQ_OK) return st;
+        } else if (c->heads_built < Hkv) {
+            return TQ_ERR_LIMIT;
+        }
+    }
+    return TQ_OK;
+}
