@@ -60,6 +60,20 @@ def peaks():
         return 6650.0, "fallback"
 
 
+WORKLOAD_DESC = {
+    "mha_decode": "mha_decode: batch 8, 32 query heads over 32 kv heads, 4096 tokens, d128, m128, bits 4 "
+                  "(K 3+1, V 4), float16",
+    "gqa_decode": "gqa_decode: batch 4, 32 query heads over 8 kv heads, 32768 tokens, d128, m128, bits 2 "
+                  "(K 1+1, V 2), bfloat16",
+    "shared_prefix": "shared_prefix: 16 agents, prefix 4096 tokens at bits 2 read once per kv head + 16 tails of "
+                     "1024 tokens at bits 4, 32 q heads over 8 kv heads, d128, m128, bf16",
+    "bulk_encode": "bulk_encode: 32 layers x 8 kv heads x 8192 tokens x d128, bf16; bits 3 on layers 2..29, bits 4 "
+                   "on layers 0, 1, 30, 31; m128",
+    "single_head": "single_head: batch 1, 4 query heads over 1 kv heads, 1024 tokens, d128, m128, bits 3 "
+                   "(K 2+1, V 3), float32",
+}
+
+
 def row_bytes(bits):
     return (bits - 1) * D // 8 + M // 8 + 8, bits * D // 8 + 4
 
@@ -99,8 +113,7 @@ class Workload:
             es = w["k"].element_size()
             self.enc_bytes = B * Hkv * T * (2 * D * es + kr + vr)
             self.dec_bytes = B * Hkv * T * (kr + vr) + B * Hq * D * 2 * w["q"].element_size()
-            self.desc = (f"{name}: batch {B}, {Hq} query heads over {Hkv} kv heads, {T} tokens, d{D}, "
-                         f"m{M}, bits {bits} (K {bits - 1}+1, V {bits}), {str(w['k'].dtype).split('.')[-1]}")
+            self.desc = WORKLOAD_DESC[name]
         elif name == "shared_prefix":
             w = W.shared_prefix(device=device, data_seed=5 + seed_shift)
             self.w = w
@@ -121,9 +134,7 @@ class Workload:
             es = w["prefix_k"].element_size()
             self.enc_bytes = Hkv * P * (2 * D * es + pkr + pvr) + A * Hkv * Tt * (2 * D * es + tkr + tvr)
             self.dec_bytes = Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + A * Hq * D * 4
-            self.desc = (f"shared_prefix: {A} agents, prefix {P} tokens at bits {w['prefix_bits']} read once per "
-                         f"kv head + {A} tails of {Tt} tokens at bits {w['tail_bits']}, {Hq} q heads over {Hkv} kv "
-                         f"heads, d{D}, m{M}, bf16")
+            self.desc = WORKLOAD_DESC[name]
         elif name == "bulk_encode":
             w = W.bulk_encode(device=device, data_seed=4 + seed_shift)
             self.w = w
@@ -143,8 +154,7 @@ class Workload:
             self.out_bytes = H * T * (28 * (k3 + v3) + 4 * (k4 + v4))
             self.enc_bytes = self.in_bytes + self.out_bytes
             self.dec_bytes = 0
-            self.desc = (f"bulk_encode: {L} layers x {H} kv heads x {T} tokens x d{D}, bf16; bits 3 on layers "
-                         f"2..29, bits 4 on layers 0, 1, 30, 31; m{M}")
+            self.desc = WORKLOAD_DESC[name]
         self.out = None
         self.ws = None
 
@@ -219,6 +229,24 @@ def summarize_clocks(rows):
     sm.sort()
     return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
             "samples": len(sm)}
+
+
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """Max of a per-rank time over all ranks (every rank must call this)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput of a weak-scaling run: every rank processes the
+    same number of units; the job takes the slowest rank's time."""
+    return world * units_per_rank / seconds
 
 
 # ------------------------------------------------------------ CPU oracle arm
@@ -309,7 +337,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit_name, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample": desc},
+            "config": {"workload": WORKLOAD_DESC[args.workload], "l2": "inputs larger than L2 (no flush needed)",
+                       "step": "encode all K/V rows + one decode step per query head", "oracle_sample": desc},
             "cpu_baseline": {"value": val, "unit": unit_name, "cores": 1, "kind": "oracle",
                              "sample": f"{args.steps} timed steps, each {desc}"},
             "e2e": {"value": val, "unit": unit_name, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -367,10 +396,7 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     enc_ms = sum(e["enc0"].elapsed_time(e["enc1"]) for e in evs) / args.steps
     dec_ms = (sum(e["enc1"].elapsed_time(e["dec1"]) for e in evs) / args.steps) if wl.dec_bytes else 0.0
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
     clocks = summarize_clocks(rows)
 
@@ -401,21 +427,18 @@ def main():
         b.record()
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, world, dev)
         if wl.name == "bulk_encode":
-            ev, eu = world * wl.in_bytes / (e_ms * 1e-3) / 1e9, "GB/s in"
+            ev, eu = job_throughput(wl.in_bytes, world, e_ms * 1e-3) / 1e9, "GB/s in"
         else:
-            ev, eu = world * wl.tokens_scored / (e_ms * 1e-3), "KV tokens scored/s"
+            ev, eu = job_throughput(wl.tokens_scored, world, e_ms * 1e-3), "KV tokens scored/s"
         e2e = {"value": ev, "unit": eu, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     hbm, peak_kind = peaks()
     if wl.name == "bulk_encode":
-        value, unit = world * wl.in_bytes / (ms_step * 1e-3) / 1e9, "GB/s in"
+        value, unit = job_throughput(wl.in_bytes, world, ms_step * 1e-3) / 1e9, "GB/s in"
     else:
-        value, unit = world * wl.tokens_scored / (ms_step * 1e-3), "KV tokens scored/s"
+        value, unit = job_throughput(wl.tokens_scored, world, ms_step * 1e-3), "KV tokens scored/s"
     enc_gbs = wl.enc_bytes / (enc_ms * 1e-3) / 1e9 if enc_ms > 0 else None
     dec_gbs = wl.dec_bytes / (dec_ms * 1e-3) / 1e9 if dec_ms > 0 else None
     kernels = {"encode": {"ms": enc_ms, "algorithmic_bytes": wl.enc_bytes, "achieved_gbs": enc_gbs,

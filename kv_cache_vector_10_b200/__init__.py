@@ -287,3 +287,59 @@ def decode_attention(segments, q, n_kv_heads: int, out_dtype=None, workspace=Non
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     tq_decode_attention(segments, q.contiguous(), B, Hq, n_kv_heads, out, workspace, stream)
     return out
+
+
+class KvCache:
+    """Multi-head compressed KV cache with the call shapes of bitpolar's
+    KvCacheCompressor / MultiHeadKvCache (bitpolar 0.3.3 src/kv_cache.rs):
+    push (append one or more tokens for every head), len / is_empty,
+    attention_scores (pre-softmax, scaled by 1/sqrt(head_dim)),
+    decode_values, compression_ratio (original fp32 bytes / packed bytes) and
+    clear.  Head h uses seed + h.  Only bookkeeping lives here (the token
+    count); every computation is a libtq call.  Batch 1; capacity fixed at
+    construction (a multiple of 16)."""
+
+    def __init__(self, num_heads: int, head_dim: int, bits: int, projections: int, seed: int,
+                 capacity: int = 1024, device="cuda"):
+        if num_heads <= 0:
+            raise TQError(7, "KvCache")                      # TQ_ERR_EMPTY, bitpolar EmptyInput
+        self.codec = Codec(head_dim, bits, projections, seed)
+        self.num_heads, self.head_dim = num_heads, head_dim
+        self.cache = self.codec.alloc(1, num_heads, capacity, device)
+        self._len = 0
+
+    def push(self, keys, values, stream=None):
+        """keys, values: [num_heads, head_dim] (one token) or [num_heads, T, head_dim]."""
+        k = keys if keys.dim() == 3 else keys[:, None, :]
+        v = values if values.dim() == 3 else values[:, None, :]
+        if k.shape[0] != self.num_heads or v.shape != k.shape or k.shape[-1] != self.head_dim:
+            raise TQError(8, "KvCache.push")                 # TQ_ERR_DIM_MISMATCH
+        self.codec.encode_kv(k[None].contiguous(), v[None].contiguous(), self.cache, self._len, stream)
+        self._len += k.shape[1]
+
+    def __len__(self):
+        return self._len
+
+    def is_empty(self) -> bool:
+        return self._len == 0
+
+    def attention_scores(self, queries, stream=None):
+        """queries: [num_heads, head_dim] -> scores [num_heads, len]."""
+        if queries.shape != (self.num_heads, self.head_dim):
+            raise TQError(8, "KvCache.attention_scores")
+        return self.codec.attention_scores(self.cache, queries[None], self._len, stream)[0]
+
+    def decode_values(self, stream=None):
+        """-> [num_heads, len, head_dim] reconstructed values."""
+        _, vh = self.codec.dequantize(self.cache, self._len, keys=False, values=True, stream=stream)
+        return vh[0]
+
+    def compression_ratio(self) -> float:
+        if self._len == 0:
+            return 1.0
+        original = 2 * self._len * self.num_heads * self.head_dim * 4
+        packed = self._len * self.num_heads * (self.codec.k_row_bytes + self.codec.v_row_bytes)
+        return original / packed
+
+    def clear(self):
+        self._len = 0

@@ -160,8 +160,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         const int seq_local = qi / P.G, j = h * P.G + qi % P.G;
         return qp_base + ((int64_t)seq_local * P.Hq + j) * (D + M);
     };
-    {
-        const int gslot = tid % 16, lo = tid / 16;   // fixed low nibble per thread
+    for (int li = tid; li < 256; li += blockDim.x) {
+        const int gslot = li % 16, lo = li / 16;     // fixed low nibble per build lane
         for (int kind = 0; kind < 2; ++kind) {
             const int NG = kind == 0 ? NGK : NGS, R = kind == 0 ? RK : RS;
             VT *lut = kind == 0 ? lutq : luts;

@@ -5,7 +5,7 @@
 #include "tq_internal.cuh"
 
 #define TQ_DEC_CHUNK 32       // tokens per warp chunk
-#define TQ_DEC_WARPS 8        // warps per CTA
+#define TQ_DEC_WARPS 12       // warps per CTA
 #define TQ_DEC_SPLIT_UNIT (TQ_DEC_CHUNK * TQ_DEC_WARPS)
 
 // One segment as the kernels see it.  Codes pointers already point at the

@@ -9,61 +9,70 @@
 //   keys: r = (u - n_s C[idx]) / sqrt(d), gamma = |r|, bit_i = [<S_i, r> >= 0].
 // Keys use b-1 index bits, values b bits (values are MSE-only).
 //
-// Kernel design (CTAs of 128 threads, one thread per row; a CTA covers
-// ENC_TILES x 128 consecutive tokens of one (batch, head); the first half
-// of the grid encodes keys, the second half values, so each thread holds a
-// single row and the hardware scheduler interleaves both kinds):
-//   * A row lives in its thread's registers: 128-bit loads, norm, sign flip
-//     and the full 7-stage butterfly without any shuffle, quantization
-//     against the codebook boundaries scaled by n, bit-plane / field packing.
-//   * The key residual, normalised to |e| = sqrt(d) and split into binary16
-//     hi + lo parts, is written to shared memory in the 128-byte-swizzled
-//     K-major layout; one thread per group issues 2*(d/16) tcgen05.mma
-//     (M = 128 rows, N = m projections, K = 16) against S (binary16, loaded
-//     once per head by TMA), accumulating P = e S^T in fp32 in TMEM.  The two
-//     passes make the projection accurate to ~1e-7 relative, so sign bits
-//     agree with an fp64 evaluation away from |p| ~ 1e-6.
-//   * Epilogue: each thread reads its row of P from TMEM (tcgen05.ld
-//     32x32b), turns signs into the m-bit plane and stores it.
-#include <float.h>
-
+// Kernel design: one thread per row, CTAs of 128 threads (one 128-row tile
+// at a time, ENC_TILES tiles per CTA, all of one (batch, head)).  Keys and
+// values are separate kernels.  A row is processed in 32-coordinate chunks,
+// with the thread's TMEM lane as scratch (Blackwell tensor memory: 128 lanes
+// x up to 512 32-bit columns per SM):
+//   A. per chunk: 128-bit loads of the 32 inputs with the rotation's signs
+//      applied to the packed words, the five butterfly stages inside the
+//      chunk in registers, one tcgen05.st of the chunk to its TMEM columns;
+//   B. the remaining butterfly stages (across chunks) on 8-column slices
+//      read back from TMEM, accumulating |u|^2 (= d |x|^2);
+//   C. per chunk: quantization of z = u / n by a branchless binary search
+//      over the positive boundaries (pre-scaled by n), bit-plane (keys) or
+//      bit-field (values) packing, sums of C[idx]^2 and u C[idx];
+//   D. keys: the residual u - n_s C[idx], scaled to |e| ~ sqrt(d) and split
+//      into binary16 hi + lo, written to shared memory in the 128-byte
+//      swizzled K-major layout; one thread issues 2*(d/16) tcgen05.mma
+//      (M = 128 rows, N = m projections, K = 16) against S (binary16, loaded
+//      once per CTA by TMA), accumulating P = e S^T in fp32 in TMEM (the
+//      same columns the row used).  Two passes make the projection accurate
+//      to ~1e-7 relative, so sign bits agree with an fp64 evaluation away
+//      from |p| ~ 1e-6.  Each thread then reads its row of P (tcgen05.ld)
+//      and stores the m-bit sign plane.
+// Small unrolled bodies and few live registers keep the instruction cache
+// and the warp scheduler busy; DRAM traffic is the inputs read once plus the
+// packed rows written once.  Rows whose sum of squares overflows or
+// underflows fp32 (|x| beyond ~1e18 or below ~1e-18) are treated as
+// non-finite / zero rows.
 #include "tq_internal.cuh"
 
 namespace {
 
-constexpr int ENC_GROUP = 128;   // threads per CTA = rows per tile = MMA M
+constexpr int ENC_ROWS = 128;    // threads per CTA = rows per tile = MMA M
 constexpr int ENC_TILES = 4;     // tiles per CTA (S is loaded once per CTA)
 
 struct EncodeParams {
-    const void *k;
-    const void *v;
+    const void *x;          // keys or values
     int64_t sb, sh, st;     // input strides in elements
-    uint8_t *kc;
-    uint8_t *vc;
+    uint8_t *out;           // packed rows of this side
     int64_t capacity, token_offset, T;
     int H;
-    int krow, vrow;
+    int row_bytes;
     int M;
-    int64_t blocks_per_bh, k_blocks;
+    int64_t blocks_per_bh;
     const uint32_t *signs;  // [heads][d/32]
     unsigned long long *status;
-    TqBook book;
+    float mag[16];          // positive-half centroid magnitudes
+    float pb[16];           // positive boundaries
 };
 
-// Row loaders.  The rotation's random signs are applied while converting:
-// `sm` holds, per 32-bit input word, a mask with the sign bit of every
-// element that D flips (bits 15/31 for 16-bit types, bit 31 for fp32).
+// ------------------------------------------------------------- row loading
+// Chunk loaders: 32 consecutive elements, the rotation's random signs applied
+// to the packed words (mask words hold the sign bit of every flipped element:
+// bits 15/31 for 16-bit types, bit 31 for fp32).
 template <typename Tin>
-struct Loader;
+struct Chunk;
 
 template <>
-struct Loader<float> {
-    template <int D>
-    __device__ static void load(const float *src, const uint32_t *sm, float (&x)[D]) {
+struct Chunk<float> {
+    static constexpr int MASK_WORDS = 32;
+    __device__ static void load(const float *src, const uint32_t *sm, float (&x)[32]) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src);
         const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
-        for (int i = 0; i < D / 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
             const uint4 q = __ldg(p + i), f = m[i];
             x[4 * i] = __uint_as_float(q.x ^ f.x);
             x[4 * i + 1] = __uint_as_float(q.y ^ f.y);
@@ -74,13 +83,13 @@ struct Loader<float> {
 };
 
 template <>
-struct Loader<__half> {
-    template <int D>
-    __device__ static void load(const __half *src, const uint32_t *sm, float (&x)[D]) {
+struct Chunk<__half> {
+    static constexpr int MASK_WORDS = 16;
+    __device__ static void load(const __half *src, const uint32_t *sm, float (&x)[32]) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src);
         const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const uint4 q = __ldg(p + i), f = m[i];
             const uint32_t w[4] = {q.x ^ f.x, q.y ^ f.y, q.z ^ f.z, q.w ^ f.w};
 #pragma unroll
@@ -95,13 +104,13 @@ struct Loader<__half> {
 };
 
 template <>
-struct Loader<__nv_bfloat16> {
-    template <int D>
-    __device__ static void load(const __nv_bfloat16 *src, const uint32_t *sm, float (&x)[D]) {
+struct Chunk<__nv_bfloat16> {
+    static constexpr int MASK_WORDS = 16;
+    __device__ static void load(const __nv_bfloat16 *src, const uint32_t *sm, float (&x)[32]) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src);
         const uint4 *m = reinterpret_cast<const uint4 *>(sm);
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const uint4 q = __ldg(p + i), f = m[i];
             const uint32_t w[4] = {q.x ^ f.x, q.y ^ f.y, q.z ^ f.z, q.w ^ f.w};
 #pragma unroll
@@ -113,14 +122,11 @@ struct Loader<__nv_bfloat16> {
     }
 };
 
-template <typename Tin>
-constexpr int mask_words(int D) { return sizeof(Tin) == 4 ? D : D / 2; }
-
-// Per-head input sign masks: word w covers the elements stored in input
-// word w.
+// Per-head input sign masks, in input-word order.
 template <typename Tin, int D>
 __device__ void build_sign_masks(const uint32_t *signs, uint32_t *sm) {
-    for (int w = threadIdx.x; w < mask_words<Tin>(D); w += blockDim.x) {
+    constexpr int MW = Chunk<Tin>::MASK_WORDS * (D / 32);
+    for (int w = threadIdx.x; w < MW; w += blockDim.x) {
         if constexpr (sizeof(Tin) == 4) {
             sm[w] = ((signs[w / 32] >> (w % 32)) & 1u) << 31;
         } else {
@@ -130,41 +136,12 @@ __device__ void build_sign_masks(const uint32_t *signs, uint32_t *sm) {
     }
 }
 
-// Norm of a row held in registers.  Returns -1 for a row with a non-finite
-// value, 0 for an all-zero row.  Rows whose sum of squares over- or
-// underflows fp32 are rescaled by their largest magnitude.
-template <int D>
-__device__ __forceinline__ float row_norm(const float (&x)[D]) {
-    float n2 = 0.f;
+// In-register Walsh-Hadamard butterflies over 32 values (strides 1..16).
+__device__ __forceinline__ void fwht32(float (&x)[32]) {
 #pragma unroll
-    for (int j = 0; j < D; ++j) n2 = fmaf(x[j], x[j], n2);
-    if (n2 >= 1e-30f && n2 <= 1e30f) return sqrtf(n2);
-    float mx = 0.f;
-    bool bad = false;
+    for (int len = 1; len < 32; len <<= 1) {
 #pragma unroll
-    for (int j = 0; j < D; ++j) {
-        bad |= !isfinite(x[j]);
-        mx = fmaxf(mx, fabsf(x[j]));
-    }
-    if (bad) return -1.f;
-    if (mx == 0.f) return 0.f;
-    const float inv = 1.f / mx;
-    float acc = 0.f;
-#pragma unroll
-    for (int j = 0; j < D; ++j) {
-        const float t = x[j] * inv;
-        acc = fmaf(t, t, acc);
-    }
-    return mx * sqrtf(acc);
-}
-
-// u <- H u in place (the signs were applied by the loader).
-template <int D>
-__device__ __forceinline__ void fwht_inplace(float (&x)[D]) {
-#pragma unroll
-    for (int len = 1; len < D; len <<= 1) {
-#pragma unroll
-        for (int i = 0; i < D; i += 2 * len) {
+        for (int i = 0; i < 32; i += 2 * len) {
 #pragma unroll
             for (int j = i; j < i + len; ++j) {
                 const float a = x[j], b = x[j + len];
@@ -177,8 +154,7 @@ __device__ __forceinline__ void fwht_inplace(float (&x)[D]) {
 
 // Magnitude index of a = |u| among the HB cells of the positive half of the
 // codebook: the number of positive boundaries nb[k] (pre-scaled by n) with
-// a >= nb[k], found by a branchless binary search (bit k of the result is
-// decided at level k from the top).
+// a >= nb[k], found by a branchless binary search.
 template <int HB>
 __device__ __forceinline__ uint32_t mag_index(float a, const float (&nb)[16]) {
     if constexpr (HB == 1) {
@@ -206,96 +182,177 @@ __device__ __forceinline__ uint32_t mag_index(float a, const float (&nb)[16]) {
     }
 }
 
-template <int D, int BK, int BV, typename Tin>
-__global__ void __launch_bounds__(ENC_GROUP, 1)
-    tq_encode_kernel(const __grid_constant__ EncodeParams p, const __grid_constant__ CUtensorMap tmapS) {
-    constexpr int HK = (1 << BK) / 2;
+// Phases A and B: the row's rotation u = H (D x) into TMEM columns [0, D) of
+// this thread's lane; returns |u|^2.  Rows past the end rotate zeros.
+template <int D, typename Tin>
+__device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, const uint32_t *s_mask,
+                                                    uint32_t tlane) {
+    constexpr int NC = D / 32;
+#pragma unroll 1
+    for (int c = 0; c < NC; ++c) {
+        float v[32];
+        if (valid) {
+            Chunk<Tin>::load(row + 32 * c, s_mask + c * Chunk<Tin>::MASK_WORDS, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        fwht32(v);
+        tqdev::tmem_st_32x32b_x32(tlane + 32 * c, v);
+    }
+    tqdev::tmem_wait_st();
+    float n2 = 0.f;
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+        float w[NC][8];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tqdev::tmem_ld_32x32b_x8_nowait(tlane + 32 * c + 8 * g, w[c]);
+        tqdev::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int len = 1; len < NC; len <<= 1)
+#pragma unroll
+                for (int c = 0; c < NC; c += 2 * len)
+#pragma unroll
+                    for (int cc = c; cc < c + len; ++cc) {
+                        const float a = w[cc][i], b = w[cc + len][i];
+                        w[cc][i] = a + b;
+                        w[cc + len][i] = a - b;
+                    }
+#pragma unroll
+            for (int c = 0; c < NC; ++c) n2 = fmaf(w[c][i], w[c][i], n2);
+        }
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tqdev::tmem_st_32x32b_x8(tlane + 32 * c + 8 * g, w[c]);
+    }
+    tqdev::tmem_wait_st();
+    return n2;
+}
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
+    return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : 256u;
+}
+
+// ------------------------------------------------------------------ values
+template <int D, int BV, typename Tin>
+__global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_constant__ EncodeParams p) {
     constexpr int HV = (1 << BV) / 2;
-    constexpr int NW = D / 32;                 // 32-bit words per bit plane
-    constexpr int ATOM = ENC_GROUP * 128;      // bytes of one 128-row x 128-byte swizzle column
-    constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
-    constexpr int MW = mask_words<Tin>(D);
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // misc region [0, 1024): sign masks, centroid magnitudes, barriers
-    uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // [MW] (<= 512 B)
-    float *s_mag = reinterpret_cast<float *>(smem + 512);                   // [16] magnitudes
-    float *s_mag2 = s_mag + 16;                                             // [16] squared
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);              // [0] S loaded, [1] MMA done
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
-    int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
+    constexpr int NC = D / 32;
+    __shared__ __align__(16) uint32_t s_mask[Chunk<Tin>::MASK_WORDS * NC];
+    __shared__ float s_mag2[16];
+    __shared__ uint32_t s_tmem;
     const int tid = threadIdx.x, warp = tid / 32;
-    // Blocks [0, k_blocks) encode keys, the rest encode values.
-    const bool is_key = blockIdx.x < p.k_blocks;
-    const int64_t blk = is_key ? blockIdx.x : blockIdx.x - p.k_blocks;
+    const int64_t blk = blockIdx.x;
     const int64_t bh = blk / p.blocks_per_bh;
     const int head = (int)(bh % p.H);
     const int64_t b = bh / p.H;
-    const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_GROUP;
-    build_sign_masks<Tin, D>(p.signs + (int64_t)head * NW, s_mask);
+    const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_ROWS;
+    build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
+    if (tid < 16) s_mag2[tid] = tid < HV ? p.mag[tid] * p.mag[tid] : 0.f;
+    if (warp == 0) tqdev::tmem_alloc(&s_tmem, tmem_cols_for(D));
+    tqdev::tc_fence_before();
+    __syncthreads();
+    tqdev::tc_fence_after();
+    const uint32_t tlane = s_tmem + ((uint32_t)(warp * 32) << 16);
+    const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
+    float nb[16];
+#pragma unroll 1
+    for (int tile = 0; tile < ENC_TILES; ++tile) {
+        const int64_t t0 = tb0 + tile * ENC_ROWS;
+        if (t0 >= p.T) break;
+        const int64_t t = t0 + tid;
+        const bool valid = t < p.T;
+        const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+        const bool nonfinite = !(n2 <= 3.0e38f);
+        const bool degenerate = nonfinite || !(n2 > 0.f);
+        if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
+        const float n = sqrtf(n2 * (1.f / D));
+#pragma unroll
+        for (int k = 0; k < HV - 1; ++k) nb[k] = n * p.pb[k];
+        float c2 = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            float u[32];
+            tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
+            tqdev::tmem_wait_ld();
+            uint32_t f[BV];
+#pragma unroll
+            for (int w = 0; w < BV; ++w) f[w] = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                uint32_t idx;
+                if (degenerate) {
+                    idx = HV;
+                } else {
+                    const uint32_t cnt = mag_index<HV>(fabsf(u[i]), nb);
+                    idx = u[i] < 0.f ? (uint32_t)(HV - 1) - cnt : (uint32_t)HV + cnt;
+                    c2 += s_mag2[cnt];
+                }
+                const int bit = BV * i;
+                f[bit / 32] |= idx << (bit % 32);
+                if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
+            }
+            if (valid) {
+#pragma unroll
+                for (int w = 0; w < BV; ++w) dst[BV * c + w] = f[w];
+            }
+        }
+        if (valid) dst[BV * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2));
+    }
+    tqdev::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tqdev::tc_fence_after();
+        tqdev::tmem_dealloc(s_tmem, tmem_cols_for(D));
+    }
+}
+
+// -------------------------------------------------------------------- keys
+template <int BK, int D>
+__host__ __device__ constexpr size_t k_mb_bytes() {
+    return 4096 * (((size_t)(BK > 1 ? BK - 1 : 1) * (D / 32) * ENC_ROWS * 4 + 4095) / 4096);
+}
+
+template <int D, int BK, typename Tin>
+__global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_constant__ EncodeParams p,
+                                                               const __grid_constant__ CUtensorMap tmapS) {
+    constexpr int HK = (1 << BK) / 2;
+    constexpr int NC = D / 32;                 // chunks = 32-bit words per bit plane
+    constexpr int ATOM = ENC_ROWS * 128;       // bytes of one 128-row x 128-byte swizzle column
+    constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
+    constexpr int MB = BK > 1 ? BK - 1 : 1;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // misc region [0, 1024): sign masks, centroid magnitudes, barriers
+    uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // <= 512 B
+    float *s_mag = reinterpret_cast<float *>(smem + 512);                   // [16]
+    float *s_mag2 = s_mag + 16;                                             // [16]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);              // [0] S loaded, [1] MMA done
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
+    int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
+    const int M = p.M;
+    uint32_t *s_mb = reinterpret_cast<uint32_t *>(smem + 1024);             // [MB][NC][128] magnitude bits
+    uint8_t *sS = smem + 1024 + k_mb_bytes<BK, D>();                        // [D/64][M rows][128 B]
+    uint8_t *sA = sS + (D / 64) * M * 128;                                   // [pass][D/64][128 rows][128 B]
+    const int tid = threadIdx.x, warp = tid / 32;
+    const int64_t blk = blockIdx.x;
+    const int64_t bh = blk / p.blocks_per_bh;
+    const int head = (int)(bh % p.H);
+    const int64_t b = bh / p.H;
+    const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_ROWS;
+    const uint32_t tmem_cols = tmem_cols_for(M > D ? M : D);
+    build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
     if (tid < 16) {
-        const float mg = is_key ? (tid < HK ? p.book.kmag[tid] : 0.f) : (tid < HV ? p.book.vmag[tid] : 0.f);
+        const float mg = tid < HK ? p.mag[tid] : 0.f;
         s_mag[tid] = mg;
         s_mag2[tid] = mg * mg;
     }
-    const Tin *src = reinterpret_cast<const Tin *>(is_key ? p.k : p.v) + b * p.sb + (int64_t)head * p.sh;
-
-    if (!is_key) {
-        __syncthreads();
-        // ------------------------------------------------------- values
-        constexpr int VW = BV * D / 32;
-        for (int tile = 0; tile < ENC_TILES; ++tile) {
-            const int64_t t = tb0 + tile * ENC_GROUP + tid;
-            if (t >= p.T) break;
-            float x[D];
-            Loader<Tin>::template load<D>(src + t * p.st, s_mask, x);
-            const float n = row_norm<D>(x);
-            if (n < 0.f) atomicAdd(&p.status[0], 1ull);
-            uint32_t f[VW];
-#pragma unroll
-            for (int w = 0; w < VW; ++w) f[w] = 0u;
-            float ns = 0.f;
-            if (n <= 0.f) {
-#pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    const int bit = BV * j;
-                    f[bit / 32] |= (uint32_t)HV << (bit % 32);
-                    if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= (uint32_t)HV >> (32 - bit % 32);
-                }
-            } else {
-                fwht_inplace<D>(x);
-                float nb[16];
-#pragma unroll
-                for (int k2 = 0; k2 < HV - 1; ++k2) nb[k2] = n * p.book.vpb[k2];
-                float c2 = 0.f;
-#pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    const uint32_t cnt = mag_index<HV>(fabsf(x[j]), nb);
-                    const uint32_t idx = x[j] < 0.f ? (uint32_t)(HV - 1) - cnt : (uint32_t)HV + cnt;
-                    c2 += s_mag2[cnt];
-                    const int bit = BV * j;
-                    f[bit / 32] |= idx << (bit % 32);
-                    if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
-                }
-                ns = n * sqrtf((float)D / c2);
-            }
-            uint32_t *dst = reinterpret_cast<uint32_t *>(p.vc + (bh * p.capacity + p.token_offset + t) * p.vrow);
-#pragma unroll
-            for (int w = 0; w < VW; ++w) dst[w] = f[w];
-            dst[VW] = __float_as_uint(ns);
-        }
-        return;
-    }
-
-    // ------------------------------------------------------------- keys
-    const int M = p.M;
-    uint8_t *sS = smem + 1024;                            // [D/64][M rows][128 B]
-    uint8_t *sA = sS + (D / 64) * M * 128;                // [pass][D/64][128 rows][128 B]
-    const uint32_t tmem_cols = M <= 128 ? 128u : 256u;
     if (tid == 0) {
         tqdev::mbar_init(&bars[0], 1);
         tqdev::mbar_init(&bars[1], 1);
-        *s_abort = 0;
+        *s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
         tqdev::fence_barrier_init();
     }
     if (warp == 0) tqdev::tmem_alloc(s_tmem, tmem_cols);
@@ -303,125 +360,117 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
     __syncthreads();
     tqdev::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
-    if (tid == 0) {
+    const uint32_t tlane = tmem_base + ((uint32_t)(warp * 32) << 16);
+    if (tid == 0 && !*s_abort) {
         tqdev::mbar_expect_tx(&bars[0], (uint32_t)(M * D * 2));
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) tqdev::tma_load_2d(sS + a * M * 128, &tmapS, a * 64, head * M, &bars[0]);
     }
-    const float inv_sqrt_d = rsqrtf((float)D);
+    const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
-    if (tid == 0 && tqdev::status_aborted(p.status)) *s_abort = 1;
-    __syncthreads();
+    float nb[16];
+    int tiles_done = 0;
+#pragma unroll 1
     for (int tile = 0; tile < ENC_TILES && !*s_abort; ++tile) {
-        const int64_t tt0 = tb0 + tile * ENC_GROUP;
-        if (tt0 >= p.T) break;
-        const int64_t t = tt0 + tid;
+        const int64_t t0 = tb0 + tile * ENC_ROWS;
+        if (t0 >= p.T) break;
+        const int64_t t = t0 + tid;
         const bool valid = t < p.T;
-        uint8_t *rowp = p.kc + (bh * p.capacity + p.token_offset + t) * p.krow;
-        {
-            float x[D];
-            float n = 0.f;
-            if (valid) {
-                Loader<Tin>::template load<D>(src + t * p.st, s_mask, x);
-                n = row_norm<D>(x);
-                if (n < 0.f) atomicAdd(&p.status[0], 1ull);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
+        const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+        const bool nonfinite = !(n2 <= 3.0e38f);
+        const bool degenerate = nonfinite || !(n2 > 0.f);
+        if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
+        const float n = sqrtf(n2 * (1.f / D));
+#pragma unroll
+        for (int k = 0; k < HK - 1; ++k) nb[k] = n * p.pb[k];
+        // C: index planes, sum C[idx]^2 and sum u C[idx]
+        float c2 = 0.f, uc = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            float u[32];
+            tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
+            tqdev::tmem_wait_ld();
+            uint32_t negw = 0u, mbw[MB];
+#pragma unroll
+            for (int q = 0; q < MB; ++q) mbw[q] = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t cnt = mag_index<HK>(fabsf(u[i]), nb);
+                negw |= (__float_as_uint(u[i]) >> 31) << i;
+#pragma unroll
+                for (int q = 0; q < BK - 1; ++q) mbw[q] |= ((cnt >> q) & 1u) << i;
+                const float cm = s_mag[cnt];
+                c2 = fmaf(cm, cm, c2);
+                uc = fmaf(fabsf(u[i]), cm, uc);
             }
-            float ns = 0.f, gamma = 0.f;
-            if (!valid || n <= 0.f) {
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    const int off = (c / 8) * ATOM + tid * 128 + (((c % 8) ^ (tid & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(aHi + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(aLo + off) = make_uint4(0, 0, 0, 0);
-                }
-                if (valid) {
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(rowp);
-#pragma unroll
-                    for (int q = 0; q < BK; ++q)
-#pragma unroll
-                        for (int w = 0; w < NW; ++w) dst[q * NW + w] = ((HK >> q) & 1) ? 0xFFFFFFFFu : 0u;
-                }
-            } else {
-                fwht_inplace<D>(x);
-                float nb[16];
-#pragma unroll
-                for (int k2 = 0; k2 < HK - 1; ++k2) nb[k2] = n * p.book.kpb[k2];
-                // pass 1: magnitude and sign bits of every index, squared centroid norm
-                float c2 = 0.f;
-                uint32_t *dst = reinterpret_cast<uint32_t *>(rowp);
-                uint32_t mb[BK > 1 ? BK - 1 : 1][NW];
-#pragma unroll
-                for (int w = 0; w < NW; ++w) {
-                    uint32_t negw = 0u;
-#pragma unroll
-                    for (int q = 0; q < BK - 1; ++q) mb[q][w] = 0u;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float u = x[32 * w + i];
-                        const uint32_t cnt = mag_index<HK>(fabsf(u), nb);
-                        negw |= (__float_as_uint(u) >> 31) << i;
-#pragma unroll
-                        for (int q = 0; q < BK - 1; ++q) mb[q][w] |= ((cnt >> q) & 1u) << i;
-                        c2 += s_mag2[cnt];
-                    }
-                    // ascending index: top bit = non-negative, low bits = magnitude
-                    // index, complemented for negative values
-#pragma unroll
-                    for (int q = 0; q < BK - 1; ++q) dst[q * NW + w] = mb[q][w] ^ negw;
-                    dst[(BK - 1) * NW + w] = ~negw;
-                }
-                ns = n * sqrtf((float)D / c2);
-                // Hide the packed words' provenance so the compiler re-extracts
-                // the bits instead of keeping 128 indices live across passes.
+            for (int q = 0; q < BK - 1; ++q) s_mb[(q * NC + c) * ENC_ROWS + tid] = mbw[q];
+            if (valid) {
+                // ascending index: top bit = non-negative, low bits = magnitude
+                // index, complemented for negative values
 #pragma unroll
                 for (int q = 0; q < BK - 1; ++q)
-#pragma unroll
-                    for (int w = 0; w < NW; ++w) asm volatile("" : "+r"(mb[q][w]));
-                // pass 2: residual u - n_s C[idx], the magnitude index read back
-                // from the packed bits
-                float e2 = 0.f;
-#pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    const float u = x[j];
-                    uint32_t cnt = 0u;
-#pragma unroll
-                    for (int q = 0; q < BK - 1; ++q) cnt |= ((mb[q][j / 32] >> (j % 32)) & 1u) << q;
-                    const float c = copysignf(s_mag[cnt], u);
-                    x[j] = fmaf(-ns, c, u);
-                    e2 = fmaf(x[j], x[j], e2);
-                }
-                gamma = sqrtf(e2) * inv_sqrt_d;
-                // pass 3: |e| = sqrt(d) scaled residual as binary16 hi + lo, swizzled K-major
-                const float sc = e2 > 0.f ? sqrtf((float)D / e2) : 0.f;
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    uint32_t hw[4], lw[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a0 = x[8 * c + 2 * e] * sc, a1 = x[8 * c + 2 * e + 1] * sc;
-                        const __half2 hh = __floats2half2_rn(a0, a1);
-                        const float2 hf = __half22float2(hh);
-                        const __half2 ll = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
-                        hw[e] = (uint32_t)__half_as_ushort(__low2half(hh)) | ((uint32_t)__half_as_ushort(__high2half(hh)) << 16);
-                        lw[e] = (uint32_t)__half_as_ushort(__low2half(ll)) | ((uint32_t)__half_as_ushort(__high2half(ll)) << 16);
-                    }
-                    const int off = (c / 8) * ATOM + tid * 128 + (((c % 8) ^ (tid & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(aHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4 *>(aLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-            }
-            if (valid) {
-                uint32_t *dst = reinterpret_cast<uint32_t *>(rowp);
-                const int tail = BK * NW + M / 32;
-                dst[tail] = __float_as_uint(ns);
-                dst[tail + 1] = __float_as_uint(gamma);
+                    dst[q * NC + c] = degenerate ? (((HK >> q) & 1) ? ~0u : 0u) : (mbw[q] ^ negw);
+                dst[(BK - 1) * NC + c] = degenerate ? ~0u : ~negw;
             }
         }
+        const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
+        // |e|^2 from the sums, only to scale the MMA operand (the stored gamma
+        // comes from the direct sum below)
+        float e2a = n2 - 2.f * ns * uc + ns * ns * c2;
+        e2a = fmaxf(e2a, 1e-10f * n2);
+        const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
+        // D: residual as binary16 hi + lo, swizzled K-major operand
+        float e2 = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            float u[32];
+            tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
+            uint32_t mbw[MB];
+#pragma unroll
+            for (int q = 0; q < BK - 1; ++q) mbw[q] = s_mb[(q * NC + c) * ENC_ROWS + tid];
+            tqdev::tmem_wait_ld();
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float a[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int i = 8 * j8 + 2 * e + h;
+                        uint32_t cnt = 0u;
+#pragma unroll
+                        for (int q = 0; q < BK - 1; ++q) cnt |= ((mbw[q] >> i) & 1u) << q;
+                        const float cc = copysignf(s_mag[cnt], u[i]);
+                        const float ee = fmaf(-ns, cc, u[i]);
+                        e2 = fmaf(ee, ee, e2);
+                        a[h] = degenerate ? 0.f : ee * sc;
+                    }
+                    const __half2 hh = __floats2half2_rn(a[0], a[1]);
+                    const float2 hf = __half22float2(hh);
+                    const __half2 ll = __floats2half2_rn(a[0] - hf.x, a[1] - hf.y);
+                    hw[e] = (uint32_t)__half_as_ushort(__low2half(hh)) | ((uint32_t)__half_as_ushort(__high2half(hh)) << 16);
+                    lw[e] = (uint32_t)__half_as_ushort(__low2half(ll)) | ((uint32_t)__half_as_ushort(__high2half(ll)) << 16);
+                }
+                const int kk = 4 * c + j8;          // 16-byte unit of the row
+                const int off = (kk / 8) * ATOM + tid * 128 + (((kk % 8) ^ (tid & 7)) << 4);
+                *reinterpret_cast<uint4 *>(aHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(aLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+        }
+        if (valid) {
+            const int tail = BK * NC + M / 32;
+            dst[tail] = __float_as_uint(ns);
+            dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)));
+        }
+        // E: the QJL projection on the tensor cores (writes TMEM columns [0, M))
         tqdev::fence_proxy_async_smem();
         tqdev::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            bool ok = tile > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
+            const bool ok = tiles_done > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
             if (!ok) {
                 atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
                 *s_abort = 1;
@@ -445,28 +494,30 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
         }
         __syncthreads();
         if (*s_abort) break;
-        // ---------------------------------------------- sign epilogue
-        if (!tqdev::mbar_wait_bounded(&bars[1], (uint32_t)(tile & 1))) {
+        // F: sign epilogue
+        if (!tqdev::mbar_wait_bounded(&bars[1], (uint32_t)(tiles_done & 1))) {
             if (tid == 0) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
             *s_abort = 1;   // benign race: every writer stores 1
         } else {
             tqdev::tc_fence_after();
-            uint32_t *dst = reinterpret_cast<uint32_t *>(rowp) + BK * NW;
-            const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+            uint32_t *sdst = dst + BK * NC;
+#pragma unroll 1
             for (int c = 0; c < M / 32; ++c) {
                 float pv[32];
-                tqdev::tmem_ld_32x32b_x32(tmem_base + lane_base + (uint32_t)(c * 32), pv);
+                tqdev::tmem_ld_32x32b_x32_nowait(tlane + (uint32_t)(c * 32), pv);
+                tqdev::tmem_wait_ld();
                 uint32_t word = 0u;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) word |= (pv[i] >= 0.f ? 1u : 0u) << i;
-                if (valid) dst[c] = word;
+                if (valid) sdst[c] = degenerate ? ~0u : word;
             }
         }
+        ++tiles_done;
         tqdev::tc_fence_before();
         __syncthreads();
         tqdev::tc_fence_after();
-        if (*s_abort) break;
     }
+    tqdev::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tqdev::tc_fence_after();
@@ -474,34 +525,47 @@ __global__ void __launch_bounds__(ENC_GROUP, 1)
     }
 }
 
-template <int D, int BK, int BV, typename Tin>
-cudaError_t launch_t(const EncodeParams &p, const CUtensorMap &map, int grid, cudaStream_t s) {
-    const size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_GROUP * 128;
-    auto kern = tq_encode_kernel<D, BK, BV, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-        cudaGetLastError();   // do not leave the failure as the thread's sticky last error
-        return e;
+template <int D, typename Tin>
+cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, int64_t grid, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    auto go = [&](auto kern, size_t mb_bytes) {
+        const size_t smem = 2048 + mb_bytes + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();   // do not leave the failure as the thread's sticky last error
+            return;
+        }
+        kern<<<(unsigned)grid, ENC_ROWS, smem, s>>>(p, map);
+        e = cudaGetLastError();
+    };
+    switch (bits) {
+        case 2: go(tq_encode_k_kernel<D, 1, Tin>, k_mb_bytes<1, D>()); break;
+        case 3: go(tq_encode_k_kernel<D, 2, Tin>, k_mb_bytes<2, D>()); break;
+        case 4: go(tq_encode_k_kernel<D, 3, Tin>, k_mb_bytes<3, D>()); break;
+        case 5: go(tq_encode_k_kernel<D, 4, Tin>, k_mb_bytes<4, D>()); break;
+        default: return cudaErrorInvalidValue;
     }
-    kern<<<grid, ENC_GROUP, smem, s>>>(p, map);
-    return cudaGetLastError();
+    return e;
 }
 
 template <int D, typename Tin>
-cudaError_t launch_bits(int bits, const EncodeParams &p, const CUtensorMap &map, int grid, cudaStream_t s) {
+cudaError_t launch_v(int bits, const EncodeParams &p, int64_t grid, cudaStream_t s) {
     switch (bits) {
-        case 2: return launch_t<D, 1, 2, Tin>(p, map, grid, s);
-        case 3: return launch_t<D, 2, 3, Tin>(p, map, grid, s);
-        case 4: return launch_t<D, 3, 4, Tin>(p, map, grid, s);
-        case 5: return launch_t<D, 4, 5, Tin>(p, map, grid, s);
+        case 2: tq_encode_v_kernel<D, 2, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
+        case 3: tq_encode_v_kernel<D, 3, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
+        case 4: tq_encode_v_kernel<D, 4, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
+        case 5: tq_encode_v_kernel<D, 5, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
+        default: return cudaErrorInvalidValue;
     }
-    return cudaErrorInvalidValue;
+    return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t launch_dim(int d, int bits, const EncodeParams &p, const CUtensorMap &map, int grid, cudaStream_t s) {
-    if (d == 128) return launch_bits<128, Tin>(bits, p, map, grid, s);
-    if (d == 64) return launch_bits<64, Tin>(bits, p, map, grid, s);
+cudaError_t launch_side(const tq_ctx *ctx, bool keys, const EncodeParams &p, int64_t grid, cudaStream_t s) {
+    if (ctx->d == 128)
+        return keys ? launch_k<128, Tin>(ctx->bits, p, ctx->tmap_S, grid, s) : launch_v<128, Tin>(ctx->bits, p, grid, s);
+    if (ctx->d == 64)
+        return keys ? launch_k<64, Tin>(ctx->bits, p, ctx->tmap_S, grid, s) : launch_v<64, Tin>(ctx->bits, p, grid, s);
     return cudaErrorInvalidValue;
 }
 
@@ -510,40 +574,45 @@ cudaError_t launch_dim(int d, int bits, const EncodeParams &p, const CUtensorMap
 tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch, int H,
                            int64_t T, int64_t sb, int64_t sh, int64_t st, const tq_codes *codes,
                            int64_t token_offset, cudaStream_t stream, int n_sms) {
-    EncodeParams p{};
-    p.k = k;
-    p.v = v;
-    p.sb = sb; p.sh = sh; p.st = st;
-    p.kc = static_cast<uint8_t *>(codes->k);
-    p.vc = static_cast<uint8_t *>(codes->v);
-    p.capacity = codes->capacity;
-    p.token_offset = token_offset;
-    p.T = T;
-    p.H = H;
-    p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
-    p.vrow = (int)tq_row_bytes(ctx, TQ_VALUES);
-    p.M = ctx->m;
-    p.blocks_per_bh = (T + ENC_TILES * ENC_GROUP - 1) / (ENC_TILES * ENC_GROUP);
-    const int64_t per_side = p.blocks_per_bh * (int64_t)batch * H;
-    p.k_blocks = k ? per_side : 0;
-    p.signs = ctx->d_signs;
-    p.status = ctx->d_status;
-    const int HK = (1 << ctx->BK) / 2, HV = (1 << ctx->BV) / 2;
-    for (int i = 0; i < HK; ++i) p.book.kmag[i] = ctx->ck[HK + i];
-    for (int i = 0; i + 1 < HK; ++i) p.book.kpb[i] = ctx->bk[HK + i];
-    for (int i = 0; i < HV; ++i) p.book.vmag[i] = ctx->cv[HV + i];
-    for (int i = 0; i + 1 < HV; ++i) p.book.vpb[i] = ctx->bv[HV + i];
-    const int64_t total = p.k_blocks + (v ? per_side : 0);
-    if (total == 0) return TQ_OK;
-    if (total > 0x7FFFFFFF) return TQ_ERR_LIMIT;
-    const int grid = (int)total;
     (void)n_sms;
-    cudaError_t e;
-    switch (dtype) {
-        case TQ_F32: e = launch_dim<float>(ctx->d, ctx->bits, p, ctx->tmap_S, grid, stream); break;
-        case TQ_F16: e = launch_dim<__half>(ctx->d, ctx->bits, p, ctx->tmap_S, grid, stream); break;
-        case TQ_BF16: e = launch_dim<__nv_bfloat16>(ctx->d, ctx->bits, p, ctx->tmap_S, grid, stream); break;
-        default: return TQ_ERR_DIM_MISMATCH;
+    const int64_t blocks_per_bh = (T + ENC_TILES * ENC_ROWS - 1) / (ENC_TILES * ENC_ROWS);
+    const int64_t grid = blocks_per_bh * (int64_t)batch * H;
+    if (grid == 0) return TQ_OK;
+    if (grid > 0x7FFFFFFF) return TQ_ERR_LIMIT;
+    for (int side = 0; side < 2; ++side) {
+        const bool keys = side == 0;
+        const void *x = keys ? k : v;
+        if (!x) continue;
+        EncodeParams p{};
+        p.x = x;
+        p.sb = sb;
+        p.sh = sh;
+        p.st = st;
+        p.out = static_cast<uint8_t *>(keys ? codes->k : codes->v);
+        p.capacity = codes->capacity;
+        p.token_offset = token_offset;
+        p.T = T;
+        p.H = H;
+        p.row_bytes = (int)tq_row_bytes(ctx, keys ? TQ_KEYS : TQ_VALUES);
+        p.M = ctx->m;
+        p.blocks_per_bh = blocks_per_bh;
+        p.signs = ctx->d_signs;
+        p.status = ctx->d_status;
+        const int B = keys ? ctx->BK : ctx->BV;
+        const float *cb = keys ? ctx->ck : ctx->cv;
+        const float *bd = keys ? ctx->bk : ctx->bv;
+        const int HB = (1 << B) / 2;
+        for (int i = 0; i < HB; ++i) p.mag[i] = cb[HB + i];
+        for (int i = 0; i + 1 < HB; ++i) p.pb[i] = bd[HB + i];
+        cudaError_t e;
+        switch (dtype) {
+            case TQ_F32: e = launch_side<float>(ctx, keys, p, grid, stream); break;
+            case TQ_F16: e = launch_side<__half>(ctx, keys, p, grid, stream); break;
+            case TQ_BF16: e = launch_side<__nv_bfloat16>(ctx, keys, p, grid, stream); break;
+            default: return TQ_ERR_DIM_MISMATCH;
+        }
+        tq_status s = tq_check_cuda(e);
+        if (s != TQ_OK) return s;
     }
-    return tq_check_cuda(e);
+    return TQ_OK;
 }
