@@ -41,12 +41,30 @@ __device__ void prep_query(const float *sq_in, const uint32_t *signs, const __ha
     const float sc = rsqrtf((float)D);
     for (int j = tid; j < D; j += blockDim.x) s_qr[j] *= sc;
     __syncthreads();
-    for (int i = tid; i < M; i += blockDim.x) {
-        const __half *row = S + (int64_t)i * D;
+    // sq = S q_rot: LPR lanes per row, 8 binary16 values (16 bytes) per lane
+    constexpr int LPR = D / 8;
+    constexpr int RPW = 32 / LPR;   // rows per warp pass
+    const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int sub = lane / LPR, part = lane % LPR;
+    float qv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qv[e] = s_qr[8 * part + e];
+    for (int i0 = warp * RPW; i0 < M; i0 += nwarps * RPW) {
+        const int i = i0 + sub;
         float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < D; ++j) acc = fmaf(__half2float(row[j]), s_qr[j], acc);
-        s_sq[i] = acc;
+        if (i < M) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(S + (int64_t)i * D + 8 * part);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
+                acc = fmaf(f.x, qv[2 * e], acc);
+                acc = fmaf(f.y, qv[2 * e + 1], acc);
+            }
+        }
+#pragma unroll
+        for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (part == 0 && i < M) s_sq[i] = acc;
     }
     __syncthreads();
 }

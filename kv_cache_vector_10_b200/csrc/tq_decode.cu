@@ -38,19 +38,19 @@ template <>
 struct Vec<1> {
     using T = float;
     __device__ static float get(const float &v, int) { return v; }
-    __device__ static void set(float &v, int, float x) { v = x; }
+    __device__ static float make(const float (&a)[1]) { return a[0]; }
 };
 template <>
 struct Vec<2> {
     using T = float2;
     __device__ static float get(const float2 &v, int i) { return i == 0 ? v.x : v.y; }
-    __device__ static void set(float2 &v, int i, float x) { (i == 0 ? v.x : v.y) = x; }
+    __device__ static float2 make(const float (&a)[2]) { return make_float2(a[0], a[1]); }
 };
 template <>
 struct Vec<4> {
     using T = float4;
     __device__ static float get(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
-    __device__ static void set(float4 &v, int i, float x) { (i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w) = x; }
+    __device__ static float4 make(const float (&a)[4]) { return make_float4(a[0], a[1], a[2], a[3]); }
 };
 
 // Odd subsets of BK index bits: XOR masks of the sigma-planes.
@@ -74,6 +74,18 @@ __host__ __device__ constexpr int lut_entries(int rounds) {
     return rounds * 256 * 16 * (QC == 1 ? 2 : 1);
 }
 
+// Stage one chunk of packed key and value rows (tokens [tb, tb + 32),
+// clipped to the buffer capacity) into shared memory with two bulk copies
+// completing on `bar`.
+__device__ __forceinline__ void issue_chunk(uint8_t *dk, uint64_t *bar, const uint8_t *kbase, const uint8_t *vbase,
+                                            int64_t tb, int64_t capacity, int krow, int vrow) {
+    const int64_t ntok = min((int64_t)TQ_DEC_CHUNK, capacity - tb);
+    uint8_t *dv = dk + TQ_DEC_CHUNK * krow;
+    tqdev::mbar_expect_tx(bar, (uint32_t)(ntok * (krow + vrow)));
+    tqdev::bulk_load(dk, kbase + tb * krow, (uint32_t)(ntok * krow), bar);
+    tqdev::bulk_load(dv, vbase + tb * vrow, (uint32_t)(ntok * vrow), bar);
+}
+
 // Value pair table: entry e = two consecutive B_V-bit codes (low code in the
 // low bits) -> the two centroids.  VCOPIES copies, indexed by the lane's slot,
 // keep every half-warp access conflict-free.
@@ -82,7 +94,8 @@ __host__ __device__ constexpr int vpair_copies() { return BV <= 4 ? 16 : 1; }
 template <int BV>
 __host__ __device__ constexpr int vpair_entries() { return 1 << (2 * BV); }
 
-template <int D, int BK, int BV, int QC>
+// MT = number of QJL projections when known at compile time (128), else 0.
+template <int D, int BK, int BV, int QC, int MT>
 __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const __grid_constant__ DecodePlan P) {
     using VT = typename Vec<QC>::T;
     constexpr int NGK = D / 8;                    // byte groups of an index plane = value slots
@@ -107,9 +120,10 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int qchunk = (int)(local % g.n_qchunks);
     const int split = (int)((local / g.n_qchunks) % g.n_splits);
     const int h = (int)(local / ((int64_t)g.n_qchunks * g.n_splits));
-    const int M = g.m;
+    const int M = MT > 0 ? MT : g.m;
     const int NGS = M / 8, RS = (NGS + 15) / 16;
-    const int krow = g.krow, vrow = g.vrow;
+    const int krow = MT > 0 ? BK * D / 8 + MT / 8 + 8 : g.krow;
+    const int vrow = MT > 0 ? BV * D / 8 + 4 : g.vrow;
     const int64_t t_begin = (int64_t)split * g.split_len;
     const int64_t t_end = std::min<int64_t>(g.T, t_begin + g.split_len);
     const int nq = g.n_seqs * P.G;
@@ -138,28 +152,17 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int64_t n_chunks = t_end > t_begin ? (t_end - t_begin + TQ_DEC_CHUNK - 1) / TQ_DEC_CHUNK : 0;
     const uint8_t *kbase = g.kc + (int64_t)h * g.capacity * krow;
     const uint8_t *vbase = g.vc + (int64_t)h * g.capacity * vrow;
-    auto issue = [&](int64_t ci, int buf) {
-        const int64_t tb = t_begin + ci * TQ_DEC_CHUNK;
-        const int64_t ntok = std::min<int64_t>(TQ_DEC_CHUNK, g.capacity - tb);
-        uint8_t *dk = stage + (warp * 2 + buf) * chunk_bytes;
-        uint8_t *dv = dk + TQ_DEC_CHUNK * krow;
-        tqdev::mbar_expect_tx(&bars[warp * 2 + buf], (uint32_t)(ntok * (krow + vrow)));
-        tqdev::bulk_load(dk, kbase + tb * krow, (uint32_t)(ntok * krow), &bars[warp * 2 + buf]);
-        tqdev::bulk_load(dv, vbase + tb * vrow, (uint32_t)(ntok * vrow), &bars[warp * 2 + buf]);
-    };
     if (lane == 0) {
-        if (warp < n_chunks) issue(warp, 0);
-        if (warp + TQ_DEC_WARPS < n_chunks) issue(warp + TQ_DEC_WARPS, 1);
+        if (warp < n_chunks)
+            issue_chunk(stage + (warp * 2 + 0) * chunk_bytes, &bars[warp * 2 + 0], kbase, vbase, t_begin + warp * TQ_DEC_CHUNK,
+                        g.capacity, krow, vrow);
+        if (warp + TQ_DEC_WARPS < n_chunks)
+            issue_chunk(stage + (warp * 2 + 1) * chunk_bytes, &bars[warp * 2 + 1], kbase, vbase,
+                        t_begin + (warp + TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
     }
 
     // ---- per-query lookup tables
     const float *qp_base = P.qprep + g.qprep_base;
-    auto qvec = [&](int qq) -> const float * {
-        const int qi = qchunk * QC + qq;
-        if (qi >= nq) return nullptr;
-        const int seq_local = qi / P.G, j = h * P.G + qi % P.G;
-        return qp_base + ((int64_t)seq_local * P.Hq + j) * (D + M);
-    };
     for (int li = tid; li < 256; li += blockDim.x) {
         const int gslot = li % 16, lo = li / 16;     // fixed low nibble per build lane
         for (int kind = 0; kind < 2; ++kind) {
@@ -170,7 +173,9 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                 float lo_v[QC], hi_v[QC], hv[QC][4];
 #pragma unroll
                 for (int qq = 0; qq < QC; ++qq) {
-                    const float *v = qvec(qq);
+                    const int qi = qchunk * QC + qq;
+                    const float *v = qi < nq ? qp_base + ((int64_t)(qi / P.G) * P.Hq + h * P.G + qi % P.G) * (D + M)
+                                             : nullptr;
                     float vals[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) vals[i] = (v && gg < NG) ? v[(kind == 0 ? 0 : D) + 8 * gg + i] : 0.f;
@@ -185,6 +190,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                     hi_v[qq] = b;
                 }
                 int gray = 0;
+#pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     if (k > 0) {
                         const int f = __ffs(k) - 1;
@@ -194,9 +200,10 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                         for (int qq = 0; qq < QC; ++qq) hi_v[qq] += up ? hv[qq][f] : -hv[qq][f];
                     }
                     const int byte = lo | (gray << 4);
-                    VT e;
+                    float ev[QC];
 #pragma unroll
-                    for (int qq = 0; qq < QC; ++qq) Vec<QC>::set(e, qq, lo_v[qq] + hi_v[qq]);
+                    for (int qq = 0; qq < QC; ++qq) ev[qq] = lo_v[qq] + hi_v[qq];
+                    const VT e = Vec<QC>::make(ev);
                     lut[lut_slot<QC>(r, byte, 0, gslot)] = e;
                     if constexpr (QC == 1) lut[lut_slot<QC>(r, byte, 1, gslot)] = e;
                 }
@@ -355,7 +362,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         __syncwarp();
         if (lane == 0 && ci + 2 * TQ_DEC_WARPS < n_chunks) {
             tqdev::fence_proxy_async_smem();
-            issue(ci + 2 * TQ_DEC_WARPS, buf);
+            issue_chunk(stage + (warp * 2 + buf) * chunk_bytes, &bars[warp * 2 + buf], kbase, vbase,
+                        t_begin + (ci + 2 * TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
         }
     }
     if (aborted && lane == 0) atomicOr(reinterpret_cast<unsigned int *>(g.status + 1), TQ_FLAG_WAIT_TIMEOUT);
@@ -474,17 +482,33 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
         p.n_qchunks = (nq + p.qc - 1) / p.qc;
         work += segs[s].n_tokens * (int64_t)Hkv * p.n_qchunks;
     }
-    const int64_t target_items = 2 * (int64_t)n_sms;
-    int64_t L = (work + target_items - 1) / std::max<int64_t>(target_items, 1);
-    L = std::max<int64_t>(L, TQ_DEC_SPLIT_UNIT);
+    // Split length: one value for all segments, chosen to minimise the
+    // estimated time = waves x (tokens per CTA + fixed per-CTA cost), so the
+    // last wave is not mostly empty.  One decode CTA per SM is resident.
+    (void)work;
+    const int64_t kFixedTokens = 256;   // per-CTA set-up (tables, merge) in token-equivalents
+    int64_t Tmax = 0;
+    for (int s = 0; s < n_segs; ++s) Tmax = std::max<int64_t>(Tmax, segs[s].n_tokens);
+    int64_t bestL = TQ_DEC_SPLIT_UNIT;
+    double best = 1e300;
+    for (int64_t L = TQ_DEC_SPLIT_UNIT; ; L += TQ_DEC_SPLIT_UNIT) {
+        int64_t items = 0;
+        for (int s = 0; s < n_segs; ++s)
+            items += (int64_t)Hkv * out[s].n_qchunks * std::max<int64_t>(1, (segs[s].n_tokens + L - 1) / L);
+        const int64_t waves = (items + n_sms - 1) / std::max(n_sms, 1);
+        const double t = (double)waves * (double)(std::min(L, std::max<int64_t>(Tmax, 1)) + kFixedTokens);
+        if (t < best - 1e-9) {
+            best = t;
+            bestL = L;
+        }
+        if (L >= Tmax) break;
+    }
     const int d = segs[0].ctx->d;
     for (int s = 0; s < n_segs; ++s) {
         SegPlan &p = out[s];
         const int64_t T = segs[s].n_tokens;
-        int64_t ns = std::max<int64_t>(1, (T + L - 1) / L);
-        int64_t sl = (T + ns - 1) / ns;
-        sl = std::max<int64_t>(TQ_DEC_SPLIT_UNIT, (sl + TQ_DEC_SPLIT_UNIT - 1) / TQ_DEC_SPLIT_UNIT * TQ_DEC_SPLIT_UNIT);
-        ns = std::max<int64_t>(1, (T + sl - 1) / sl);
+        const int64_t ns = std::max<int64_t>(1, (T + bestL - 1) / bestL);
+        const int64_t sl = bestL;
         p.n_splits = (int)ns;
         p.split_len = (int)sl;
         p.part_floats = (int64_t)ns * segs[s].n_seqs * Hq * tq_part_floats(d);
@@ -495,7 +519,7 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
 template <int D, int BK, int BV, int QC>
 cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vrow, int M, cudaStream_t stream) {
     const size_t smem = decode_smem_bytes(D, BV, QC, krow, vrow, M);
-    auto kern = tq_decode_kernel<D, BK, BV, QC>;
+    auto kern = M == 128 ? tq_decode_kernel<D, BK, BV, QC, 128> : tq_decode_kernel<D, BK, BV, QC, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
         cudaGetLastError();   // do not leave the failure as the thread's sticky last error

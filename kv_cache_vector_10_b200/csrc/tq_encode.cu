@@ -22,7 +22,8 @@
 //   C. per chunk: quantization of z = u / n by a branchless binary search
 //      over the positive boundaries (pre-scaled by n), bit-plane (keys) or
 //      bit-field (values) packing, sums of C[idx]^2 and u C[idx];
-//   D. keys: the residual u - n_s C[idx], scaled to |e| ~ sqrt(d) and split
+//   D. keys (the signed centroids kept in TMEM columns [d, 2d) by C): the
+//      residual u - n_s C[idx], scaled to |e| ~ sqrt(d) and split
 //      into binary16 hi + lo, written to shared memory in the 128-byte
 //      swizzled K-major layout; one thread issues 2*(d/16) tcgen05.mma
 //      (M = 128 rows, N = m projections, K = 16) against S (binary16, loaded
@@ -137,18 +138,49 @@ __device__ void build_sign_masks(const uint32_t *signs, uint32_t *sm) {
 }
 
 // In-register Walsh-Hadamard butterflies over 32 values (strides 1..16).
+// Strides 2..16 pair (x[j], x[j+1]) with (x[j+len], x[j+len+1]), so they run
+// as packed fp32x2 adds / subtracts; stride 1 is done with scalar ops.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    uint64_t r;
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%1, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "add.rn.f32x2 %0, ra, rb;\n\t}"
+        : "=l"(r)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    uint64_t r;
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%1, %2};\n\t"
+        "mov.b64 rb, {%3, %4};\n\t"
+        "sub.rn.f32x2 %0, ra, rb;\n\t}"
+        : "=l"(r)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
+}
+
 __device__ __forceinline__ void fwht32(float (&x)[32]) {
+    float2 P[16];   // P[k] = (x[2k], x[2k+1]) after the stride-1 stage
 #pragma unroll
-    for (int len = 1; len < 32; len <<= 1) {
+    for (int k = 0; k < 16; ++k) P[k] = make_float2(x[2 * k] + x[2 * k + 1], x[2 * k] - x[2 * k + 1]);
 #pragma unroll
-        for (int i = 0; i < 32; i += 2 * len) {
+    for (int h = 1; h < 16; h <<= 1) {          // stride 2h in x, h in P
 #pragma unroll
-            for (int j = i; j < i + len; ++j) {
-                const float a = x[j], b = x[j + len];
-                x[j] = a + b;
-                x[j + len] = a - b;
+        for (int i = 0; i < 16; i += 2 * h) {
+#pragma unroll
+            for (int k = i; k < i + h; ++k) {
+                const float2 a = P[k], b = P[k + h];
+                P[k] = add2(a, b);
+                P[k + h] = sub2(a, b);
             }
         }
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        x[2 * k] = P[k].x;
+        x[2 * k + 1] = P[k].y;
     }
 }
 
@@ -209,19 +241,26 @@ __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, 
         for (int c = 0; c < NC; ++c) tqdev::tmem_ld_32x32b_x8_nowait(tlane + 32 * c + 8 * g, w[c]);
         tqdev::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 8; i += 2) {
 #pragma unroll
             for (int len = 1; len < NC; len <<= 1)
 #pragma unroll
                 for (int c = 0; c < NC; c += 2 * len)
 #pragma unroll
                     for (int cc = c; cc < c + len; ++cc) {
-                        const float a = w[cc][i], b = w[cc + len][i];
-                        w[cc][i] = a + b;
-                        w[cc + len][i] = a - b;
+                        const float2 a = make_float2(w[cc][i], w[cc][i + 1]);
+                        const float2 b = make_float2(w[cc + len][i], w[cc + len][i + 1]);
+                        const float2 s0 = add2(a, b), s1 = sub2(a, b);
+                        w[cc][i] = s0.x;
+                        w[cc][i + 1] = s0.y;
+                        w[cc + len][i] = s1.x;
+                        w[cc + len][i + 1] = s1.y;
                     }
 #pragma unroll
-            for (int c = 0; c < NC; ++c) n2 = fmaf(w[c][i], w[c][i], n2);
+            for (int c = 0; c < NC; ++c) {
+                n2 = fmaf(w[c][i], w[c][i], n2);
+                n2 = fmaf(w[c][i + 1], w[c][i + 1], n2);
+            }
         }
 #pragma unroll
         for (int c = 0; c < NC; ++c) tqdev::tmem_st_32x32b_x8(tlane + 32 * c + 8 * g, w[c]);
@@ -310,11 +349,6 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
 }
 
 // -------------------------------------------------------------------- keys
-template <int BK, int D>
-__host__ __device__ constexpr size_t k_mb_bytes() {
-    return 4096 * (((size_t)(BK > 1 ? BK - 1 : 1) * (D / 32) * ENC_ROWS * 4 + 4095) / 4096);
-}
-
 template <int D, int BK, typename Tin>
 __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_constant__ EncodeParams p,
                                                                const __grid_constant__ CUtensorMap tmapS) {
@@ -322,7 +356,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     constexpr int NC = D / 32;                 // chunks = 32-bit words per bit plane
     constexpr int ATOM = ENC_ROWS * 128;       // bytes of one 128-row x 128-byte swizzle column
     constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
-    constexpr int MB = BK > 1 ? BK - 1 : 1;
+    constexpr int MB = BK > 1 ? BK - 1 : 1;     // magnitude bit planes (at least one slot)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // misc region [0, 1024): sign masks, centroid magnitudes, barriers
@@ -333,8 +367,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
     int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
     const int M = p.M;
-    uint32_t *s_mb = reinterpret_cast<uint32_t *>(smem + 1024);             // [MB][NC][128] magnitude bits
-    uint8_t *sS = smem + 1024 + k_mb_bytes<BK, D>();                        // [D/64][M rows][128 B]
+    uint8_t *sS = smem + 1024;                                              // [D/64][M rows][128 B]
     uint8_t *sA = sS + (D / 64) * M * 128;                                   // [pass][D/64][128 rows][128 B]
     const int tid = threadIdx.x, warp = tid / 32;
     const int64_t blk = blockIdx.x;
@@ -342,7 +375,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     const int head = (int)(bh % p.H);
     const int64_t b = bh / p.H;
     const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_ROWS;
-    const uint32_t tmem_cols = tmem_cols_for(M > D ? M : D);
+    const uint32_t tmem_cols = tmem_cols_for(M > 2 * D ? M : 2 * D);   // U [0,d), C [d,2d); P reuses [0,m)
     build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
     if (tid < 16) {
         const float mg = tid < HK ? p.mag[tid] : 0.f;
@@ -384,7 +417,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         const float n = sqrtf(n2 * (1.f / D));
 #pragma unroll
         for (int k = 0; k < HK - 1; ++k) nb[k] = n * p.pb[k];
-        // C: index planes, sum C[idx]^2 and sum u C[idx]
+        // C: index planes, the signed centroids (to TMEM columns [d, 2d)),
+        // sum C[idx]^2 and sum u C[idx]
         float c2 = 0.f, uc = 0.f;
 #pragma unroll 1
         for (int c = 0; c < NC; ++c) {
@@ -403,9 +437,9 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 const float cm = s_mag[cnt];
                 c2 = fmaf(cm, cm, c2);
                 uc = fmaf(fabsf(u[i]), cm, uc);
+                u[i] = copysignf(cm, u[i]);
             }
-#pragma unroll
-            for (int q = 0; q < BK - 1; ++q) s_mb[(q * NC + c) * ENC_ROWS + tid] = mbw[q];
+            tqdev::tmem_st_32x32b_x32(tlane + D + 32 * c, u);
             if (valid) {
                 // ascending index: top bit = non-negative, low bits = magnitude
                 // index, complemented for negative values
@@ -415,21 +449,20 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 dst[(BK - 1) * NC + c] = degenerate ? ~0u : ~negw;
             }
         }
+        tqdev::tmem_wait_st();
         const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
         // |e|^2 from the sums, only to scale the MMA operand (the stored gamma
         // comes from the direct sum below)
         float e2a = n2 - 2.f * ns * uc + ns * ns * c2;
         e2a = fmaxf(e2a, 1e-10f * n2);
         const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
-        // D: residual as binary16 hi + lo, swizzled K-major operand
+        // D: residual u - n_s C[idx] as binary16 hi + lo, swizzled K-major operand
         float e2 = 0.f;
 #pragma unroll 1
         for (int c = 0; c < NC; ++c) {
-            float u[32];
+            float u[32], cv[32];
             tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
-            uint32_t mbw[MB];
-#pragma unroll
-            for (int q = 0; q < BK - 1; ++q) mbw[q] = s_mb[(q * NC + c) * ENC_ROWS + tid];
+            tqdev::tmem_ld_32x32b_x32_nowait(tlane + D + 32 * c, cv);
             tqdev::tmem_wait_ld();
 #pragma unroll
             for (int j8 = 0; j8 < 4; ++j8) {
@@ -440,11 +473,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int i = 8 * j8 + 2 * e + h;
-                        uint32_t cnt = 0u;
-#pragma unroll
-                        for (int q = 0; q < BK - 1; ++q) cnt |= ((mbw[q] >> i) & 1u) << q;
-                        const float cc = copysignf(s_mag[cnt], u[i]);
-                        const float ee = fmaf(-ns, cc, u[i]);
+                        const float ee = fmaf(-ns, cv[i], u[i]);
                         e2 = fmaf(ee, ee, e2);
                         a[h] = degenerate ? 0.f : ee * sc;
                     }
@@ -528,8 +557,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
 template <int D, typename Tin>
 cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, int64_t grid, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
-    auto go = [&](auto kern, size_t mb_bytes) {
-        const size_t smem = 2048 + mb_bytes + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+    auto go = [&](auto kern) {
+        const size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) {
             cudaGetLastError();   // do not leave the failure as the thread's sticky last error
@@ -539,10 +568,10 @@ cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, in
         e = cudaGetLastError();
     };
     switch (bits) {
-        case 2: go(tq_encode_k_kernel<D, 1, Tin>, k_mb_bytes<1, D>()); break;
-        case 3: go(tq_encode_k_kernel<D, 2, Tin>, k_mb_bytes<2, D>()); break;
-        case 4: go(tq_encode_k_kernel<D, 3, Tin>, k_mb_bytes<3, D>()); break;
-        case 5: go(tq_encode_k_kernel<D, 4, Tin>, k_mb_bytes<4, D>()); break;
+        case 2: go(tq_encode_k_kernel<D, 1, Tin>); break;
+        case 3: go(tq_encode_k_kernel<D, 2, Tin>); break;
+        case 4: go(tq_encode_k_kernel<D, 3, Tin>); break;
+        case 5: go(tq_encode_k_kernel<D, 4, Tin>); break;
         default: return cudaErrorInvalidValue;
     }
     return e;
