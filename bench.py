@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha_decode",
-                    choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head"])
+                    choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head",
+                             "mha_append"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -71,7 +72,42 @@ WORKLOAD_DESC = {
                    "on layers 0, 1, 30, 31; m128",
     "single_head": "single_head: batch 1, 4 query heads over 1 kv heads, 1024 tokens, d128, m128, bits 3 "
                    "(K 2+1, V 3), float32",
+    "mha_append": "mha_append: batch 8, 32 query heads over 32 kv heads, 4096 cached tokens + 1 appended per "
+                  "(sequence, kv head), d128, m128, bits 4 (K 3+1, V 4), float16",
 }
+
+
+STEP_DESC = {w: "encode all K/V rows + one decode step per query head"
+             for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head")}
+STEP_DESC["bulk_encode"] = "encode all K/V rows of 32 layers"
+STEP_DESC["mha_append"] = "append one token per (sequence, kv head) + one decode step per query head"
+L2_DESC = ("flushed (256 MiB write) before every timed piece, outside its CUDA events; "
+           "ms_per_step = sum of the pieces")
+
+
+def arm_config(workload):
+    return {"workload": WORKLOAD_DESC[workload], "step": STEP_DESC[workload], "l2": L2_DESC}
+
+
+# DRAM traffic of a piece (dram__bytes_read.sum + dram__bytes_write.sum over
+# its launches) from one ncu capture, keyed by (piece, workload), with the
+# SHA-1 of the source file holding the piece's main kernel at capture time:
+# once that source changes the entry no longer applies (traffic: null).
+MEASURED_TRAFFIC = {}
+
+
+def measured_traffic(piece, workload):
+    import hashlib
+    ent = MEASURED_TRAFFIC.get((piece, workload))
+    if not ent:
+        return None
+    src, sha, nbytes = ent
+    try:
+        with open(os.path.join(ROOT, "kv_cache_vector_10_b200", "csrc", src), "rb") as f:
+            cur = hashlib.sha1(f.read()).hexdigest()
+    except OSError:
+        return None
+    return nbytes if cur == sha else None
 
 
 def row_bytes(bits):
@@ -81,7 +117,9 @@ def row_bytes(bits):
 # ------------------------------------------------------------------ workloads
 
 class Workload:
-    """Holds device inputs, caches and the step function of one workload."""
+    """Device inputs, caches and the step of one workload.  A step is a list
+    of pieces (one or more libtq calls each), bracketed by CUDA events on the
+    launching stream: (name, algorithmic bytes, kernel launches)."""
 
     def __init__(self, name, device, rank=0):
         import torch
@@ -89,12 +127,11 @@ class Workload:
         import kv_cache_vector_10_b200 as tq
         from kv_cache_vector_10_b200 import workloads as W
         self.name, self.tq, self.torch = name, tq, torch
-        self.codecs = {}
-        self.launches = 0
         seed_shift = 1000 * rank
-        if name in ("mha_decode", "gqa_decode", "single_head"):
-            if name == "mha_decode":
-                w = W.mha_decode(device=device, data_seed=2 + seed_shift)
+        if name in ("mha_decode", "gqa_decode", "single_head", "mha_append"):
+            if name in ("mha_decode", "mha_append"):
+                w = W.mha_decode(device=device, data_seed=2 + seed_shift,
+                                 n_tokens=4097 if name == "mha_append" else 4096)
             elif name == "gqa_decode":
                 w = W.gqa_decode(device=device, data_seed=3 + seed_shift)
             else:
@@ -103,17 +140,30 @@ class Workload:
             B, Hkv, T, _ = w["k"].shape
             Hq = w["q"].shape[1]
             bits = w["bits"]
-            self.codec = tq.Codec(D, bits, M, w["seed"])
-            self.cache = self.codec.alloc(B, Hkv, (T + 15) // 16 * 16, device)
-            self.segments = [tq.Segment(self.cache, T, b, 1, codes_batch=b) for b in range(B)]
-            self.inputs = dict(k=w["k"], v=w["v"], q=w["q"])
-            self.B, self.Hq, self.Hkv = B, Hq, Hkv
-            self.tokens_scored = B * Hq * T
             kr, vr = row_bytes(bits)
             es = w["k"].element_size()
-            self.enc_bytes = B * Hkv * T * (2 * D * es + kr + vr)
-            self.dec_bytes = B * Hkv * T * (kr + vr) + B * Hq * D * 2 * w["q"].element_size()
-            self.desc = WORKLOAD_DESC[name]
+            qb = B * Hq * D * 2 * w["q"].element_size()          # query in + output out
+            self.codec = tq.Codec(D, bits, M, w["seed"])
+            self.B, self.Hq, self.Hkv = B, Hq, Hkv
+            if name == "mha_append":
+                T -= 1                                            # history; row T is the step's new row
+                self.T = T
+                self.cache = self.codec.alloc(B, Hkv, T + 16, device)
+                self.codec.encode_kv(w["k"][:, :, :T], w["v"][:, :, :T], self.cache)   # set-up, untimed
+                self.segments = [tq.Segment(self.cache, T, b, 1, codes_batch=b) for b in range(B)]
+                self.inputs = dict(k_new=w["k"][:, :, T].contiguous(), v_new=w["v"][:, :, T].contiguous(),
+                                   q=w["q"])
+                self.tokens_scored = B * Hq * (T + 1)
+                self.pieces = [("decode_append", B * Hkv * (T + 1) * (kr + vr) + B * Hkv * (2 * D * es + kr + vr)
+                                + qb, 3)]
+            else:
+                self.cache = self.codec.alloc(B, Hkv, (T + 15) // 16 * 16, device)
+                self.segments = [tq.Segment(self.cache, T, b, 1, codes_batch=b) for b in range(B)]
+                self.inputs = dict(k=w["k"], v=w["v"], q=w["q"])
+                self.tokens_scored = B * Hq * T
+                self.pieces = [("encode_keys", B * Hkv * T * (D * es + kr), 1),
+                               ("encode_values", B * Hkv * T * (D * es + vr), 1),
+                               ("decode", B * Hkv * T * (kr + vr) + qb, 3)]
         elif name == "shared_prefix":
             w = W.shared_prefix(device=device, data_seed=5 + seed_shift)
             self.w = w
@@ -132,9 +182,9 @@ class Workload:
             pkr, pvr = row_bytes(w["prefix_bits"])
             tkr, tvr = row_bytes(w["tail_bits"])
             es = w["prefix_k"].element_size()
-            self.enc_bytes = Hkv * P * (2 * D * es + pkr + pvr) + A * Hkv * Tt * (2 * D * es + tkr + tvr)
-            self.dec_bytes = Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + A * Hq * D * 4
-            self.desc = WORKLOAD_DESC[name]
+            self.pieces = [("encode_keys", Hkv * P * (D * es + pkr) + A * Hkv * Tt * (D * es + tkr), 2),
+                           ("encode_values", Hkv * P * (D * es + pvr) + A * Hkv * Tt * (D * es + tvr), 2),
+                           ("decode", Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + 2 * A * Hq * D * es, 4)]
         elif name == "bulk_encode":
             w = W.bulk_encode(device=device, data_seed=4 + seed_shift)
             self.w = w
@@ -151,47 +201,65 @@ class Workload:
             k3, v3 = row_bytes(3)
             k4, v4 = row_bytes(4)
             self.in_bytes = 2 * L * H * T * D * es
-            self.out_bytes = H * T * (28 * (k3 + v3) + 4 * (k4 + v4))
-            self.enc_bytes = self.in_bytes + self.out_bytes
-            self.dec_bytes = 0
-            self.desc = WORKLOAD_DESC[name]
+            self.pieces = [("encode_keys", L * H * T * D * es + H * T * (28 * k3 + 4 * k4), 3),
+                           ("encode_values", L * H * T * D * es + H * T * (28 * v3 + 4 * v4), 3)]
+        self.desc = WORKLOAD_DESC[name]
         self.out = None
         self.ws = None
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)   # 2x the L2
 
-    # one step with device-resident inputs; returns (encode_events, decode_events)
-    def step(self, inp, ev=None):
+    def _decode(self, inp):
         torch, tq = self.torch, self.tq
-        e = ev or {}
-        if "enc0" in e:
-            e["enc0"].record()
-        n = 0
-        if self.name in ("mha_decode", "gqa_decode", "single_head"):
-            self.codec.encode_kv(inp["k"], inp["v"], self.cache)
-            n += 1
-        elif self.name == "shared_prefix":
-            self.pcodec.encode_kv(inp["pk"], inp["pv"], self.pcache)
-            self.tcodec.encode_kv(inp["tk"], inp["tv"], self.tcache)
-            n += 2
+        if self.out is None:
+            need = tq.tq_decode_workspace_bytes(self.segments, self.B, self.Hq, self.Hkv)
+            if self.name == "mha_append":
+                need = tq.tq_decode_append_workspace_bytes(self.segments, self.B, self.Hq, self.Hkv)
+            self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=inp["q"].device)
+            self.out = torch.empty(self.B, self.Hq, D, dtype=inp["q"].dtype, device=inp["q"].device)
+        if self.name == "mha_append":
+            for sg in self.segments:          # every step appends at the same row T
+                sg.n_tokens = self.T
+            tq.tq_decode_append(self.segments, inp["k_new"], inp["v_new"], inp["q"], self.B, self.Hq, self.Hkv,
+                                self.out, self.ws)
         else:
-            k, v = inp["k"], inp["v"]
-            self.c4.encode_kv(k[:2], v[:2], self.cache4a)
-            self.c3.encode_kv(k[2:30], v[2:30], self.cache3)
-            self.c4.encode_kv(k[30:], v[30:], self.cache4b)
-            n += 3
-        if "enc1" in e:
-            e["enc1"].record()
-        if self.name != "bulk_encode":
-            if self.out is None:
-                need = tq.tq_decode_workspace_bytes(self.segments, self.B, self.Hq, self.Hkv)
-                self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=inp["q"].device)
-                self.out = torch.empty(self.B, self.Hq, D, dtype=inp["q"].dtype, device=inp["q"].device)
             tq.tq_decode_attention(self.segments, inp["q"], self.B, self.Hq, self.Hkv, self.out, self.ws)
-            groups = len(set((s.codec.bits) for s in self.segments))
-            n += 2 + groups
-        if "dec1" in e:
-            e["dec1"].record()
-        self.launches = n
+
+    def _run_piece(self, name, inp):
+        if name == "encode_keys" or name == "encode_values":
+            side = "k" if name == "encode_keys" else "v"
+            if self.name == "shared_prefix":
+                args_p = (inp["pk"], None) if side == "k" else (None, inp["pv"])
+                args_t = (inp["tk"], None) if side == "k" else (None, inp["tv"])
+                self.pcodec.encode_kv(*args_p, self.pcache)
+                self.tcodec.encode_kv(*args_t, self.tcache)
+            elif self.name == "bulk_encode":
+                x = inp[side]
+                for codec, cache, sl in ((self.c4, self.cache4a, slice(0, 2)), (self.c3, self.cache3, slice(2, 30)),
+                                         (self.c4, self.cache4b, slice(30, 32))):
+                    a = (x[sl], None) if side == "k" else (None, x[sl])
+                    codec.encode_kv(*a, cache)
+            else:
+                a = (inp["k"], None) if side == "k" else (None, inp["v"])
+                self.codec.encode_kv(*a, self.cache)
+        else:
+            self._decode(inp)
+
+    def step(self, inp, events=None):
+        """One step; events: two CUDA events per piece (start, end).  Returns
+        the decode output (None for encode-only workloads)."""
+        for i, (name, _, _) in enumerate(self.pieces):
+            if self.flush is not None:
+                self.flush.zero_()            # evict L2 before each piece (outside its events)
+            if events:
+                events[2 * i].record()
+            self._run_piece(name, inp)
+            if events:
+                events[2 * i + 1].record()
         return self.out
+
+    @property
+    def launches(self):
+        return sum(n for _, _, n in self.pieces)
 
 
 def clock_sampler(device_index):
@@ -283,6 +351,17 @@ def oracle_unit(wl_name, rank_seed=0):
                              [(pc, 0, ekp["rows"], evp["rows"]), (tc, 0, ekt["rows"], evt["rows"])])
         dt = time.perf_counter() - t0
         return dt, 4 * (1024 + 256), "tokens", "1 agent x 1 kv head (4 q heads), prefix 1024 + tail 256 tokens"
+    if wl_name == "mha_append":
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1025)
+        oc = oracle.Codec(D, w["bits"], M, w["seed"])
+        k, v = w["k"][0, 0].double().numpy(), w["v"][0, 0].double().numpy()
+        ek, ev = oc.encode(k[:1024], 0, True), oc.encode(v[:1024], 0, False)     # the cached history
+        t0 = time.perf_counter()
+        nk, nv = oc.encode(k[1024:], 0, True), oc.encode(v[1024:], 0, False)
+        oracle.attention(w["q"][0, 0].double().numpy(),
+                         [(oc, 0, np.concatenate([ek["rows"], nk["rows"]]), np.concatenate([ev["rows"], nv["rows"]]))])
+        dt = time.perf_counter() - t0
+        return dt, 1025, "tokens", "1 kv head x 1 query head: append 1 token to 1024 + decode over 1025"
     if wl_name == "mha_decode":
         w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024)
         G = 1
@@ -337,8 +416,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit_name, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_DESC[args.workload], "l2": "inputs larger than L2 (no flush needed)",
-                       "step": "encode all K/V rows + one decode step per query head", "oracle_sample": desc},
+            "config": dict(arm_config(args.workload), oracle_sample=desc),
             "cpu_baseline": {"value": val, "unit": unit_name, "cores": 1, "kind": "oracle",
                              "sample": f"{args.steps} timed steps, each {desc}"},
             "e2e": {"value": val, "unit": unit_name, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -375,29 +453,23 @@ def main():
     for _ in range(max(args.warmup, 3)):
         wl.step(inp)
     torch.cuda.synchronize()
-    # timed region
-    evs = [dict(enc0=torch.cuda.Event(enable_timing=True), enc1=torch.cuda.Event(enable_timing=True),
-                dec1=torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # timed region: every piece of every step between its own CUDA events on
+    # the launching stream; L2 is flushed before each piece, outside them
+    npieces = len(wl.pieces)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * npieces)] for _ in range(args.steps)]
     smi, rows = clock_sampler(dev.index)
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record()
     for i in range(args.steps):
         wl.step(inp, evs[i])
-    t_end.record()
     torch.cuda.synchronize()
     barrier()
     if smi is not None:
         time.sleep(0.25)
         smi.terminate()
-    total_ms = t_start.elapsed_time(t_end)
-    enc_ms = sum(e["enc0"].elapsed_time(e["enc1"]) for e in evs) / args.steps
-    dec_ms = (sum(e["enc1"].elapsed_time(e["dec1"]) for e in evs) / args.steps) if wl.dec_bytes else 0.0
-    total_ms = max_over_ranks(total_ms, world, dev)
-    ms_step = total_ms / args.steps
+    piece_ms = [sum(e[2 * p].elapsed_time(e[2 * p + 1]) for e in evs) / args.steps for p in range(npieces)]
+    ms_step = max_over_ranks(sum(piece_ms), world, dev)
     clocks = summarize_clocks(rows)
 
     # end to end through host buffers
@@ -408,25 +480,32 @@ def main():
         out_host = torch.empty(wl.B, wl.Hq, D, dtype=inp["q"].dtype).pin_memory() if "q" in inp else None
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = out_host.numel() * out_host.element_size() if out_host is not None else 0
+        e_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(10)]
 
-        def e2e_step():
+        def e2e_step(ev=None):
+            if wl.flush is not None:
+                wl.flush.zero_()
+            if ev:
+                ev[0].record()
             for k2, v2 in host.items():
                 dev_bufs[k2].copy_(v2, non_blocking=True)
+            saved = wl.flush
+            wl.flush = None
             o = wl.step(dev_bufs)
+            wl.flush = saved
             if out_host is not None:
                 out_host.copy_(o, non_blocking=True)
+            if ev:
+                ev[1].record()
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
         barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, min(args.steps, 10))
-        a.record()
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record()
+        for i in range(n_e2e):
+            e2e_step(e_evs[i])
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / n_e2e
+        e_ms = sum(e_evs[i][0].elapsed_time(e_evs[i][1]) for i in range(n_e2e)) / n_e2e
         e_ms = max_over_ranks(e_ms, world, dev)
         if wl.name == "bulk_encode":
             ev, eu = job_throughput(wl.in_bytes, world, e_ms * 1e-3) / 1e9, "GB/s in"
@@ -439,24 +518,22 @@ def main():
         value, unit = job_throughput(wl.in_bytes, world, ms_step * 1e-3) / 1e9, "GB/s in"
     else:
         value, unit = job_throughput(wl.tokens_scored, world, ms_step * 1e-3), "KV tokens scored/s"
-    enc_gbs = wl.enc_bytes / (enc_ms * 1e-3) / 1e9 if enc_ms > 0 else None
-    dec_gbs = wl.dec_bytes / (dec_ms * 1e-3) / 1e9 if dec_ms > 0 else None
-    kernels = {"encode": {"ms": enc_ms, "algorithmic_bytes": wl.enc_bytes, "achieved_gbs": enc_gbs,
-                          "frac_of_" + peak_kind + "_hbm": enc_gbs / hbm if enc_gbs else None}}
-    if wl.dec_bytes:
-        kernels["decode"] = {"ms": dec_ms, "algorithmic_bytes": wl.dec_bytes, "achieved_gbs": dec_gbs,
-                             "frac_of_" + peak_kind + "_hbm": dec_gbs / hbm if dec_gbs else None,
-                             "kv_tokens_scored_per_s": wl.tokens_scored / (dec_ms * 1e-3)}
-    dom = "encode" if enc_ms >= dec_ms else "decode"
+    kernels = {}
+    for (name, nbytes, nl), ms in zip(wl.pieces, piece_ms):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        kernels[name] = {"ms": ms, "launches": nl, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+                         "frac_of_" + peak_kind + "_hbm": gbs / hbm}
+        if name.startswith("decode"):
+            kernels[name]["kv_tokens_scored_per_s"] = wl.tokens_scored / (ms * 1e-3)
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved_gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": dk["achieved_gbs"] / hbm, "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)",
-                "traffic": None}
+                "traffic": measured_traffic(dom, wl.name)}
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.desc, "l2": "inputs larger than L2 (no flush needed)",
-                       "step": "encode all K/V rows + one decode step per query head"},
+            "config": arm_config(wl.name),
             "roofline": roofline, "kernels": kernels, "gpu_launches": wl.launches * args.steps,
             "clocks": clocks, "e2e": e2e}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -185,6 +185,35 @@ tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q,
                               int batch, int n_q_heads, int n_kv_heads, void *out,
                               tq_dtype out_dtype, void *workspace, size_t ws_bytes, void *stream);
 
+/* One decode step that first appends the step's new key and value rows
+ * (bitpolar MultiHeadKvCache::push_token followed by attention over the
+ * cache; fib-quant README, "Streaming KV encoder": a cache built one token
+ * at a time).
+ * Sequence b's private tail -- the one segment with n_seqs == 1 and
+ * first_seq == b -- receives the rows of b as token n_tokens (keys: b-1
+ * PolarQuant bits + QJL signs; values: b bits; the same codes tq_encode_kv
+ * produces for them, up to decisions within float rounding of a boundary)
+ * and is attended over n_tokens + 1 tokens; every other argument and the
+ * output are those of tq_decode_attention.  The encode runs inside the
+ * step's query-preparation kernel, so the step launches the same kernels as
+ * tq_decode_attention.
+ *  k_new, v_new : device [batch][n_kv_heads][d] in kv_dtype (contiguous).
+ *  Every sequence needs exactly one private tail with n_tokens < capacity
+ *  (TQ_ERR_DIM_MISMATCH otherwise); tails must be distinct rows of memory.
+ *  The segments are read, not modified: the caller advances each tail's
+ *  n_tokens by one after the call.  Non-finite new rows are encoded as zero
+ *  vectors and counted in the tail context's status word.
+ *  workspace : >= tq_decode_append_workspace_bytes(...) bytes. */
+tq_status tq_decode_append(const tq_segment *segs, int n_segs, const void *k_new, const void *v_new,
+                           tq_dtype kv_dtype, const void *q, tq_dtype q_dtype, int batch, int n_q_heads,
+                           int n_kv_heads, void *out, tq_dtype out_dtype, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/* Workspace bytes tq_decode_append needs (that of tq_decode_attention over
+ * the segments with every tail one token longer); 0 on invalid arguments. */
+size_t tq_decode_append_workspace_bytes(const tq_segment *segs, int n_segs, int batch, int n_q_heads,
+                                        int n_kv_heads);
+
 /* Bytes of the scratch array compiled into the library for
  * tq_decode_attention_static (8 MiB). */
 #define TQ_STATIC_SCRATCH_BYTES (8u << 20)

@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
 EXPORTED = ["tq_create", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
-            "tq_decode_attention_static"]
+            "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes"]
 
 
 class TQError(RuntimeError):
@@ -74,6 +74,8 @@ def _load():
         "tq_decode_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
         "tq_decode_attention": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V, SZ, V]),
         "tq_decode_attention_static": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V]),
+        "tq_decode_append": (I, [ctypes.POINTER(tq_segment), I, V, V, I, V, I, I, I, I, V, I, V, SZ, V]),
+        "tq_decode_append_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
         "tq_get_status": (I, [V, V, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32)]),
         "tq_reset_status": (I, [V, V]),
         "tq_status_string": (ctypes.c_char_p, [I]),
@@ -193,6 +195,23 @@ def tq_decode_attention_static(segments, q, batch: int, n_q_heads: int, n_kv_hea
            "tq_decode_attention_static")
 
 
+def tq_decode_append_workspace_bytes(segments, batch: int, n_q_heads: int, n_kv_heads: int) -> int:
+    arr = _segment_array(segments)
+    return _lib.tq_decode_append_workspace_bytes(arr, len(segments), batch, n_q_heads, n_kv_heads)
+
+
+def tq_decode_append(segments, k_new, v_new, q, batch: int, n_q_heads: int, n_kv_heads: int, out, workspace,
+                     stream=None):
+    arr = _segment_array(segments)
+    if k_new.dtype != v_new.dtype:
+        raise TQError(8, "tq_decode_append")
+    _check(_lib.tq_decode_append(arr, len(segments), k_new.data_ptr(), v_new.data_ptr(), _dtype_code(k_new.dtype),
+                                 q.data_ptr(), _dtype_code(q.dtype), batch, n_q_heads, n_kv_heads, out.data_ptr(),
+                                 _dtype_code(out.dtype), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tq_decode_append")
+
+
 def tq_get_status(ctx: int, stream=None):
     n = ctypes.c_uint64()
     f = ctypes.c_uint32()
@@ -286,6 +305,27 @@ def decode_attention(segments, q, n_kv_heads: int, out_dtype=None, workspace=Non
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     tq_decode_attention(segments, q.contiguous(), B, Hq, n_kv_heads, out, workspace, stream)
+    return out
+
+
+def decode_append(segments, k_new, v_new, q, n_kv_heads: int, out_dtype=None, workspace=None, stream=None):
+    """One decode step that first appends this step's rows: k_new, v_new
+    [batch, n_kv_heads, d] go to token n_tokens of each sequence's private
+    tail segment, which is then attended over n_tokens + 1 tokens.  The
+    Segment objects are advanced (n_tokens += 1) after the call is enqueued."""
+    import torch
+    B, Hq, d = q.shape
+    out = torch.empty(B, Hq, d, dtype=out_dtype or q.dtype, device=q.device)
+    need = tq_decode_append_workspace_bytes(segments, B, Hq, n_kv_heads)
+    if need == 0:
+        raise TQError(8, "decode_append")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    tq_decode_append(segments, k_new.contiguous(), v_new.contiguous(), q.contiguous(), B, Hq, n_kv_heads, out,
+                     workspace, stream)
+    for s in segments:
+        if s.n_seqs == 1:
+            s.n_tokens += 1
     return out
 
 

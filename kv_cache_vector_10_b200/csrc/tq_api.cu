@@ -6,7 +6,7 @@
 #include <cstring>
 #include <vector>
 
-#include "tq_internal.cuh"
+#include "tq_decode.cuh"
 
 extern "C" void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t *sign_words,
                                     uint16_t *S_bits);
@@ -22,7 +22,7 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
 tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,
                            int Hq, int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes,
-                           cudaStream_t stream, int n_sms);
+                           cudaStream_t stream, int n_sms, const TqAppend *app = nullptr);
 
 static thread_local char g_cuda_msg[256] = "no error";
 
@@ -115,8 +115,16 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
     c->device = dev;
     c->LK = tq_host_codebook(c->BK, c->ck, c->bk);
     c->LV = tq_host_codebook(c->BV, c->cv, c->bv);
+    TqBook book;
+    std::memset(&book, 0, sizeof(book));
+    for (int i = 0; i < c->LK / 2; ++i) book.kmag[i] = c->ck[c->LK / 2 + i];
+    for (int i = 0; i + 1 < c->LK / 2; ++i) book.kpb[i] = c->bk[c->LK / 2 + i];
+    for (int i = 0; i < c->LV / 2; ++i) book.vmag[i] = c->cv[c->LV / 2 + i];
+    for (int i = 0; i + 1 < c->LV / 2; ++i) book.vpb[i] = c->bv[c->LV / 2 + i];
     tq_status st = tq_check_cuda(cudaMalloc(&c->d_status, 2 * sizeof(unsigned long long)));
     if (st == TQ_OK) st = tq_check_cuda(cudaMemset(c->d_status, 0, 2 * sizeof(unsigned long long)));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMalloc(&c->d_book, sizeof(TqBook)));
+    if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(c->d_book, &book, sizeof(TqBook), cudaMemcpyHostToDevice));
     if (st != TQ_OK) {
         tq_destroy(c);
         return st;
@@ -131,6 +139,7 @@ void tq_destroy(tq_ctx *ctx) {
     cudaFree(ctx->d_signs);
     cudaFree(ctx->d_S);
     cudaFree(ctx->d_status);
+    cudaFree(ctx->d_book);
     delete ctx;
 }
 
@@ -311,6 +320,76 @@ tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q,
     if (!aligned16(workspace)) return TQ_ERR_ALIGN;
     return tq_launch_decode(segs, n_segs, q, q_dtype, batch, n_q_heads, n_kv_heads, out, out_dtype, workspace,
                             ws_bytes, static_cast<cudaStream_t>(stream), device_sms(dev));
+}
+
+}  // extern "C"
+
+// Segments as an append step sees them: the private tail of every sequence b
+// (the one segment with n_seqs == 1 and first_seq == b) grows by one token,
+// which the step writes.
+static tq_status append_segments(const tq_segment *segs, int n_segs, int batch, std::vector<tq_segment> &grown,
+                                 std::vector<uint8_t> &flags) {
+    grown.assign(segs, segs + n_segs);
+    flags.assign(n_segs, 0);
+    std::vector<int> tail(batch, -1);
+    for (int s = 0; s < n_segs; ++s) {
+        if (segs[s].n_seqs != 1) continue;
+        const int b = segs[s].first_seq;
+        if (tail[b] >= 0) return TQ_ERR_DIM_MISMATCH;   // two private tails
+        tail[b] = s;
+    }
+    for (int b = 0; b < batch; ++b) {
+        if (tail[b] < 0) return TQ_ERR_DIM_MISMATCH;   // nowhere to append
+        tq_segment &g = grown[tail[b]];
+        if (g.n_tokens + 1 > g.codes.capacity) return TQ_ERR_DIM_MISMATCH;
+        g.n_tokens += 1;
+        flags[tail[b]] = 1;
+    }
+    return TQ_OK;
+}
+
+extern "C" {
+
+size_t tq_decode_append_workspace_bytes(const tq_segment *segs, int n_segs, int batch, int n_q_heads,
+                                        int n_kv_heads) {
+    if (check_segments(segs, n_segs, batch, n_q_heads, n_kv_heads) != TQ_OK) return 0;
+    std::vector<tq_segment> grown;
+    std::vector<uint8_t> flags;
+    if (append_segments(segs, n_segs, batch, grown, flags) != TQ_OK) return 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return tq_decode_ws(grown.data(), n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
+}
+
+tq_status tq_decode_append(const tq_segment *segs, int n_segs, const void *k_new, const void *v_new,
+                           tq_dtype kv_dtype, const void *q, tq_dtype q_dtype, int batch, int n_q_heads,
+                           int n_kv_heads, void *out, tq_dtype out_dtype, void *workspace, size_t ws_bytes,
+                           void *stream) {
+    if (!q || !out || !k_new || !v_new) return TQ_ERR_NULL;
+    tq_status st = check_segments(segs, n_segs, batch, n_q_heads, n_kv_heads);
+    if (st != TQ_OK) return st;
+    if ((q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) ||
+        (out_dtype != TQ_F32 && out_dtype != TQ_F16 && out_dtype != TQ_BF16) ||
+        (kv_dtype != TQ_F32 && kv_dtype != TQ_F16 && kv_dtype != TQ_BF16))
+        return TQ_ERR_DIM_MISMATCH;
+    const uintptr_t es = kv_dtype == TQ_F32 ? 4 : 2;
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) % es) return TQ_ERR_ALIGN;
+    std::vector<tq_segment> grown;
+    std::vector<uint8_t> flags;
+    if ((st = append_segments(segs, n_segs, batch, grown, flags)) != TQ_OK) return st;
+    for (int s = 0; s < n_segs; ++s) {
+        tq_ctx *c = const_cast<tq_ctx *>(segs[s].ctx);
+        if ((st = tq_check_device(c)) != TQ_OK) return st;
+        if ((st = tq_ensure_heads(c, n_kv_heads)) != TQ_OK) return st;
+    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const size_t need = tq_decode_ws(grown.data(), n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
+    if (!workspace || ws_bytes < need) return TQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return TQ_ERR_ALIGN;
+    const TqAppend app{k_new, v_new, kv_dtype, flags.data()};
+    return tq_launch_decode(grown.data(), n_segs, q, q_dtype, batch, n_q_heads, n_kv_heads, out, out_dtype,
+                            workspace, ws_bytes, static_cast<cudaStream_t>(stream), device_sms(dev), &app);
 }
 
 tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags) {

@@ -220,18 +220,156 @@ __device__ __forceinline__ float load_as_float<__nv_bfloat16>(const void *p, int
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
 }
 
-// One block per (segment, seq_local, head): prepared query [q_rot | S q_rot].
+__device__ __forceinline__ float load_dt(const void *p, int64_t i, int dt) {
+    if (dt == TQ_F32) return static_cast<const float *>(p)[i];
+    if (dt == TQ_F16) return __half2float(static_cast<const __half *>(p)[i]);
+    return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+// Sum over the block (AUX_THREADS threads); every thread gets the total.
+__device__ __forceinline__ float block_sum(float v, float *s_red) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < AUX_THREADS / 32; ++w) t += s_red[w];
+    return t;
+}
+
+// Append step (bitpolar MultiHeadKvCache::push_token): encode one new key or
+// value row of kv head h and store it as row t of the segment.  The same
+// method as the bulk encoder (turboquant-plus-rs README, Architecture):
+// u = H (D x); n = |x|; cell = #{positive boundaries <= |u| / n}; index
+// 2^(B-1) + cell, mirrored for u < 0; n_s = n / |C[idx]/sqrt(d)|; keys add
+// the QJL signs of S (u - n_s C[idx]) and gamma = |u - n_s C[idx]| / sqrt(d).
+// One block of AUX_THREADS threads, coordinate j on thread j.
+template <int D>
+__device__ void append_row(bool key, const void *src, int64_t src_off, int dt, const SegDesc &g, int h, int64_t t,
+                           float *s_u, float *s_e, float *s_red, uint8_t *s_idx) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const TqBook &book = *g.book;
+    const int B = key ? g.bk : g.bv;
+    const int HB = 1 << (B - 1);
+    const float *mag = key ? book.kmag : book.vmag;
+    const float *pb = key ? book.kpb : book.vpb;
+    if (tid < D) {
+        const float x = load_dt(src, src_off + tid, dt);
+        s_u[tid] = ((g.signs[(int64_t)h * (D / 32) + tid / 32] >> (tid % 32)) & 1) ? -x : x;
+    }
+    __syncthreads();
+    for (int len = 1; len < D; len <<= 1) {
+        for (int i = tid; i < D / 2; i += blockDim.x) {
+            const int j = (i / len) * 2 * len + (i % len);
+            const float a = s_u[j], b = s_u[j + len];
+            s_u[j] = a + b;
+            s_u[j + len] = a - b;
+        }
+        __syncthreads();
+    }
+    const float u = tid < D ? s_u[tid] : 0.f;
+    const float n2 = block_sum(u * u, s_red);
+    const bool nonfinite = !(n2 <= 3.0e38f);
+    const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
+    if (tid == 0 && nonfinite) atomicAdd(&g.status[0], 1ull);
+    const float n = sqrtf(n2 * (1.f / D));
+    int cell = 0;
+    for (int k = 0; k + 1 < HB; ++k) cell += fabsf(u) >= n * pb[k] ? 1 : 0;
+    const float cm = mag[cell];
+    const float c2 = block_sum(tid < D ? cm * cm : 0.f, s_red);
+    const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
+    const uint32_t idx = degenerate ? (uint32_t)HB : u < 0.f ? (uint32_t)(HB - 1 - cell) : (uint32_t)(HB + cell);
+    const int64_t rowb = key ? g.krow : g.vrow;
+    uint32_t *row = reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(key ? g.kc : g.vc) +
+                                                 ((int64_t)h * g.capacity + t) * rowb);
+    if (key) {
+        const float e = tid < D && !degenerate ? u - ns * (u < 0.f ? -cm : cm) : 0.f;
+        if (tid < D) s_e[tid] = e;
+        const float e2 = block_sum(e * e, s_red);   // its barriers publish s_e
+        // index bit planes: warp w holds coordinates [32w, 32w + 32)
+#pragma unroll 1
+        for (int q = 0; q < B; ++q) {
+            const uint32_t w = __ballot_sync(0xffffffffu, (idx >> q) & 1u);
+            if (lane == 0 && tid < D) row[q * (D / 32) + warp] = w;
+        }
+        // QJL signs: projection i on thread i (and i + blockDim.x, ...)
+        const int sw0 = B * (D / 32);
+#pragma unroll 1
+        for (int i0 = 0; i0 < g.m; i0 += blockDim.x) {
+            const int i = i0 + tid;
+            float p = 0.f;
+            if (i < g.m) {
+                const uint4 *Srow = reinterpret_cast<const uint4 *>(g.S + ((int64_t)h * g.m + i) * D);
+#pragma unroll 4
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 w = Srow[c];
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e2i = 0; e2i < 4; ++e2i) {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e2i]));
+                        p = fmaf(f.x, s_e[8 * c + 2 * e2i], p);
+                        p = fmaf(f.y, s_e[8 * c + 2 * e2i + 1], p);
+                    }
+                }
+            }
+            const uint32_t w = __ballot_sync(0xffffffffu, p >= 0.f);
+            if (lane == 0 && i0 + 32 * warp < g.m) row[sw0 + (i0 + 32 * warp) / 32] = degenerate ? ~0u : w;
+        }
+        if (tid == 0) {
+            const int tail = sw0 + g.m / 32;
+            row[tail] = __float_as_uint(ns);
+            row[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)));
+        }
+    } else {
+        if (tid < D) s_idx[tid] = (uint8_t)idx;
+        __syncthreads();
+        // B-bit fields, coordinate j at bit B j of the little-endian stream
+        for (int w = tid; w < B * D / 32; w += blockDim.x) {
+            uint32_t word = 0u;
+            for (int b = 0; b < 32; ++b) {
+                const int bit = 32 * w + b;
+                word |= (uint32_t)((s_idx[bit / B] >> (bit % B)) & 1) << b;
+            }
+            row[w] = word;
+        }
+        if (tid == 0) row[B * D / 32] = __float_as_uint(ns);
+    }
+    __syncthreads();
+}
+
+// Blocks [0, query blocks): one per (segment, seq_local, head), the prepared
+// query [q_rot | S q_rot].  Blocks after those: one per (appending segment,
+// kv head), the append step's new key and value rows.
 template <int D, typename Tq>
 __global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
     __shared__ float s_in[D];
     __shared__ float s_qr[D];
     __shared__ float s_sq[256];
+    __shared__ float s_red[AUX_THREADS / 32];
+    __shared__ uint8_t s_idx[D];
     int s = 0;
     int64_t blk = blockIdx.x;
     for (; s < P.n_segs; ++s) {
         const int64_t n = (int64_t)P.seg[s].n_seqs * P.Hq;
         if (blk < n) break;
         blk -= n;
+    }
+    if (s == P.n_segs) {
+        // append block: blk counts (appending segment, kv head) pairs
+        for (s = 0; s < P.n_segs; ++s) {
+            if (!P.seg[s].append) continue;
+            if (blk < P.Hkv) break;
+            blk -= P.Hkv;
+        }
+        if (s == P.n_segs) return;
+        const SegDesc &g = P.seg[s];
+        const int h = (int)blk;
+        const int64_t src = ((int64_t)g.first_seq * P.Hkv + h) * D;
+        append_row<D>(true, P.k_new, src, P.kv_dtype, g, h, g.T - 1, s_in, s_qr, s_red, s_idx);
+        append_row<D>(false, P.v_new, src, P.kv_dtype, g, h, g.T - 1, s_in, s_qr, s_red, s_idx);
+        return;
     }
     const SegDesc &g = P.seg[s];
     const int seq_local = (int)(blk / P.Hq), j = (int)(blk % P.Hq);
@@ -354,7 +492,7 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
 }
 
 cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cudaStream_t stream) {
-    int64_t blocks = 0;
+    int64_t blocks = P.n_append_blocks;
     for (int s = 0; s < P.n_segs; ++s) blocks += (int64_t)P.seg[s].n_seqs * P.Hq;
     if (blocks == 0) return cudaSuccess;
 #define TQ_QPREP(DD, TT) tq_qprep_kernel<DD, TT><<<(unsigned)blocks, AUX_THREADS, 0, stream>>>(P, q)

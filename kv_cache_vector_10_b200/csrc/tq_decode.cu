@@ -583,7 +583,7 @@ size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int H
 
 tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch, int Hq,
                            int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes, cudaStream_t stream,
-                           int n_sms) {
+                           int n_sms, const TqAppend *app) {
     (void)ws_bytes;
     std::vector<SegPlan> pl;
     plan_segments(segs, n_segs, Hq, Hkv, n_sms, pl);
@@ -610,6 +610,9 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         d.signs = c->d_signs;
         d.S = c->d_S;
         d.status = c->d_status;
+        d.book = c->d_book;
+        d.append = app && app->flags[s] ? 1 : 0;
+        if (d.append) P.n_append_blocks += Hkv;
         d.capacity = sg.codes.capacity;
         d.T = sg.n_tokens;
         d.part_base = poff / tq_part_floats(P.d);
@@ -630,6 +633,11 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         for (int i = 0; i < 32; ++i) d.vtab[i] = i < c->LV ? c->cv[i] : 0.f;
         qoff += pl[s].qprep_floats;
         poff += pl[s].part_floats;
+    }
+    if (app) {
+        P.k_new = app->k_new;
+        P.v_new = app->v_new;
+        P.kv_dtype = (int)app->dtype;
     }
     cudaError_t e = tq_launch_qprep(P, q, q_dtype, stream);
     if (e != cudaSuccess) return tq_check_cuda(e);

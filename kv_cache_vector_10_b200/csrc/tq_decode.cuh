@@ -16,6 +16,7 @@ struct SegDesc {
     const uint32_t *signs;     // [H_kv][d/32]
     const __half *S;           // [H_kv][m][d]
     unsigned long long *status;  // the segment context's status word
+    const TqBook *book;        // the segment context's codebooks (device)
     int64_t capacity;
     int64_t T;
     int64_t part_base;         // first partial slot of this segment
@@ -25,6 +26,7 @@ struct SegDesc {
     int krow, vrow, m, bk, bv;
     int n_splits, split_len, n_qchunks;
     int n_planes;              // odd subsets of the key index bits
+    int append;                // 1: this step's new key/value rows go to row T-1
     uint32_t plane_sets[8];    // bit mask of index planes XOR-ed into sigma-plane s
     float alpha[8];            // Walsh coefficient of sigma-plane s
     float vtab[32];            // value centroids, indexed by code
@@ -37,6 +39,21 @@ struct DecodePlan {
     int batch;
     float *qprep;              // prepared queries: [q_rot (d) | S q_rot (m)] per (segment, seq, head)
     float *part;               // partial slots: [m, l, pad, pad, o (d)]
+    // Append step: new rows [batch][H_kv][d] in kv_dtype, encoded by the
+    // query-preparation kernel into the segments flagged `append`.
+    const void *k_new;
+    const void *v_new;
+    int kv_dtype;
+    int n_append_blocks;
+};
+static_assert(sizeof(DecodePlan) <= 32764, "the plan is passed as a kernel parameter");
+
+// Host-side description of an append step (tq_decode_append).
+struct TqAppend {
+    const void *k_new;
+    const void *v_new;
+    tq_dtype dtype;
+    const uint8_t *flags;      // [n_segs]: 1 = the segment receives the new rows
 };
 
 // Floats per partial slot.

@@ -19,9 +19,12 @@
 //      chunk in registers, one tcgen05.st of the chunk to its TMEM columns;
 //   B. the remaining butterfly stages (across chunks) on 8-column slices
 //      read back from TMEM, accumulating |u|^2 (= d |x|^2);
-//   C. per chunk: quantization of z = u / n by a branchless binary search
-//      over the positive boundaries (pre-scaled by n), bit-plane (keys) or
-//      bit-field (values) packing, sums of C[idx]^2 and u C[idx];
+//   C. per chunk: quantization of z = u / n by a binary search over the
+//      positive boundaries (pre-scaled by n) done on pairs of coordinates in
+//      packed fp32x2 arithmetic, each level's decision bit gathered from the
+//      sign of |u| - boundary with a funnel shift; bit-plane (keys) or
+//      bit-field (values) packing; sum C[idx]^2 from per-cell counts
+//      (popcounts of the level words), sum |u| C[idx] (keys);
 //   D. keys (the signed centroids kept in TMEM columns [d, 2d) by C): the
 //      residual u - n_s C[idx], scaled to |e| ~ sqrt(d) and split
 //      into binary16 hi + lo, written to shared memory in the 128-byte
@@ -34,9 +37,10 @@
 //      and stores the m-bit sign plane.
 // Small unrolled bodies and few live registers keep the instruction cache
 // and the warp scheduler busy; DRAM traffic is the inputs read once plus the
-// packed rows written once.  Rows whose sum of squares overflows or
-// underflows fp32 (|x| beyond ~1e18 or below ~1e-18) are treated as
-// non-finite / zero rows.
+// packed rows written once.  Rows whose rotated sum of squares d |x|^2
+// overflows fp32 (|x| beyond ~1.5e18) are counted as non-finite; rows where
+// it falls below the smallest normal float (|x| below ~1e-20) are encoded as
+// zero rows (the exact search steps need normal-range boundaries).
 #include "tq_internal.cuh"
 
 namespace {
@@ -57,6 +61,7 @@ struct EncodeParams {
     unsigned long long *status;
     float mag[16];          // positive-half centroid magnitudes
     float pb[16];           // positive boundaries
+    float cl[8];            // keys: centroid magnitude as a multilinear form in the search bits
 };
 
 // ------------------------------------------------------------- row loading
@@ -186,32 +191,117 @@ __device__ __forceinline__ void fwht32(float (&x)[32]) {
 
 // Magnitude index of a = |u| among the HB cells of the positive half of the
 // codebook: the number of positive boundaries nb[k] (pre-scaled by n) with
-// a >= nb[k], found by a branchless binary search.
+// a >= nb[k], found by a branchless binary search.  Used for 16 cells (5-bit
+// values); fewer cells go through the packed search below.
 template <int HB>
 __device__ __forceinline__ uint32_t mag_index(float a, const float (&nb)[16]) {
-    if constexpr (HB == 1) {
-        return 0u;
-    } else if constexpr (HB == 2) {
-        return a >= nb[0] ? 1u : 0u;
+    static_assert(HB == 16, "the compare-and-select search serves 16 cells");
+    const bool t3 = a >= nb[7];
+    const bool t2 = a >= (t3 ? nb[11] : nb[3]);
+    const bool t1 = a >= (t3 ? (t2 ? nb[13] : nb[9]) : (t2 ? nb[5] : nb[1]));
+    const float b0 = t3 ? (t2 ? (t1 ? nb[14] : nb[12]) : (t1 ? nb[10] : nb[8]))
+                        : (t2 ? (t1 ? nb[6] : nb[4]) : (t1 ? nb[2] : nb[0]));
+    const bool t0 = a >= b0;
+    return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+}
+
+// ------------------------------------------------------ packed quantization
+// For up to 8 cells per half the binary search runs on pairs of coordinates
+// in packed fp32x2 arithmetic (FMA pipe) instead of compares and selects:
+// level L tests d_L = |u| - b_L >= 0, where b_L is the boundary chosen by the
+// levels above; T_L = [d_L >= 0] in {0, 1} is saturate(d_L * 2^126 + 1) and
+// selects the next boundary with one fused multiply-add.  The magnitude
+// index is sum_L T_L 2^L; bit L of every coordinate of a 32-coordinate chunk
+// is collected from the sign of d_L with one funnel shift.
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// [d >= 0] as 0.0 or 1.0, exact for d = 0 and |d| >= 2^-126; NaN gives 0.
+__device__ __forceinline__ float step01(float d) {
+    float r;
+    asm("fma.rn.sat.f32 %0, %1, 0f7E800000, 0f3F800000;" : "=f"(r) : "f"(d));
+    return r;
+}
+__device__ __forceinline__ float2 step2(float2 d) { return make_float2(step01(d.x), step01(d.y)); }
+
+// Shift the sign bit of x into the bottom of w (coordinates are visited from
+// 31 down to 0, so coordinate i ends at bit i).
+__device__ __forceinline__ uint32_t push_sign(uint32_t w, float x) { return __funnelshift_l(__float_as_uint(x), w, 1); }
+
+template <int HB>
+struct Levels {
+    static constexpr int L = HB == 1 ? 0 : HB == 2 ? 1 : HB == 4 ? 2 : 3;
+};
+
+// Row boundaries of the search (scaled by the row norm n), in the order the
+// levels use them.
+template <int HB>
+__device__ __forceinline__ void row_bounds(float n, const float (&pb)[16], float (&rb)[8]) {
+    float nb[8];
+#pragma unroll
+    for (int k = 0; k < HB - 1; ++k) nb[k] = n * pb[k];
+    if constexpr (HB == 2) {
+        rb[0] = nb[0];
     } else if constexpr (HB == 4) {
-        const bool t1 = a >= nb[1];
-        const bool t0 = a >= (t1 ? nb[2] : nb[0]);
-        return (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+        rb[0] = nb[1];
+        rb[1] = nb[2] - nb[0];
+        rb[2] = nb[0];
     } else if constexpr (HB == 8) {
-        const bool t2 = a >= nb[3];
-        const bool t1 = a >= (t2 ? nb[5] : nb[1]);
-        const float b0 = t2 ? (t1 ? nb[6] : nb[4]) : (t1 ? nb[2] : nb[0]);
-        const bool t0 = a >= b0;
-        return (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
-    } else {
-        const bool t3 = a >= nb[7];
-        const bool t2 = a >= (t3 ? nb[11] : nb[3]);
-        const bool t1 = a >= (t3 ? (t2 ? nb[13] : nb[9]) : (t2 ? nb[5] : nb[1]));
-        const float b0 = t3 ? (t2 ? (t1 ? nb[14] : nb[12]) : (t1 ? nb[10] : nb[8]))
-                            : (t2 ? (t1 ? nb[6] : nb[4]) : (t1 ? nb[2] : nb[0]));
-        const bool t0 = a >= b0;
-        return (t3 ? 8u : 0u) | (t2 ? 4u : 0u) | (t1 ? 2u : 0u) | (t0 ? 1u : 0u);
+        rb[0] = nb[3];
+        rb[1] = nb[5] - nb[1];
+        rb[2] = nb[1];
+        rb[3] = (nb[6] - nb[4]) - (nb[2] - nb[0]);
+        rb[4] = nb[2] - nb[0];
+        rb[5] = nb[4] - nb[0];
+        rb[6] = nb[0];
     }
+}
+
+// The search for one pair of magnitudes A; T[L] and d[L] per level.
+template <int HB>
+__device__ __forceinline__ void search2(float2 A, const float (&rb)[8], float2 (&T)[3], float2 (&d)[3]) {
+    if constexpr (HB == 2) {
+        d[0] = sub2(A, dup2(rb[0]));
+        T[0] = step2(d[0]);
+    } else if constexpr (HB == 4) {
+        d[1] = sub2(A, dup2(rb[0]));
+        T[1] = step2(d[1]);
+        d[0] = sub2(A, fma2(T[1], dup2(rb[1]), dup2(rb[2])));
+        T[0] = step2(d[0]);
+    } else if constexpr (HB == 8) {
+        d[2] = sub2(A, dup2(rb[0]));
+        T[2] = step2(d[2]);
+        d[1] = sub2(A, fma2(T[2], dup2(rb[1]), dup2(rb[2])));
+        T[1] = step2(d[1]);
+        const float2 b0 = fma2(T[1], fma2(T[2], dup2(rb[3]), dup2(rb[4])), fma2(T[2], dup2(rb[5]), dup2(rb[6])));
+        d[0] = sub2(A, b0);
+        T[0] = step2(d[0]);
+    }
+}
+
+// Number of coordinates of a chunk in each magnitude cell k = sum_L T_L 2^L,
+// from the per-level sign words S[L] (bit set = T_L is 0); cell 0 is implied.
+template <int HB>
+__device__ __forceinline__ void count_cells(const uint32_t (&S)[3], int (&cnt)[8]) {
+#pragma unroll
+    for (int k = 1; k < HB; ++k) {
+        uint32_t w = ~0u;
+#pragma unroll
+        for (int l = 0; l < Levels<HB>::L; ++l) w &= ((k >> l) & 1) ? ~S[l] : S[l];
+        cnt[k] += __popc(w);
+    }
+}
+
+// Packed-input words of the degenerate value row: every B-bit field = 2^(B-1).
+template <int B>
+__host__ __device__ constexpr uint32_t degenerate_field_word(int w) {
+    uint32_t r = 0;
+    for (int b = 0; b < 32; ++b) {
+        const int bit = 32 * w + b;
+        if (((1 << (B - 1)) >> (bit % B)) & 1) r |= 1u << b;
+    }
+    return r;
 }
 
 // Phases A and B: the row's rotation u = H (D x) into TMEM columns [0, D) of
@@ -233,7 +323,7 @@ __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, 
         tqdev::tmem_st_32x32b_x32(tlane + 32 * c, v);
     }
     tqdev::tmem_wait_st();
-    float n2 = 0.f;
+    float2 n2p = make_float2(0.f, 0.f);
 #pragma unroll 1
     for (int g = 0; g < 4; ++g) {
         float w[NC][8];
@@ -258,15 +348,15 @@ __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, 
                     }
 #pragma unroll
             for (int c = 0; c < NC; ++c) {
-                n2 = fmaf(w[c][i], w[c][i], n2);
-                n2 = fmaf(w[c][i + 1], w[c][i + 1], n2);
+                const float2 wc = make_float2(w[c][i], w[c][i + 1]);
+                n2p = fma2(wc, wc, n2p);
             }
         }
 #pragma unroll
         for (int c = 0; c < NC; ++c) tqdev::tmem_st_32x32b_x8(tlane + 32 * c + 8 * g, w[c]);
     }
     tqdev::tmem_wait_st();
-    return n2;
+    return n2p.x + n2p.y;
 }
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
@@ -278,6 +368,7 @@ template <int D, int BV, typename Tin>
 __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_constant__ EncodeParams p) {
     constexpr int HV = (1 << BV) / 2;
     constexpr int NC = D / 32;
+    constexpr uint32_t FMASK = (1u << BV) - 1u;
     __shared__ __align__(16) uint32_t s_mask[Chunk<Tin>::MASK_WORDS * NC];
     __shared__ float s_mag2[16];
     __shared__ uint32_t s_tmem;
@@ -295,7 +386,6 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
     tqdev::tc_fence_after();
     const uint32_t tlane = s_tmem + ((uint32_t)(warp * 32) << 16);
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
-    float nb[16];
 #pragma unroll 1
     for (int tile = 0; tile < ENC_TILES; ++tile) {
         const int64_t t0 = tb0 + tile * ENC_ROWS;
@@ -304,38 +394,90 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
         const bool valid = t < p.T;
         const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
         const bool nonfinite = !(n2 <= 3.0e38f);
-        const bool degenerate = nonfinite || !(n2 > 0.f);
+        const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
         const float n = sqrtf(n2 * (1.f / D));
-#pragma unroll
-        for (int k = 0; k < HV - 1; ++k) nb[k] = n * p.pb[k];
         float c2 = 0.f;
+        if constexpr (HV <= 8) {
+            float rb[8];
+            row_bounds<HV>(n, p.pb, rb);
+            int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            // HV + magnitude index lands in the low bits of K = 2^23 + HV + sum T_L 2^L
+            const float magic = 8388608.0f + (float)HV;
 #pragma unroll 1
-        for (int c = 0; c < NC; ++c) {
-            float u[32];
-            tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
-            tqdev::tmem_wait_ld();
-            uint32_t f[BV];
+            for (int c = 0; c < NC; ++c) {
+                float u[32];
+                tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
+                tqdev::tmem_wait_ld();
+                uint32_t f[BV], S[3] = {0u, 0u, 0u};
 #pragma unroll
-            for (int w = 0; w < BV; ++w) f[w] = 0u;
+                for (int w = 0; w < BV; ++w) f[w] = 0u;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                uint32_t idx;
-                if (degenerate) {
-                    idx = HV;
-                } else {
-                    const uint32_t cnt = mag_index<HV>(fabsf(u[i]), nb);
-                    idx = u[i] < 0.f ? (uint32_t)(HV - 1) - cnt : (uint32_t)HV + cnt;
-                    c2 += s_mag2[cnt];
+                for (int j = 15; j >= 0; --j) {
+                    const float2 A = make_float2(fabsf(u[2 * j]), fabsf(u[2 * j + 1]));
+                    float2 T[3], dd[3];
+                    search2<HV>(A, rb, T, dd);
+                    float2 K = add2(T[0], dup2(magic));
+                    if constexpr (HV >= 4) K = fma2(T[1], dup2(2.f), K);
+                    if constexpr (HV >= 8) K = fma2(T[2], dup2(4.f), K);
+#pragma unroll
+                    for (int h = 1; h >= 0; --h) {
+                        const int i = 2 * j + h;
+                        const uint32_t kb = __float_as_uint(h ? K.y : K.x);
+                        const uint32_t sg = (uint32_t)((int32_t)__float_as_uint(u[i]) >> 31);
+                        const uint32_t idx = (kb ^ sg) & FMASK;   // negative: HV - 1 - cell
+                        const int bit = BV * i;
+                        f[bit / 32] |= idx << (bit % 32);
+                        if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
+#pragma unroll
+                        for (int l = 0; l < Levels<HV>::L; ++l) S[l] = push_sign(S[l], h ? dd[l].y : dd[l].x);
+                    }
                 }
-                const int bit = BV * i;
-                f[bit / 32] |= idx << (bit % 32);
-                if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
-            }
-            if (valid) {
+                count_cells<HV>(S, cnt);
+                if (valid) {
 #pragma unroll
-                for (int w = 0; w < BV; ++w) dst[BV * c + w] = f[w];
+                    for (int w = 0; w < BV; ++w)
+                        dst[BV * c + w] = degenerate ? degenerate_field_word<BV>(BV * c + w) : f[w];
+                }
+            }
+            int rest = D;
+#pragma unroll
+            for (int k = 1; k < HV; ++k) {
+                rest -= cnt[k];
+                c2 = fmaf((float)cnt[k], s_mag2[k], c2);
+            }
+            c2 = fmaf((float)rest, s_mag2[0], c2);
+        } else {
+            float nb[16];
+#pragma unroll
+            for (int k = 0; k < HV - 1; ++k) nb[k] = n * p.pb[k];
+#pragma unroll 1
+            for (int c = 0; c < NC; ++c) {
+                float u[32];
+                tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
+                tqdev::tmem_wait_ld();
+                uint32_t f[BV];
+#pragma unroll
+                for (int w = 0; w < BV; ++w) f[w] = 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    uint32_t idx;
+                    if (degenerate) {
+                        idx = HV;
+                    } else {
+                        const uint32_t cell = mag_index<HV>(fabsf(u[i]), nb);
+                        idx = u[i] < 0.f ? (uint32_t)(HV - 1) - cell : (uint32_t)HV + cell;
+                        c2 += s_mag2[cell];
+                    }
+                    const int bit = BV * i;
+                    f[bit / 32] |= idx << (bit % 32);
+                    if ((bit % 32) + BV > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
+                }
+                if (valid) {
+#pragma unroll
+                    for (int w = 0; w < BV; ++w) dst[BV * c + w] = f[w];
+                }
             }
         }
         if (valid) dst[BV * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2));
@@ -356,7 +498,6 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     constexpr int NC = D / 32;                 // chunks = 32-bit words per bit plane
     constexpr int ATOM = ENC_ROWS * 128;       // bytes of one 128-row x 128-byte swizzle column
     constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
-    constexpr int MB = BK > 1 ? BK - 1 : 1;     // magnitude bit planes (at least one slot)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // misc region [0, 1024): sign masks, centroid magnitudes, barriers
@@ -401,7 +542,6 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     }
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
-    float nb[16];
     int tiles_done = 0;
 #pragma unroll 1
     for (int tile = 0; tile < ENC_TILES && !*s_abort; ++tile) {
@@ -412,44 +552,75 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
         const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
         const bool nonfinite = !(n2 <= 3.0e38f);
-        const bool degenerate = nonfinite || !(n2 > 0.f);
+        const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
         const float n = sqrtf(n2 * (1.f / D));
-#pragma unroll
-        for (int k = 0; k < HK - 1; ++k) nb[k] = n * p.pb[k];
+        float rb[8];
+        row_bounds<HK>(n, p.pb, rb);
         // C: index planes, the signed centroids (to TMEM columns [d, 2d)),
-        // sum C[idx]^2 and sum u C[idx]
-        float c2 = 0.f, uc = 0.f;
+        // cell counts (for sum C[idx]^2) and sum |u| C[idx]
+        int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        float2 ucp = make_float2(0.f, 0.f);
 #pragma unroll 1
         for (int c = 0; c < NC; ++c) {
             float u[32];
             tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
             tqdev::tmem_wait_ld();
-            uint32_t negw = 0u, mbw[MB];
+            uint32_t S[3] = {0u, 0u, 0u}, Sn = 0u;
 #pragma unroll
-            for (int q = 0; q < MB; ++q) mbw[q] = 0u;
+            for (int j = 15; j >= 0; --j) {
+                const float2 A = make_float2(fabsf(u[2 * j]), fabsf(u[2 * j + 1]));
+                float2 T[3], dd[3];
+                search2<HK>(A, rb, T, dd);
+                float2 cm;
+                if constexpr (HK == 1) {
+                    cm = dup2(p.cl[0]);
+                } else if constexpr (HK == 2) {
+                    cm = fma2(T[0], dup2(p.cl[0]), dup2(p.cl[1]));
+                } else if constexpr (HK == 4) {
+                    const float2 lo = fma2(T[1], dup2(p.cl[0]), dup2(p.cl[1]));
+                    const float2 df = fma2(T[1], dup2(p.cl[2]), dup2(p.cl[3]));
+                    cm = fma2(T[0], df, lo);
+                } else {
+                    const float2 lo = fma2(T[1], fma2(T[2], dup2(p.cl[0]), dup2(p.cl[1])),
+                                           fma2(T[2], dup2(p.cl[2]), dup2(p.cl[3])));
+                    const float2 df = fma2(T[1], fma2(T[2], dup2(p.cl[4]), dup2(p.cl[5])),
+                                           fma2(T[2], dup2(p.cl[6]), dup2(p.cl[7])));
+                    cm = fma2(T[0], df, lo);
+                }
+                ucp = fma2(A, cm, ucp);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const uint32_t cnt = mag_index<HK>(fabsf(u[i]), nb);
-                negw |= (__float_as_uint(u[i]) >> 31) << i;
+                for (int h = 1; h >= 0; --h) {
 #pragma unroll
-                for (int q = 0; q < BK - 1; ++q) mbw[q] |= ((cnt >> q) & 1u) << i;
-                const float cm = s_mag[cnt];
-                c2 = fmaf(cm, cm, c2);
-                uc = fmaf(fabsf(u[i]), cm, uc);
-                u[i] = copysignf(cm, u[i]);
+                    for (int l = 0; l < Levels<HK>::L; ++l) S[l] = push_sign(S[l], h ? dd[l].y : dd[l].x);
+                    Sn = push_sign(Sn, u[2 * j + h]);
+                }
+                u[2 * j] = copysignf(cm.x, u[2 * j]);
+                u[2 * j + 1] = copysignf(cm.y, u[2 * j + 1]);
             }
             tqdev::tmem_st_32x32b_x32(tlane + D + 32 * c, u);
+            count_cells<HK>(S, cnt);
             if (valid) {
                 // ascending index: top bit = non-negative, low bits = magnitude
                 // index, complemented for negative values
 #pragma unroll
                 for (int q = 0; q < BK - 1; ++q)
-                    dst[q * NC + c] = degenerate ? (((HK >> q) & 1) ? ~0u : 0u) : (mbw[q] ^ negw);
-                dst[(BK - 1) * NC + c] = degenerate ? ~0u : ~negw;
+                    dst[q * NC + c] = degenerate ? (((HK >> q) & 1) ? ~0u : 0u) : (~S[q] ^ Sn);
+                dst[(BK - 1) * NC + c] = degenerate ? ~0u : ~Sn;
             }
         }
         tqdev::tmem_wait_st();
+        float c2 = 0.f;
+        {
+            int rest = D;
+#pragma unroll
+            for (int k = 1; k < HK; ++k) {
+                rest -= cnt[k];
+                c2 = fmaf((float)cnt[k], s_mag2[k], c2);
+            }
+            c2 = fmaf((float)rest, s_mag2[0], c2);
+        }
+        const float uc = ucp.x + ucp.y;
         const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
         // |e|^2 from the sums, only to scale the MMA operand (the stored gamma
         // comes from the direct sum below)
@@ -457,7 +628,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         e2a = fmaxf(e2a, 1e-10f * n2);
         const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
         // D: residual u - n_s C[idx] as binary16 hi + lo, swizzled K-major operand
-        float e2 = 0.f;
+        float2 e2p = make_float2(0.f, 0.f);
 #pragma unroll 1
         for (int c = 0; c < NC; ++c) {
             float u[32], cv[32];
@@ -469,19 +640,15 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 uint32_t hw[4], lw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float a[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int i = 8 * j8 + 2 * e + h;
-                        const float ee = fmaf(-ns, cv[i], u[i]);
-                        e2 = fmaf(ee, ee, e2);
-                        a[h] = degenerate ? 0.f : ee * sc;
-                    }
-                    const __half2 hh = __floats2half2_rn(a[0], a[1]);
-                    const float2 hf = __half22float2(hh);
-                    const __half2 ll = __floats2half2_rn(a[0] - hf.x, a[1] - hf.y);
-                    hw[e] = (uint32_t)__half_as_ushort(__low2half(hh)) | ((uint32_t)__half_as_ushort(__high2half(hh)) << 16);
-                    lw[e] = (uint32_t)__half_as_ushort(__low2half(ll)) | ((uint32_t)__half_as_ushort(__high2half(ll)) << 16);
+                    const int i = 8 * j8 + 2 * e;
+                    const float2 E = fma2(dup2(-ns), make_float2(cv[i], cv[i + 1]), make_float2(u[i], u[i + 1]));
+                    e2p = fma2(E, E, e2p);
+                    const float2 a = mul2(E, dup2(sc));
+                    const __half2 hh = __floats2half2_rn(a.x, a.y);
+                    const float2 l = sub2(a, __half22float2(hh));
+                    const __half2 ll = __floats2half2_rn(l.x, l.y);
+                    hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                    lw[e] = *reinterpret_cast<const uint32_t *>(&ll);
                 }
                 const int kk = 4 * c + j8;          // 16-byte unit of the row
                 const int off = (kk / 8) * ATOM + tid * 128 + (((kk % 8) ^ (tid & 7)) << 4);
@@ -489,6 +656,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 *reinterpret_cast<uint4 *>(aLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
         }
+        const float e2 = e2p.x + e2p.y;
         if (valid) {
             const int tail = BK * NC + M / 32;
             dst[tail] = __float_as_uint(ns);
@@ -535,10 +703,15 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 float pv[32];
                 tqdev::tmem_ld_32x32b_x32_nowait(tlane + (uint32_t)(c * 32), pv);
                 tqdev::tmem_wait_ld();
-                uint32_t word = 0u;
+                // bit i = [p_i >= 0]: collect the sign bits (p + 0 turns -0 into +0)
+                uint32_t neg = 0u;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) word |= (pv[i] >= 0.f ? 1u : 0u) << i;
-                if (valid) sdst[c] = degenerate ? ~0u : word;
+                for (int j = 15; j >= 0; --j) {
+                    const float2 q = add2(make_float2(pv[2 * j], pv[2 * j + 1]), dup2(0.f));
+                    neg = push_sign(neg, q.y);
+                    neg = push_sign(neg, q.x);
+                }
+                if (valid) sdst[c] = degenerate ? ~0u : ~neg;
             }
         }
         ++tiles_done;
@@ -633,6 +806,35 @@ tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype d
         const int HB = (1 << B) / 2;
         for (int i = 0; i < HB; ++i) p.mag[i] = cb[HB + i];
         for (int i = 0; i + 1 < HB; ++i) p.pb[i] = bd[HB + i];
+        if (keys) {
+            // cell k = sum_L T_L 2^L; the magnitude C_k written as the
+            // multilinear form the key kernel evaluates in the bits T_L
+            double m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            for (int i = 0; i < HB && i < 8; ++i) m[i] = cb[HB + i];
+            double c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (HB == 1) {
+                c[0] = m[0];
+            } else if (HB == 2) {
+                c[0] = m[1] - m[0];
+                c[1] = m[0];
+            } else if (HB == 4) {
+                c[0] = m[2] - m[0];
+                c[1] = m[0];
+                c[2] = (m[3] - m[2]) - (m[1] - m[0]);
+                c[3] = m[1] - m[0];
+            } else if (HB == 8) {
+                const double d0 = m[1] - m[0], d2 = m[3] - m[2], d4 = m[5] - m[4], d6 = m[7] - m[6];
+                c[0] = m[6] - m[4] - m[2] + m[0];
+                c[1] = m[2] - m[0];
+                c[2] = m[4] - m[0];
+                c[3] = m[0];
+                c[4] = d6 - d4 - d2 + d0;
+                c[5] = d2 - d0;
+                c[6] = d4 - d0;
+                c[7] = d0;
+            }
+            for (int i = 0; i < 8; ++i) p.cl[i] = (float)c[i];
+        }
         cudaError_t e;
         switch (dtype) {
             case TQ_F32: e = launch_side<float>(ctx, keys, p, grid, stream); break;

@@ -29,11 +29,12 @@ struct tq_ctx {
     CUtensorMap tmap_S;             // 2-D view of d_S: inner d, outer heads*m
     // Lloyd-Max codebooks of N(0,1): centroids ascending and boundaries.
     float ck[TQ_MAX_LEVELS], bk[TQ_MAX_LEVELS], cv[TQ_MAX_LEVELS], bv[TQ_MAX_LEVELS];
+    struct TqBook *d_book;          // device copy of the positive halves (TqBook)
 };
 
-// Codebook data handed to kernels by value: positive-half magnitudes of the
-// centroids and positive boundaries.  For L levels, mag[k] = c[L/2 + k]
-// (k < L/2) and pb[k] = beta[L/2 + k] (k < L/2 - 1).
+// Positive halves of the codebooks: magnitudes of the centroids and the
+// positive boundaries.  For L levels, mag[k] = c[L/2 + k] (k < L/2) and
+// pb[k] = beta[L/2 + k] (k < L/2 - 1).
 struct TqBook {
     float kmag[16];
     float kpb[16];

@@ -19,9 +19,10 @@
 #include "tq_internal.cuh"
 
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
-tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch, int Hq,
-                           int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes, cudaStream_t stream,
-                           int n_sms);
+struct TqAppend;
+tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,
+                           int Hq, int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes,
+                           cudaStream_t stream, int n_sms, const TqAppend *app = nullptr);
 tq_status tq_validate_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch, int Hq,
                              int Hkv, const void *out, tq_dtype out_dtype, bool build_tables);
 int tq_device_sms(int dev);

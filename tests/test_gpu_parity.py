@@ -125,6 +125,36 @@ def test_encode_nonfinite_and_zero_rows():
     assert gc.status() == (0, 0)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
+def test_encode_power_of_two_scaling_and_tiny_rows(bits):
+    """Scaling fp32 input by 2^40 or 2^-40 scales every fp32 step of the encoder
+    exactly, so the codes are identical and the stored norms scale by the same
+    power of two.  Rows whose rotated sum of squares d|x|^2 falls below the
+    smallest normal float are encoded exactly like zero rows, without being
+    counted as non-finite."""
+    g = torch.Generator().manual_seed(77 + bits)
+    k = torch.randn(1, 2, 150, 128, generator=g)
+    v = torch.randn(1, 2, 150, 128, generator=g)
+    gc = tq.Codec(128, bits, 128, 5)
+    out = []
+    for s in (1.0, 2.0 ** 40, 2.0 ** -40, 2.0 ** -75, 0.0):
+        c = gc.alloc(1, 2, 160)
+        gc.encode_kv((k * s).to(DEV), (v * s).to(DEV), c)
+        out.append((c.k[:, :, :150].cpu().numpy(), c.v[:, :, :150].cpu().numpy()))
+    torch.cuda.synchronize()
+    assert gc.status() == (0, 0)
+    base_k, base_v = out[0]
+    for (kk, vv), s in zip(out[1:3], (2.0 ** 40, 2.0 ** -40)):
+        assert np.array_equal(kk[..., :-8], base_k[..., :-8]) and np.array_equal(vv[..., :-4], base_v[..., :-4])
+        kn = kk[..., -8:].copy().view(np.float32)
+        vn = vv[..., -4:].copy().view(np.float32)
+        assert np.array_equal(kn, (base_k[..., -8:].copy().view(np.float32) * np.float32(s)))
+        assert np.array_equal(vn, (base_v[..., -4:].copy().view(np.float32) * np.float32(s)))
+    tiny, zero = out[3], out[4]
+    assert np.array_equal(tiny[0], zero[0]) and np.array_equal(tiny[1], zero[1])
+    assert not zero[0][..., -8:].any() and not zero[1][..., -4:].any()
+
+
 def test_encode_empty_and_single_token():
     gc = tq.Codec(128, 4, 128, 1)
     cache = gc.alloc(1, 1, 16)
