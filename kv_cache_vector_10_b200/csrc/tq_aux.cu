@@ -20,51 +20,72 @@ namespace {
 constexpr int AUX_THREADS = 128;
 
 // Block-wide: q_rot = H (D q) / sqrt(d) and sq = S q_rot, in shared memory.
+// Warp 0 rotates (lane l holds coordinates l + 32k: the stages of stride
+// >= 32 run in registers, the others across lanes by shuffles); then each
+// thread computes whole projections sq_i = <S_i, q_rot>, with all 16-byte
+// loads of its row of S in flight at once.
 template <int D>
 __device__ void prep_query(const float *sq_in, const uint32_t *signs, const __half *S, int M, float *s_qr,
                            float *s_sq) {
     const int tid = threadIdx.x;
-    for (int j = tid; j < D; j += blockDim.x) {
-        const float x = sq_in[j];
-        s_qr[j] = ((signs[j / 32] >> (j % 32)) & 1) ? -x : x;
-    }
-    __syncthreads();
-    for (int len = 1; len < D; len <<= 1) {
-        for (int i = tid; i < D / 2; i += blockDim.x) {
-            const int j = (i / len) * 2 * len + (i % len);
-            const float a = s_qr[j], b = s_qr[j + len];
-            s_qr[j] = a + b;
-            s_qr[j + len] = a - b;
+    if (tid < 32) {
+        constexpr int V = D / 32;
+        const int lane = tid;
+        float x[V];
+#pragma unroll
+        for (int k = 0; k < V; ++k) {
+            const int j = lane + 32 * k;
+            const float v = sq_in[j];
+            x[k] = ((signs[j / 32] >> (j % 32)) & 1) ? -v : v;
         }
-        __syncthreads();
-    }
-    const float sc = rsqrtf((float)D);
-    for (int j = tid; j < D; j += blockDim.x) s_qr[j] *= sc;
-    __syncthreads();
-    // sq = S q_rot: LPR lanes per row, 8 binary16 values (16 bytes) per lane
-    constexpr int LPR = D / 8;
-    constexpr int RPW = 32 / LPR;   // rows per warp pass
-    const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    const int sub = lane / LPR, part = lane % LPR;
-    float qv[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qv[e] = s_qr[8 * part + e];
-    for (int i0 = warp * RPW; i0 < M; i0 += nwarps * RPW) {
-        const int i = i0 + sub;
-        float acc = 0.f;
-        if (i < M) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(S + (int64_t)i * D + 8 * part);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int len = 1; len < V; len <<= 1)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
-                acc = fmaf(f.x, qv[2 * e], acc);
-                acc = fmaf(f.y, qv[2 * e + 1], acc);
+            for (int k = 0; k < V; k += 2 * len)
+#pragma unroll
+                for (int kk = k; kk < k + len; ++kk) {
+                    const float a = x[kk], b = x[kk + len];
+                    x[kk] = a + b;
+                    x[kk + len] = a - b;
+                }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const float y = __shfl_xor_sync(0xffffffffu, x[k], o);
+                x[k] = upper ? y - x[k] : x[k] + y;
             }
         }
+        const float sc = rsqrtf((float)D);
 #pragma unroll
-        for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (part == 0 && i < M) s_sq[i] = acc;
+        for (int k = 0; k < V; ++k) s_qr[lane + 32 * k] = x[k] * sc;
+    }
+    __syncthreads();
+    const float4 *q4 = reinterpret_cast<const float4 *>(s_qr);
+    for (int i = tid; i < M; i += blockDim.x) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(S + (int64_t)i * D);
+        uint4 w[D / 8];
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) w[c] = __ldg(row + c);
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const float4 qa = q4[2 * c], qb = q4[2 * c + 1];
+            const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].x));
+            const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].y));
+            const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].z));
+            const float2 f3 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].w));
+            acc0 = fmaf(f0.x, qa.x, acc0);
+            acc1 = fmaf(f0.y, qa.y, acc1);
+            acc0 = fmaf(f1.x, qa.z, acc0);
+            acc1 = fmaf(f1.y, qa.w, acc1);
+            acc0 = fmaf(f2.x, qb.x, acc0);
+            acc1 = fmaf(f2.y, qb.y, acc1);
+            acc0 = fmaf(f3.x, qb.z, acc0);
+            acc1 = fmaf(f3.y, qb.w, acc1);
+        }
+        s_sq[i] = acc0 + acc1;
     }
     __syncthreads();
 }
@@ -82,7 +103,7 @@ struct ScoresParams {
 
 template <int D>
 __global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_constant__ ScoresParams p) {
-    __shared__ float s_qr[D];
+    __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
     const int j = blockIdx.y, b = blockIdx.z;
     const int h = j / (p.Hq / p.Hkv);
@@ -345,7 +366,7 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
 template <int D, typename Tq>
 __global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
     __shared__ float s_in[D];
-    __shared__ float s_qr[D];
+    __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
     __shared__ float s_red[AUX_THREADS / 32];
     __shared__ uint8_t s_idx[D];

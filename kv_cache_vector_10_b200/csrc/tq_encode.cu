@@ -30,8 +30,9 @@
 //      into binary16 hi + lo, written to shared memory in the 128-byte
 //      swizzled K-major layout; one thread issues 2*(d/16) tcgen05.mma
 //      (M = 128 rows, N = m projections, K = 16) against S (binary16, loaded
-//      once per CTA by TMA), accumulating P = e S^T in fp32 in TMEM (the
-//      same columns the row used).  Two passes make the projection accurate
+//      once per CTA by TMA), accumulating P = e S^T in fp32 in TMEM columns
+//      [d, d + m); while it runs, the threads rotate the next tile into
+//      columns [0, d).  Two passes make the projection accurate
 //      to ~1e-7 relative, so sign bits agree with an fp64 evaluation away
 //      from |p| ~ 1e-6.  Each thread then reads its row of P (tcgen05.ld)
 //      and stores the m-bit sign plane.
@@ -41,6 +42,8 @@
 // overflows fp32 (|x| beyond ~1.5e18) are counted as non-finite; rows where
 // it falls below the smallest normal float (|x| below ~1e-20) are encoded as
 // zero rows (the exact search steps need normal-range boundaries).
+#include <type_traits>
+
 #include "tq_internal.cuh"
 
 namespace {
@@ -127,6 +130,44 @@ struct Chunk<__nv_bfloat16> {
         }
     }
 };
+
+// The same conversion from 16-byte words already in registers (16-bit
+// types: 4 words per chunk).
+template <typename Tin>
+__device__ __forceinline__ void chunk_from_words(const uint4 *q4, const uint32_t *sm, float (&x)[32]) {
+    static_assert(sizeof(Tin) == 2, "16-bit inputs");
+    const uint4 *m = reinterpret_cast<const uint4 *>(sm);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 q = q4[i], f = m[i];
+        const uint32_t w[4] = {q.x ^ f.x, q.y ^ f.y, q.z ^ f.z, q.w ^ f.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if constexpr (std::is_same<Tin, __half>::value) {
+                const float2 v = __half22float2(__halves2half2(__ushort_as_half((unsigned short)(w[e] & 0xFFFFu)),
+                                                               __ushort_as_half((unsigned short)(w[e] >> 16))));
+                x[8 * i + 2 * e] = v.x;
+                x[8 * i + 2 * e + 1] = v.y;
+            } else {
+                x[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+                x[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+        }
+    }
+}
+
+// One 16-bit input row as 16-byte words, loaded ahead of its rotation so
+// the load latency overlaps the previous tile's work.
+template <int D>
+struct RowWords {
+    uint4 w[D / 8];
+};
+template <int D, typename Tin>
+__device__ __forceinline__ void load_row_words(const Tin *row, bool valid, RowWords<D> &r) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(row);
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) r.w[i] = valid ? __ldg(p + i) : make_uint4(0u, 0u, 0u, 0u);
+}
 
 // Per-head input sign masks, in input-word order.
 template <typename Tin, int D>
@@ -306,6 +347,9 @@ __host__ __device__ constexpr uint32_t degenerate_field_word(int w) {
 
 // Phases A and B: the row's rotation u = H (D x) into TMEM columns [0, D) of
 // this thread's lane; returns |u|^2.  Rows past the end rotate zeros.
+template <int D>
+__device__ __forceinline__ float cross_chunk_stages(uint32_t tlane);
+
 template <int D, typename Tin>
 __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, const uint32_t *s_mask,
                                                     uint32_t tlane) {
@@ -322,6 +366,29 @@ __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, 
         fwht32(v);
         tqdev::tmem_st_32x32b_x32(tlane + 32 * c, v);
     }
+    return cross_chunk_stages<D>(tlane);
+}
+
+// The same from a row already in registers (16-bit inputs; invalid rows were
+// loaded as zeros).
+template <int D, typename Tin>
+__device__ __forceinline__ float rotate_words_to_tmem(const RowWords<D> &r, const uint32_t *s_mask,
+                                                      uint32_t tlane) {
+    constexpr int NC = D / 32;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        float v[32];
+        chunk_from_words<Tin>(r.w + 4 * c, s_mask + c * Chunk<Tin>::MASK_WORDS, v);
+        fwht32(v);
+        tqdev::tmem_st_32x32b_x32(tlane + 32 * c, v);
+    }
+    return cross_chunk_stages<D>(tlane);
+}
+
+// Phase B: the butterfly stages across chunks, on 8-column slices; returns |u|^2.
+template <int D>
+__device__ __forceinline__ float cross_chunk_stages(uint32_t tlane) {
+    constexpr int NC = D / 32;
     tqdev::tmem_wait_st();
     float2 n2p = make_float2(0.f, 0.f);
 #pragma unroll 1
@@ -360,7 +427,7 @@ __device__ __forceinline__ float rotate_row_to_tmem(const Tin *row, bool valid, 
 }
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
-    return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : 256u;
+    return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : cols <= 256 ? 256u : 512u;
 }
 
 // ------------------------------------------------------------------ values
@@ -386,13 +453,27 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
     tqdev::tc_fence_after();
     const uint32_t tlane = s_tmem + ((uint32_t)(warp * 32) << 16);
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
+    // 16-bit inputs: each tile's rows are loaded into registers during the
+    // previous tile's quantization
+    constexpr bool PF = sizeof(Tin) == 2;
+    RowWords<D> raw;
+    if constexpr (PF) {
+        if (tb0 < p.T) load_row_words<D, Tin>(src + (tb0 + tid) * p.st, tb0 + tid < p.T, raw);
+    }
 #pragma unroll 1
     for (int tile = 0; tile < ENC_TILES; ++tile) {
         const int64_t t0 = tb0 + tile * ENC_ROWS;
         if (t0 >= p.T) break;
         const int64_t t = t0 + tid;
         const bool valid = t < p.T;
-        const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+        float n2;
+        if constexpr (PF) {
+            n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
+            if (tile + 1 < ENC_TILES && t0 + ENC_ROWS < p.T)
+                load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+        } else {
+            n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+        }
         const bool nonfinite = !(n2 <= 3.0e38f);
         const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
@@ -516,7 +597,9 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     const int head = (int)(bh % p.H);
     const int64_t b = bh / p.H;
     const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_ROWS;
-    const uint32_t tmem_cols = tmem_cols_for(M > 2 * D ? M : 2 * D);   // U [0,d), C [d,2d); P reuses [0,m)
+    // U [0, d); C [d, 2d); P [d, d + m) (written by the MMA while the next
+    // tile's rotation fills U)
+    const uint32_t tmem_cols = tmem_cols_for(D + (M > D ? M : D));
     build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
     if (tid < 16) {
         const float mg = tid < HK ? p.mag[tid] : 0.f;
@@ -542,15 +625,32 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     }
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
-    int tiles_done = 0;
+    const uint32_t tP = tlane + (uint32_t)D;   // this lane's P columns
+    int ntiles = 0;
+    while (ntiles < ENC_TILES && tb0 + (int64_t)ntiles * ENC_ROWS < p.T) ++ntiles;
+    // A, B of the first tile; later tiles' rotations overlap the previous MMA,
+    // and (16-bit inputs) their rows are loaded into registers a tile ahead
+    constexpr bool PF = sizeof(Tin) == 2;
+    RowWords<D> raw;
+    float n2 = 0.f;
+    if (ntiles > 0 && !*s_abort) {
+        const int64_t t = tb0 + tid;
+        if constexpr (PF) {
+            load_row_words<D, Tin>(src + t * p.st, t < p.T, raw);
+            n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
+        } else {
+            n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, t < p.T, s_mask, tlane);
+        }
+    }
 #pragma unroll 1
-    for (int tile = 0; tile < ENC_TILES && !*s_abort; ++tile) {
-        const int64_t t0 = tb0 + tile * ENC_ROWS;
-        if (t0 >= p.T) break;
-        const int64_t t = t0 + tid;
+    for (int tile = 0; tile < ntiles; ++tile) {
+        if (*s_abort) break;   // uniform: set before the barrier that ends the previous tile
+        const int64_t t = tb0 + tile * ENC_ROWS + tid;
         const bool valid = t < p.T;
+        if constexpr (PF) {
+            if (tile + 1 < ntiles) load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+        }
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
-        const float n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
         const bool nonfinite = !(n2 <= 3.0e38f);
         const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
@@ -662,15 +762,16 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
             dst[tail] = __float_as_uint(ns);
             dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)));
         }
-        // E: the QJL projection on the tensor cores (writes TMEM columns [0, M))
+        // E: the QJL projection on the tensor cores (TMEM columns [d, d + m))
         tqdev::fence_proxy_async_smem();
         tqdev::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            const bool ok = tiles_done > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
+            const bool ok = tile > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
             if (!ok) {
                 atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
                 *s_abort = 1;
+                tqdev::mbar_arrive(&bars[1]);   // release the epilogue wait below
             } else {
                 tqdev::tc_fence_after();
                 const uint32_t idesc = tqdev::idesc_f16_f32(M);
@@ -682,42 +783,45 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t a_addr = abase + (ks / 4) * ATOM + (ks % 4) * 32;
                         const uint32_t b_addr = bbase + (ks / 4) * (M * 128) + (ks % 4) * 32;
-                        tqdev::mma_f16_ss(tmem_base, tqdev::smem_desc_sw128(a_addr), tqdev::smem_desc_sw128(b_addr),
-                                          idesc, (pass | ks) != 0);
+                        tqdev::mma_f16_ss(tmem_base + (uint32_t)D, tqdev::smem_desc_sw128(a_addr),
+                                          tqdev::smem_desc_sw128(b_addr), idesc, (pass | ks) != 0);
                     }
                 }
                 tqdev::mma_commit(&bars[1]);
             }
         }
-        __syncthreads();
-        if (*s_abort) break;
-        // F: sign epilogue
-        if (!tqdev::mbar_wait_bounded(&bars[1], (uint32_t)(tiles_done & 1))) {
-            if (tid == 0) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
-            *s_abort = 1;   // benign race: every writer stores 1
-        } else {
-            tqdev::tc_fence_after();
-            uint32_t *sdst = dst + BK * NC;
-#pragma unroll 1
-            for (int c = 0; c < M / 32; ++c) {
-                float pv[32];
-                tqdev::tmem_ld_32x32b_x32_nowait(tlane + (uint32_t)(c * 32), pv);
-                tqdev::tmem_wait_ld();
-                // bit i = [p_i >= 0]: collect the sign bits (p + 0 turns -0 into +0)
-                uint32_t neg = 0u;
-#pragma unroll
-                for (int j = 15; j >= 0; --j) {
-                    const float2 q = add2(make_float2(pv[2 * j], pv[2 * j + 1]), dup2(0.f));
-                    neg = push_sign(neg, q.y);
-                    neg = push_sign(neg, q.x);
-                }
-                if (valid) sdst[c] = degenerate ? ~0u : ~neg;
-            }
+        // A, B of the next tile while the MMA runs (they touch only U)
+        float n2_next = 0.f;
+        if (tile + 1 < ntiles) {
+            const int64_t tn = t + ENC_ROWS;
+            if constexpr (PF) n2_next = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
+            else n2_next = rotate_row_to_tmem<D, Tin>(src + tn * p.st, tn < p.T, s_mask, tlane);
         }
-        ++tiles_done;
-        tqdev::tc_fence_before();
-        __syncthreads();
+        // F: sign epilogue
+        const bool done = tqdev::mbar_wait_bounded(&bars[1], (uint32_t)(tile & 1));
+        if (__syncthreads_or(!done || *s_abort)) {
+            if (tid == 0 && !done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+            if (tid == 0) *s_abort = 1;
+            break;
+        }
         tqdev::tc_fence_after();
+        uint32_t *sdst = dst + BK * NC;
+#pragma unroll 1
+        for (int c = 0; c < M / 32; ++c) {
+            float pv[32];
+            tqdev::tmem_ld_32x32b_x32_nowait(tP + (uint32_t)(c * 32), pv);
+            tqdev::tmem_wait_ld();
+            // bit i = [p_i >= 0]: collect the sign bits (p + 0 turns -0 into +0)
+            uint32_t neg = 0u;
+#pragma unroll
+            for (int j = 15; j >= 0; --j) {
+                const float2 q = add2(make_float2(pv[2 * j], pv[2 * j + 1]), dup2(0.f));
+                neg = push_sign(neg, q.y);
+                neg = push_sign(neg, q.x);
+            }
+            if (valid) sdst[c] = degenerate ? ~0u : ~neg;
+        }
+        n2 = n2_next;
     }
     tqdev::tc_fence_before();
     __syncthreads();
@@ -731,7 +835,9 @@ template <int D, typename Tin>
 cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, int64_t grid, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     auto go = [&](auto kern) {
-        const size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+        size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+        // a CTA holding all 512 TMEM columns (d + m > 256) gets an SM to itself
+        if (D + p.M > 256 && smem < 120 * 1024) smem = 120 * 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) {
             cudaGetLastError();   // do not leave the failure as the thread's sticky last error
