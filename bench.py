@@ -89,11 +89,16 @@ def arm_config(workload):
     return {"workload": WORKLOAD_DESC[workload], "step": STEP_DESC[workload], "l2": L2_DESC}
 
 
-# DRAM traffic of a piece (dram__bytes_read.sum + dram__bytes_write.sum over
-# its launches) from one ncu capture, keyed by (piece, workload), with the
-# SHA-1 of the source file holding the piece's main kernel at capture time:
-# once that source changes the entry no longer applies (traffic: null).
-MEASURED_TRAFFIC = {}
+# DRAM traffic of a piece's main kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch, ncu --set full, caches flushed before
+# the launch), keyed by (piece, workload), with the SHA-1 of the source file
+# holding that kernel when the counters were taken: once the source changes
+# the entry no longer applies (traffic: null).  Summaries: profiles/.
+MEASURED_TRAFFIC = {
+    ("encode_keys", "mha_decode"): ("tq_encode.cu", "c5bf4a225cbdb7e1b79fa72f7f4140215e6c26ca", 326849024),
+    ("encode_values", "mha_decode"): ("tq_encode.cu", "c5bf4a225cbdb7e1b79fa72f7f4140215e6c26ca", 321014272),
+    ("decode", "mha_decode"): ("tq_decode.cu", "420aa8ed6238705ffaaea7f0431d3414d93fcb44", 151321344),
+}
 
 
 def measured_traffic(piece, workload):
