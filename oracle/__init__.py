@@ -38,7 +38,10 @@ class _Cfg(ctypes.Structure):
                 ("BK", ctypes.c_int), ("BV", ctypes.c_int), ("LK", ctypes.c_int),
                 ("LV", ctypes.c_int), ("norm_correct", ctypes.c_int),
                 ("ck", ctypes.c_double * 64), ("bk", ctypes.c_double * 64),
-                ("cv", ctypes.c_double * 64), ("bv", ctypes.c_double * 64)]
+                ("cv", ctypes.c_double * 64), ("bv", ctypes.c_double * 64),
+                ("rotation", ctypes.c_int)]
+
+ROTATIONS = {"hadamard": 0, "haar": 1}
 
 
 def _load():
@@ -56,6 +59,10 @@ def _load():
         _lib.tqo_fwht.argtypes = [P, ctypes.c_int]
         _lib.tqo_rotate.argtypes = [ctypes.c_int, P, P, P]
         _lib.tqo_unrotate.argtypes = [ctypes.c_int, P, P, P]
+        _lib.tqo_haar_matrix.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_int, P]
+        _lib.tqo_haar_gaussian.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_int, P]
+        _lib.tqo_rotate_dense.argtypes = [ctypes.c_int, P, P, P]
+        _lib.tqo_unrotate_dense.argtypes = [ctypes.c_int, P, P, P]
         _lib.tqo_cfg_init.restype = ctypes.c_int
         _lib.tqo_cfg_init.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         _lib.tqo_k_row_bytes.restype = ctypes.c_int
@@ -122,30 +129,54 @@ def head_tables(d: int, m: int, seed: int, h: int):
     return signs, S
 
 
-def rotate(signs, x) -> np.ndarray:
+def haar_matrix(d: int, m: int, seed: int, h: int) -> np.ndarray:
+    """The Haar rotation Q [d, d] of head h (QR of a seeded Gaussian matrix)."""
+    Q = np.zeros((d, d))
+    _load().tqo_haar_matrix(d, m, seed & 0xFFFFFFFFFFFFFFFF, h, _p(Q))
+    return Q
+
+
+def haar_gaussian(d: int, m: int, seed: int, h: int) -> np.ndarray:
+    """The Gaussian matrix G [d, d] whose QR factor is head h's Haar rotation."""
+    G = np.zeros((d, d))
+    _load().tqo_haar_gaussian(d, m, seed & 0xFFFFFFFFFFFFFFFF, h, _p(G))
+    return G
+
+
+def rotate(rot, x) -> np.ndarray:
+    """Pi x: rot is a head's signs [d] (Hadamard) or its matrix Q [d, d] (Haar)."""
     x = _f64(x)
+    rot = _f64(rot)
     out = np.zeros_like(x)
-    _load().tqo_rotate(x.shape[0], _p(_f64(signs)), _p(x), _p(out))
+    fn = _load().tqo_rotate_dense if rot.ndim == 2 else _load().tqo_rotate
+    fn(x.shape[0], _p(rot), _p(x), _p(out))
     return out
 
 
-def unrotate(signs, y) -> np.ndarray:
+def unrotate(rot, y) -> np.ndarray:
+    """Pi^T y for a head's signs or Haar matrix."""
     y = _f64(y)
+    rot = _f64(rot)
     out = np.zeros_like(y)
-    _load().tqo_unrotate(y.shape[0], _p(_f64(signs)), _p(y), _p(out))
+    fn = _load().tqo_unrotate_dense if rot.ndim == 2 else _load().tqo_unrotate
+    fn(y.shape[0], _p(rot), _p(y), _p(out))
     return out
 
 
 # ------------------------------------------------------------------- codec
 
 class Codec:
-    """One codec configuration (head_dim, bits, projections, seed) on the CPU."""
+    """One codec configuration (head_dim, bits, projections, seed, rotation)
+    on the CPU; rotation is "hadamard" (FWHT with random signs) or "haar"."""
 
-    def __init__(self, head_dim: int, bits: int, projections: int, seed: int, norm_correct: bool = True):
+    def __init__(self, head_dim: int, bits: int, projections: int, seed: int, norm_correct: bool = True,
+                 rotation: str = "hadamard"):
         self.d, self.bits, self.m, self.seed = head_dim, bits, projections, seed
+        self.rotation = rotation
         self.cfg = _Cfg()
         if _load().tqo_cfg_init(ctypes.byref(self.cfg), head_dim, bits, projections, int(norm_correct)) != 0:
             raise ValueError("invalid oracle configuration")
+        self.cfg.rotation = ROTATIONS[rotation]
         self.k_row_bytes = _lib.tqo_k_row_bytes(ctypes.byref(self.cfg))
         self.v_row_bytes = _lib.tqo_v_row_bytes(ctypes.byref(self.cfg))
         self._tables = {}
@@ -167,8 +198,11 @@ class Codec:
         return np.array(self.cfg.bv[: self.cfg.LV - 1])
 
     def tables(self, h: int):
+        """(rot, S) of head h: rot = the signs [d] (Hadamard) or Q [d, d] (Haar)."""
         if h not in self._tables:
-            self._tables[h] = head_tables(self.d, self.m, self.seed, h)
+            signs, S = head_tables(self.d, self.m, self.seed, h)
+            rot = haar_matrix(self.d, self.m, self.seed, h) if self.rotation == "haar" else signs
+            self._tables[h] = (rot, S)
         return self._tables[h]
 
     def encode(self, x, h: int, is_key: bool):

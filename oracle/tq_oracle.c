@@ -43,6 +43,14 @@
  *   R7  Zero or non-finite rows encode as: every index = 2^(B-1) (smallest
  *       positive centroid), n_s = 0, gamma = 0, all sign bits 1; non-finite
  *       rows are counted.
+ *   R9  Haar rotation (the [TQ] Modules table's other rotation: "Haar-
+ *       distributed rotation via QR"): Pi = Q, the orthogonal factor of the
+ *       QR factorization of a d x d matrix G of iid N(0,1) entries, with the
+ *       column signs chosen so that R has a positive diagonal, which makes Q
+ *       Haar-distributed (Mezzadri 2007).  G is filled row-major by Box-Muller
+ *       pairs (not rounded) from the head's SplitMix64 stream continued after
+ *       the d sign draws and the draws of S.  The rest of the method is
+ *       unchanged: z = sqrt(d) Q x / ||x||, reconstruction Q^T (...).
  *   R8  Packed layout (the pages give none):
  *       K row: B_K index bit planes (plane p holds bit p of every index;
  *       coordinate j -> byte j/8, bit j%8), then the m-bit sign plane, then
@@ -101,6 +109,73 @@ void tqo_head_tables(int d, int m, uint64_t seed, int h, double *signs, double *
         S[i] = tqo_round_fp16(rad * cos(two_pi * u2));
         if (i + 1 < n) S[i + 1] = tqo_round_fp16(rad * sin(two_pi * u2));
     }
+}
+
+/* Haar rotation of head h (R9): Householder QR of G, Q = H_0 H_1 ... H_(d-1),
+ * then column k of Q multiplied by the sign of R[k][k]. */
+/* The Gaussian matrix G [d][d] of head h (R9): Box-Muller pairs from the
+ * stream continued after the d sign draws and the draws of S. */
+void tqo_haar_gaussian(int d, int m, uint64_t seed, int h, double *G) {
+    uint64_t st = seed + (uint64_t)(int64_t)h;    /* wrapping add */
+    for (int j = 0; j < d; ++j) tqo_splitmix64_next(&st);          /* the rotation signs */
+    int64_t ns = (int64_t)m * d;
+    ns += ns & 1;                                                 /* S is drawn in pairs */
+    for (int64_t i = 0; i < ns; ++i) tqo_splitmix64_next(&st);
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int64_t i = 0; i < (int64_t)d * d; i += 2) {
+        uint64_t ua = tqo_splitmix64_next(&st);
+        uint64_t ub = tqo_splitmix64_next(&st);
+        double u1 = (double)((ua >> 11) + 1) * 0x1.0p-53;
+        double u2 = (double)(ub >> 11) * 0x1.0p-53;
+        double rad = sqrt(-2.0 * log(u1));
+        G[i] = rad * cos(two_pi * u2);
+        if (i + 1 < (int64_t)d * d) G[i + 1] = rad * sin(two_pi * u2);
+    }
+}
+
+void tqo_haar_matrix(int d, int m, uint64_t seed, int h, double *Q) {
+    double *A = (double *)malloc(sizeof(double) * d * d);
+    double *V = (double *)malloc(sizeof(double) * d * d);         /* reflector k in row k, entries k..d-1 */
+    tqo_haar_gaussian(d, m, seed, h, A);
+    for (int k = 0; k < d; ++k) {
+        double nx = 0.0;
+        for (int i = k; i < d; ++i) nx += A[i * d + k] * A[i * d + k];
+        nx = sqrt(nx);
+        double *v = V + (size_t)k * d;
+        for (int i = 0; i < d; ++i) v[i] = 0.0;
+        /* v = x - alpha e1, alpha = -sign(x0) |x| (no cancellation) */
+        double alpha = A[k * d + k] >= 0.0 ? -nx : nx;
+        for (int i = k; i < d; ++i) v[i] = A[i * d + k];
+        v[k] -= alpha;
+        double nv = 0.0;
+        for (int i = k; i < d; ++i) nv += v[i] * v[i];
+        nv = sqrt(nv);
+        if (nv > 0.0)
+            for (int i = k; i < d; ++i) v[i] /= nv;
+        /* A[k:, k:] -= 2 v (v^T A[k:, k:]) */
+        for (int j = k; j < d; ++j) {
+            double dot = 0.0;
+            for (int i = k; i < d; ++i) dot += v[i] * A[i * d + j];
+            for (int i = k; i < d; ++i) A[i * d + j] -= 2.0 * v[i] * dot;
+        }
+    }
+    /* Q = H_0 ... H_(d-1) I */
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) Q[i * d + j] = (i == j) ? 1.0 : 0.0;
+    for (int k = d - 1; k >= 0; --k) {
+        const double *v = V + (size_t)k * d;
+        for (int j = 0; j < d; ++j) {
+            double dot = 0.0;
+            for (int i = k; i < d; ++i) dot += v[i] * Q[i * d + j];
+            for (int i = k; i < d; ++i) Q[i * d + j] -= 2.0 * v[i] * dot;
+        }
+    }
+    /* positive diagonal of R: R[k][k] is A[k][k] after the reflections */
+    for (int k = 0; k < d; ++k)
+        if (A[k * d + k] < 0.0)
+            for (int i = 0; i < d; ++i) Q[i * d + k] = -Q[i * d + k];
+    free(A);
+    free(V);
 }
 
 /* ------------------------------------------------------------ codebook -- */
@@ -199,6 +274,23 @@ void tqo_unrotate(int d, const double *signs, const double *y, double *out) {
     for (int j = 0; j < d; ++j) out[j] *= s * signs[j];
 }
 
+/* out = Q x and out = Q^T y for a dense d x d rotation (R9), row-major Q. */
+void tqo_rotate_dense(int d, const double *Q, const double *x, double *out) {
+    for (int i = 0; i < d; ++i) {
+        double a = 0.0;
+        for (int j = 0; j < d; ++j) a += Q[(size_t)i * d + j] * x[j];
+        out[i] = a;
+    }
+}
+
+void tqo_unrotate_dense(int d, const double *Q, const double *y, double *out) {
+    for (int j = 0; j < d; ++j) {
+        double a = 0.0;
+        for (int i = 0; i < d; ++i) a += Q[(size_t)i * d + j] * y[i];
+        out[j] = a;
+    }
+}
+
 /* --------------------------------------------------------------- config -- */
 
 typedef struct {
@@ -206,7 +298,20 @@ typedef struct {
     int BK, BV, LK, LV;
     int norm_correct;          /* 1: n_s = n/||yhat|| (R5); 0: n_s = n */
     double ck[TQO_MAXL], bk[TQO_MAXL], cv[TQO_MAXL], bv[TQO_MAXL];
+    int rotation;              /* 0: Hadamard (R3), rot = d signs; 1: Haar (R9), rot = Q (d x d) */
 } tqo_cfg;
+
+/* Pi x and Pi^T y for the configured rotation; `rot` is the head's signs
+ * (Hadamard) or its matrix Q (Haar). */
+static void rot_apply(const tqo_cfg *c, const double *rot, const double *x, double *out) {
+    if (c->rotation == 1) tqo_rotate_dense(c->d, rot, x, out);
+    else tqo_rotate(c->d, rot, x, out);
+}
+
+static void rot_apply_t(const tqo_cfg *c, const double *rot, const double *y, double *out) {
+    if (c->rotation == 1) tqo_unrotate_dense(c->d, rot, y, out);
+    else tqo_unrotate(c->d, rot, y, out);
+}
 
 /* bits = total TurboQuant bits b: K uses b-1 PolarQuant bits + 1 QJL bit,
  * V uses b MSE bits ([TQ] Architecture, Key ideas). */
@@ -244,7 +349,8 @@ static double get_f32(const uint8_t *src) {
 }
 
 /* Encode one row.  is_key selects TurboQuant (K) or MSE-only (V).
- * signs[d], S[m*d]: the head's tables.  x[d]: the input, exactly converted.
+ * signs, S[m*d]: the head's tables (signs: the d rotation signs, or Q
+ * (d x d) for the Haar rotation).  x[d]: the input, exactly converted.
  * row: packed output (row bytes of the K or V format), zeroed here.
  * Diagnostics (may be NULL): z_out[d] quantizer inputs (HUGE_VAL for a
  * degenerate row), pn_out[m] normalized projections p_i/gamma (HUGE_VAL if
@@ -288,7 +394,7 @@ int tqo_encode_row(const tqo_cfg *cfg, int is_key, const double *signs, const do
         if (pn_out) for (int i = 0; i < m; ++i) pn_out[i] = HUGE_VAL;
     } else {
         /* a2: rotate the unit vector: y = Pi x / n */
-        tqo_rotate(d, signs, x, y);
+        rot_apply(cfg, signs, x, y);
         for (int j = 0; j < d; ++j) y[j] /= n;
         /* a3: scalar quantization of z = sqrt(d) y against the N(0,1) codebook */
         double sd = sqrt((double)d);
@@ -400,7 +506,7 @@ void tqo_dequant_v(const tqo_cfg *cfg, const double *signs, const uint8_t *row, 
     tqo_unpack_v(cfg, row, idx, &ns);
     double sd = sqrt((double)d);
     for (int j = 0; j < d; ++j) w[j] = ns * cfg->cv[idx[j]] / sd;
-    tqo_unrotate(d, signs, w, out);
+    rot_apply_t(cfg, signs, w, out);
     free(idx); free(w);
 }
 
@@ -421,7 +527,7 @@ void tqo_dequant_k(const tqo_cfg *cfg, const double *signs, const double *S, con
         for (int i = 0; i < m; ++i) acc += S[(int64_t)i * d + j] * (2.0 * bit[i] - 1.0);
         w[j] = ns * cfg->ck[idx[j]] / sd + cq * gamma * acc;
     }
-    tqo_unrotate(d, signs, w, out);
+    rot_apply_t(cfg, signs, w, out);
     free(idx); free(bit); free(w);
 }
 
@@ -438,7 +544,7 @@ void tqo_scores_fused(const tqo_cfg *cfg, const double *signs, const double *S, 
     double *sq = (double *)malloc(sizeof(double) * m);
     int *idx = (int *)malloc(sizeof(int) * d);
     int *bit = (int *)malloc(sizeof(int) * m);
-    tqo_rotate(d, signs, q, qr);
+    rot_apply(cfg, signs, q, qr);
     for (int i = 0; i < m; ++i) {
         double a = 0.0;
         for (int j = 0; j < d; ++j) a += S[(int64_t)i * d + j] * qr[j];

@@ -134,15 +134,83 @@ def test_rotation_orthonormal_and_dense_equivalent():
         assert np.allclose(oracle.unrotate(signs, x), Pi.T @ x, atol=1e-13)
 
 
+# ------------------------------------------------------------ Haar rotation
+
+def test_haar_gaussian_continues_the_head_stream():
+    """G is filled by Box-Muller pairs drawn after the d sign draws and the
+    (even) number of draws of S, from the head's stream (seed + h)."""
+    d, m, seed, h = 16, 12, 77, 3
+    G = oracle.haar_gaussian(d, m, seed, h)
+    skip = d + m * d + (m * d) % 2
+    u = oracle.splitmix64_stream(seed + h, skip + 4)[skip:].astype(object)
+    for k in range(2):
+        u1 = ((int(u[2 * k]) >> 11) + 1) * 2.0 ** -53
+        u2 = (int(u[2 * k + 1]) >> 11) * 2.0 ** -53
+        rad = math.sqrt(-2.0 * math.log(u1))
+        assert abs(G.ravel()[2 * k] - rad * math.cos(2 * math.pi * u2)) < 1e-15
+        assert abs(G.ravel()[2 * k + 1] - rad * math.sin(2 * math.pi * u2)) < 1e-15
+    G128 = oracle.haar_gaussian(128, 128, 42, 0)
+    assert stats.kstest(G128.ravel(), "norm").pvalue > 1e-3
+
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_haar_matrix_is_the_sign_fixed_qr_factor(d):
+    """Q equals LAPACK's QR factor of the same G with the columns' signs set
+    so that R has a positive diagonal; Q is orthogonal and Q^T G is upper
+    triangular with a positive diagonal."""
+    G = oracle.haar_gaussian(d, 32, 5, 1)
+    Q = oracle.haar_matrix(d, 32, 5, 1)
+    Qn, Rn = np.linalg.qr(G)
+    Qn = Qn * np.sign(np.diag(Rn))[None, :]
+    assert np.max(np.abs(Q - Qn)) < 1e-12
+    assert np.max(np.abs(Q.T @ Q - np.eye(d))) < 1e-13
+    R = Q.T @ G
+    assert np.max(np.abs(np.tril(R, -1))) < 1e-12
+    assert np.all(np.diag(R) > 0)
+
+
+def test_haar_matrix_moments():
+    """Haar on O(d): a column of Q is uniform on the sphere, so a squared
+    entry is Beta(1/2, (d-1)/2) with mean 1/d; Q v is uniform for any fixed v."""
+    d = 16
+    sq, proj = [], []
+    v = np.ones(d) / math.sqrt(d)
+    for h in range(300):
+        Q = oracle.haar_matrix(d, 8, 1234, h)
+        sq.append(Q[:, 0] ** 2)
+        proj.append((Q @ v)[3] ** 2)
+    sq = np.concatenate(sq)
+    assert abs(sq.mean() - 1.0 / d) < 4 * math.sqrt(2.0 * (d - 1) / (d * d * (d + 2))) / math.sqrt(len(sq) / d)
+    assert stats.kstest(sq, stats.beta(0.5, (d - 1) / 2.0).cdf).pvalue > 1e-3
+    assert stats.kstest(np.array(proj), stats.beta(0.5, (d - 1) / 2.0).cdf).pvalue > 1e-3
+    # different heads differ
+    assert not np.allclose(oracle.haar_matrix(d, 8, 1234, 0), oracle.haar_matrix(d, 8, 1234, 1))
+
+
+def test_haar_rotation_is_the_dense_product():
+    d = 128
+    Q = oracle.haar_matrix(d, 128, 9, 2)
+    rng = np.random.default_rng(8)
+    for _ in range(5):
+        x = rng.standard_normal(d) * rng.uniform(0.1, 10)
+        assert np.allclose(oracle.rotate(Q, x), Q @ x, atol=1e-12)
+        assert np.allclose(oracle.unrotate(Q, x), Q.T @ x, atol=1e-12)
+        assert abs(np.linalg.norm(oracle.rotate(Q, x)) - np.linalg.norm(x)) < 1e-12 * np.linalg.norm(x)
+
+
 # -------------------------------------------------------------- encode/QJL
 
 def _independent_codes(codec, h, x, is_key):
     """Quantizer indices, n_s, residual and QJL bits recomputed in numpy from
     the method's definition, sharing only the head tables and codebook."""
     d = codec.d
-    signs, S = codec.tables(h)
+    rot, S = codec.tables(h)
     n = np.linalg.norm(x)
-    Pi = _hadamard(d) @ np.diag(signs) / math.sqrt(d)
+    if codec.rotation == "haar":
+        Pi = np.linalg.qr(oracle.haar_gaussian(d, codec.m, codec.seed, h))[0]
+        Pi = Pi * np.sign(np.diag(np.linalg.qr(oracle.haar_gaussian(d, codec.m, codec.seed, h))[1]))[None, :]
+    else:
+        Pi = _hadamard(d) @ np.diag(rot) / math.sqrt(d)
     y = Pi @ x / n
     z = math.sqrt(d) * y
     c, b = (codec.ck, codec.bk) if is_key else (codec.cv, codec.bv)
@@ -154,10 +222,11 @@ def _independent_codes(codec, h, x, is_key):
     return idx, ns, r, p, z
 
 
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
 @pytest.mark.parametrize("bits", [2, 3, 4, 5])
-def test_encode_matches_independent_definition(bits):
+def test_encode_matches_independent_definition(bits, rotation):
     d, m = 64, 32
-    codec = oracle.Codec(d, bits, m, 11)
+    codec = oracle.Codec(d, bits, m, 11, rotation=rotation)
     rng = np.random.default_rng(bits)
     x = rng.standard_normal((6, d)) * rng.uniform(0.2, 5, size=(6, 1))
     for is_key in (True, False):
@@ -219,13 +288,14 @@ def _grid_indices(c, d, rng):
     return rng.permutation(np.repeat(np.arange(len(c)), cnt))
 
 
-def test_special_case_exact_reconstruction():
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+def test_special_case_exact_reconstruction(rotation):
     """x on the normalized codebook grid is reproduced exactly (norm
     correction) with zero residual, so scores are the exact inner products."""
     d, m = 128, 128
     rng = np.random.default_rng(9)
     for bits in (2, 3, 4):
-        codec = oracle.Codec(d, bits, m, 100 + bits)
+        codec = oracle.Codec(d, bits, m, 100 + bits, rotation=rotation)
         signs, S = codec.tables(0)
         for is_key, c in ((True, codec.ck), (False, codec.cv)):
             L = len(c)
@@ -314,10 +384,11 @@ def test_qjl_rotated_frame_is_a_gaussian_projection():
 
 # ------------------------------------------------------------ scores / attn
 
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
 @pytest.mark.parametrize("cfg", [(8, 4, 16, 42), (128, 3, 128, 42), (64, 2, 32, 9), (128, 5, 64, 3)])
-def test_scores_fused_equal_dequantized(cfg):
+def test_scores_fused_equal_dequantized(cfg, rotation):
     d, bits, m, seed = cfg
-    codec = oracle.Codec(d, bits, m, seed)
+    codec = oracle.Codec(d, bits, m, seed, rotation=rotation)
     rng = np.random.default_rng(d + bits)
     K = rng.standard_normal((16, d))
     enc = codec.encode(K, 1, True)
