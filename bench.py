@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha_decode",
                     choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head",
-                             "mha_append"])
+                             "mha_append", "mha_decode_haar"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -74,11 +74,13 @@ WORKLOAD_DESC = {
                    "(K 2+1, V 3), float32",
     "mha_append": "mha_append: batch 8, 32 query heads over 32 kv heads, 4096 cached tokens + 1 appended per "
                   "(sequence, kv head), d128, m128, bits 4 (K 3+1, V 4), float16",
+    "mha_decode_haar": "mha_decode_haar: the mha_decode workload with the Haar-QR rotation (batch 8, 32 heads, "
+                       "4096 tokens, d128, m128, bits 4, float16)",
 }
 
 
 STEP_DESC = {w: "encode all K/V rows + one decode step per query head"
-             for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head")}
+             for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head", "mha_decode_haar")}
 STEP_DESC["bulk_encode"] = "encode all K/V rows of 32 layers"
 STEP_DESC["mha_append"] = "append one token per (sequence, kv head) + one decode step per query head"
 L2_DESC = ("flushed (256 MiB write) before every timed piece, outside its CUDA events; "
@@ -133,8 +135,8 @@ class Workload:
         from kv_cache_vector_10_b200 import workloads as W
         self.name, self.tq, self.torch = name, tq, torch
         seed_shift = 1000 * rank
-        if name in ("mha_decode", "gqa_decode", "single_head", "mha_append"):
-            if name in ("mha_decode", "mha_append"):
+        if name in ("mha_decode", "gqa_decode", "single_head", "mha_append", "mha_decode_haar"):
+            if name in ("mha_decode", "mha_append", "mha_decode_haar"):
                 w = W.mha_decode(device=device, data_seed=2 + seed_shift,
                                  n_tokens=4097 if name == "mha_append" else 4096)
             elif name == "gqa_decode":
@@ -148,7 +150,7 @@ class Workload:
             kr, vr = row_bytes(bits)
             es = w["k"].element_size()
             qb = B * Hq * D * 2 * w["q"].element_size()          # query in + output out
-            self.codec = tq.Codec(D, bits, M, w["seed"])
+            self.codec = tq.Codec(D, bits, M, w["seed"], rotation="haar" if name == "mha_decode_haar" else "hadamard")
             self.B, self.Hq, self.Hkv = B, Hq, Hkv
             if name == "mha_append":
                 T -= 1                                            # history; row T is the step's new row
@@ -367,7 +369,7 @@ def oracle_unit(wl_name, rank_seed=0):
                          [(oc, 0, np.concatenate([ek["rows"], nk["rows"]]), np.concatenate([ev["rows"], nv["rows"]]))])
         dt = time.perf_counter() - t0
         return dt, 1025, "tokens", "1 kv head x 1 query head: append 1 token to 1024 + decode over 1025"
-    if wl_name == "mha_decode":
+    if wl_name in ("mha_decode", "mha_decode_haar"):
         w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024)
         G = 1
     elif wl_name == "gqa_decode":
@@ -376,7 +378,7 @@ def oracle_unit(wl_name, rank_seed=0):
     else:
         w = W.single_head(device="cpu")
         G = 4
-    oc = oracle.Codec(D, w["bits"], M, w["seed"])
+    oc = oracle.Codec(D, w["bits"], M, w["seed"], rotation="haar" if wl_name == "mha_decode_haar" else "hadamard")
     T = w["k"].shape[2]
     t0 = time.perf_counter()
     ek = oc.encode(w["k"][0, 0].double().numpy(), 0, True)

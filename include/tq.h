@@ -69,6 +69,14 @@ typedef enum tq_status {
 typedef enum tq_dtype { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
 typedef enum tq_which { TQ_KEYS = 0, TQ_VALUES = 1, TQ_BOTH = 2 } tq_which;
 
+/* The random rotation Pi (turboquant-plus-rs README, Architecture: "random
+ * rotation (Haar-distributed or fast Walsh-Hadamard)"; Modules: rotation). */
+typedef enum tq_rotation {
+    TQ_ROT_HADAMARD = 0,   /* Pi = H D / sqrt(d): Sylvester Walsh-Hadamard, random signs D */
+    TQ_ROT_HAAR = 1        /* Pi = Q: orthogonal factor of the QR of a d x d Gaussian matrix,
+                              R's diagonal positive (Haar-distributed) */
+} tq_rotation;
+
 typedef struct tq_ctx tq_ctx;
 
 /* A packed cache: two device buffers laid out [batch][n_kv_heads][capacity]
@@ -111,6 +119,20 @@ typedef struct tq_segment {
  * projections a multiple of 32 in [32, 256].  On success *out owns device
  * memory released by tq_destroy.  Synchronous. */
 tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_ctx **out);
+
+/* tq_create with a choice of rotation.  TQ_ROT_HADAMARD is tq_create.
+ * TQ_ROT_HAAR: head h's rotation is Q from the QR factorization of a d x d
+ * matrix of N(0,1) Box-Muller draws that continue head h's SplitMix64
+ * stream (seed + h) after the d sign draws and the m*d (rounded up to even)
+ * draws of S; Q's columns are signed so that R has a positive diagonal.  The
+ * rows are rotated on the tensor cores (sqrt(d) Q as binary16 hi + lo
+ * against the row scaled by a power of two into binary16 range: binary16
+ * and bfloat16 rows exactly, float32 rows as hi + lo), queries and outputs
+ * with fp32 Q.  Packed formats and every other call are unchanged.  In this
+ * mode a row whose largest |x_j| is below 2^-100 is encoded as a zero row.
+ * Returns TQ_ERR_DIM for an unknown rotation. */
+tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
+                       tq_ctx **out);
 
 /* Release a context and its device tables (synchronizes the device). NULL is a no-op. */
 void tq_destroy(tq_ctx *ctx);

@@ -24,6 +24,8 @@ LIB_PATH = os.path.join(_HERE, "lib", "libtq.so")
 TQ_OK = 0
 TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 TQ_KEYS, TQ_VALUES, TQ_BOTH = 0, 1, 2
+TQ_ROT_HADAMARD, TQ_ROT_HAAR = 0, 1
+ROTATIONS = {"hadamard": TQ_ROT_HADAMARD, "haar": TQ_ROT_HAAR}
 TQ_MAX_SEGMENTS = 64
 
 STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_DIM", 4: "TQ_ERR_BITS",
@@ -31,7 +33,7 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
                 9: "TQ_ERR_WORKSPACE", 10: "TQ_ERR_ALIGN", 11: "TQ_ERR_CUDA", 12: "TQ_ERR_DEVICE",
                 13: "TQ_ERR_LIMIT"}
 
-EXPORTED = ["tq_create", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
+EXPORTED = ["tq_create", "tq_create_ex", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
             "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes"]
@@ -64,6 +66,7 @@ def _load():
     V, I, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
     sig = {
         "tq_create": (I, [I, I, I, U64, ctypes.POINTER(V)]),
+        "tq_create_ex": (I, [I, I, I, U64, I, ctypes.POINTER(V)]),
         "tq_destroy": (None, [V]),
         "tq_ensure_heads": (I, [V, I]),
         "tq_row_bytes": (I64, [V, I]),
@@ -114,6 +117,13 @@ def _dtype_code(dt) -> int:
 def tq_create(head_dim: int, bits: int, projections: int, seed: int) -> int:
     out = ctypes.c_void_p()
     _check(_lib.tq_create(head_dim, bits, projections, seed & 0xFFFFFFFFFFFFFFFF, ctypes.byref(out)), "tq_create")
+    return out.value
+
+
+def tq_create_ex(head_dim: int, bits: int, projections: int, seed: int, rotation: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.tq_create_ex(head_dim, bits, projections, seed & 0xFFFFFFFFFFFFFFFF, rotation, ctypes.byref(out)),
+           "tq_create_ex")
     return out.value
 
 
@@ -226,11 +236,13 @@ def tq_reset_status(ctx: int, stream=None):
 # -------------------------------------------------------------- conveniences
 
 class Codec:
-    """A codec context: KvCacheConfig {head_dim, bits, projections, seed}."""
+    """A codec context: KvCacheConfig {head_dim, bits, projections, seed}, and
+    the rotation ("hadamard": FWHT with random signs; "haar": QR rotation)."""
 
-    def __init__(self, head_dim: int, bits: int, projections: int, seed: int):
+    def __init__(self, head_dim: int, bits: int, projections: int, seed: int, rotation: str = "hadamard"):
         self.head_dim, self.bits, self.projections, self.seed = head_dim, bits, projections, seed
-        self.ctx = tq_create(head_dim, bits, projections, seed)
+        self.rotation = rotation
+        self.ctx = tq_create_ex(head_dim, bits, projections, seed, ROTATIONS[rotation])
         self.k_row_bytes = tq_row_bytes(self.ctx, TQ_KEYS)
         self.v_row_bytes = tq_row_bytes(self.ctx, TQ_VALUES)
 

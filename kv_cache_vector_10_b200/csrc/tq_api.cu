@@ -2,6 +2,7 @@
 // table upload and kernel dispatch.  No computation on the data path
 // happens on the host; every step runs in the kernels of tq_encode.cu,
 // tq_decode.cu and tq_aux.cu.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <vector>
@@ -11,6 +12,7 @@
 extern "C" void tq_host_head_tables(int d, int m, uint64_t seed, int h, uint32_t *sign_words,
                                     uint16_t *S_bits);
 extern "C" int tq_host_codebook(int B, float *c, float *beta);
+extern "C" void tq_host_haar(int d, int m, uint64_t seed, int h, double *Q);
 
 tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch, int H,
                            int64_t T, int64_t sb, int64_t sh, int64_t st, const tq_codes *codes,
@@ -92,7 +94,16 @@ const char *tq_status_string(tq_status s) {
 const char *tq_last_cuda_error(void) { return g_cuda_msg; }
 
 tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_ctx **out) {
+    return tq_create_ex(head_dim, bits, projections, seed, TQ_ROT_HADAMARD, out);
+}
+
+tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
+                       tq_ctx **out) {
     if (!out) return TQ_ERR_NULL;
+    if (rotation != TQ_ROT_HADAMARD && rotation != TQ_ROT_HAAR) {
+        *out = nullptr;
+        return TQ_ERR_DIM;
+    }
     *out = nullptr;
     if (head_dim == 0) return TQ_ERR_ZERO_DIM;
     if (head_dim != 64 && head_dim != 128) return TQ_ERR_DIM;
@@ -113,6 +124,7 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
     c->BV = bits;
     c->seed = seed;
     c->device = dev;
+    c->rotation = (int)rotation;
     c->LK = tq_host_codebook(c->BK, c->ck, c->bk);
     c->LV = tq_host_codebook(c->BV, c->cv, c->bv);
     TqBook book;
@@ -140,6 +152,8 @@ void tq_destroy(tq_ctx *ctx) {
     cudaFree(ctx->d_S);
     cudaFree(ctx->d_status);
     cudaFree(ctx->d_book);
+    cudaFree(ctx->d_Q32);
+    cudaFree(ctx->d_Qh);
     delete ctx;
 }
 
@@ -179,17 +193,64 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
             }
         }
     }
+    float *nQ32 = nullptr;
+    __half *nQh = nullptr;
+    CUtensorMap qmap;
+    std::memset(&qmap, 0, sizeof(qmap));
+    if (st == TQ_OK && ctx->rotation == TQ_ROT_HAAR) {
+        const size_t dd = (size_t)d * d;
+        std::vector<double> Q(dd);
+        std::vector<float> q32((size_t)n_heads * dd);
+        std::vector<__half> qh((size_t)n_heads * 2 * dd);
+        const double sd = std::sqrt((double)d);
+        for (int h = 0; h < n_heads; ++h) {
+            tq_host_haar(d, m, ctx->seed, h, Q.data());
+            for (size_t i = 0; i < dd; ++i) {
+                q32[(size_t)h * dd + i] = (float)Q[i];
+                const double v = sd * Q[i];
+                const __half hi = __double2half(v);
+                qh[(size_t)h * 2 * dd + i] = hi;
+                qh[(size_t)h * 2 * dd + dd + i] = __double2half(v - (double)__half2float(hi));
+            }
+        }
+        st = tq_check_cuda(cudaMalloc(&nQ32, q32.size() * 4));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMalloc(&nQh, qh.size() * 2));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nQ32, q32.data(), q32.size() * 4, cudaMemcpyHostToDevice));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nQh, qh.data(), qh.size() * 2, cudaMemcpyHostToDevice));
+        if (st == TQ_OK) {
+            PFN_encodeTiled enc = get_encode_tiled();
+            cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n_heads * 2 * d};
+            cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+            cuuint32_t box[2] = {64, (cuuint32_t)d};
+            cuuint32_t es[2] = {1, 1};
+            CUresult r = enc ? enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, nQh, dims, strides, box, es,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+                             : CUDA_ERROR_NOT_FOUND;
+            if (r != CUDA_SUCCESS) {
+                snprintf(g_cuda_msg, sizeof(g_cuda_msg), "cuTensorMapEncodeTiled failed: %d", (int)r);
+                st = TQ_ERR_CUDA;
+            }
+        }
+    }
     if (st != TQ_OK) {
         cudaFree(nsig);
         cudaFree(nS);
+        cudaFree(nQ32);
+        cudaFree(nQh);
         return st;
     }
     cudaDeviceSynchronize();   // no kernel may still read the old tables
     cudaFree(ctx->d_signs);
     cudaFree(ctx->d_S);
+    cudaFree(ctx->d_Q32);
+    cudaFree(ctx->d_Qh);
     ctx->d_signs = nsig;
     ctx->d_S = nS;
     ctx->tmap_S = map;
+    ctx->d_Q32 = nQ32;
+    ctx->d_Qh = nQh;
+    ctx->tmap_Q = qmap;
     ctx->heads_built = n_heads;
     return TQ_OK;
 }

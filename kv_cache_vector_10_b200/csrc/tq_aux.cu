@@ -26,9 +26,24 @@ constexpr int AUX_THREADS = 128;
 // loads of its row of S in flight at once.
 template <int D>
 __device__ void prep_query(const float *sq_in, const uint32_t *signs, const __half *S, int M, float *s_qr,
-                           float *s_sq) {
+                           float *s_sq, const float *Q) {
     const int tid = threadIdx.x;
-    if (tid < 32) {
+    if (Q) {
+        // Haar rotation: q_rot = Q q, one output per thread
+        for (int i = tid; i < D; i += blockDim.x) {
+            const float4 *row = reinterpret_cast<const float4 *>(Q + (int64_t)i * D);
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < D / 4; ++c) {
+                const float4 w = __ldg(row + c);
+                a0 = fmaf(w.x, sq_in[4 * c], a0);
+                a1 = fmaf(w.y, sq_in[4 * c + 1], a1);
+                a0 = fmaf(w.z, sq_in[4 * c + 2], a0);
+                a1 = fmaf(w.w, sq_in[4 * c + 3], a1);
+            }
+            s_qr[i] = a0 + a1;
+        }
+    } else if (tid < 32) {
         constexpr int V = D / 32;
         const int lane = tid;
         float x[V];
@@ -96,6 +111,7 @@ struct ScoresParams {
     float *scores;
     const uint32_t *signs;
     const __half *S;
+    const float *Q;            // Haar rotation, or nullptr
     int64_t capacity, T;
     int Hq, Hkv, M, krow, bk;
     float ck[16];
@@ -108,7 +124,7 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_con
     const int j = blockIdx.y, b = blockIdx.z;
     const int h = j / (p.Hq / p.Hkv);
     prep_query<D>(p.q + ((int64_t)b * p.Hq + j) * D, p.signs + (int64_t)h * (D / 32), p.S + (int64_t)h * p.M * D,
-                  p.M, s_qr, s_sq);
+                  p.M, s_qr, s_sq, p.Q ? p.Q + (int64_t)h * D * D : nullptr);
     const int64_t t = (int64_t)blockIdx.x * AUX_THREADS + threadIdx.x;
     if (t >= p.T) return;
     const uint8_t *row = p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) * p.krow;
@@ -136,11 +152,24 @@ struct DequantParams {
     float *vh;
     const uint32_t *signs;
     const __half *S;
+    const float *Q;            // Haar rotation, or nullptr
     int64_t capacity, T;
     int H, M, krow, vrow, bk, bv;
     float ck[16];
     float cv[32];
 };
+
+// Haar rotation: dst = Q^T w.
+template <int D>
+__device__ __forceinline__ void unrotate_dense_store(const float (&w)[D], const float *Q, float *dst) {
+#pragma unroll 1
+    for (int j = 0; j < D; ++j) {
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) a = fmaf(__ldg(Q + i * D + j), w[i], a);
+        dst[j] = a;
+    }
+}
 
 template <int D>
 __device__ __forceinline__ void unrotate_store(float (&w)[D], const uint32_t *sg, float *dst) {
@@ -196,7 +225,8 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_dequant_kernel(const __grid_co
             if ((bit % 32) + p.bv > 32) v |= w[bit / 32 + 1] << (32 - bit % 32);
             x[j] = ns * p.cv[v & ((1u << p.bv) - 1)] * isd;
         }
-        unrotate_store<D>(x, sg, p.vh + outi);
+        if (p.Q) unrotate_dense_store<D>(x, p.Q + (int64_t)h * D * D, p.vh + outi);
+        else unrotate_store<D>(x, sg, p.vh + outi);
     }
     if (p.kh) {
         const uint32_t *w = reinterpret_cast<const uint32_t *>(p.kc + rowi * p.krow);
@@ -221,7 +251,8 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_dequant_kernel(const __grid_co
                 x[2 * j + 1] = fmaf(s, f.y, x[2 * j + 1]);
             }
         }
-        unrotate_store<D>(x, sg, p.kh + outi);
+        if (p.Q) unrotate_dense_store<D>(x, p.Q + (int64_t)h * D * D, p.kh + outi);
+        else unrotate_store<D>(x, sg, p.kh + outi);
     }
 }
 
@@ -276,21 +307,35 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
     const int HB = 1 << (B - 1);
     const float *mag = key ? book.kmag : book.vmag;
     const float *pb = key ? book.kpb : book.vpb;
-    if (tid < D) {
-        const float x = load_dt(src, src_off + tid, dt);
-        s_u[tid] = ((g.signs[(int64_t)h * (D / 32) + tid / 32] >> (tid % 32)) & 1) ? -x : x;
-    }
-    __syncthreads();
-    for (int len = 1; len < D; len <<= 1) {
-        for (int i = tid; i < D / 2; i += blockDim.x) {
-            const int j = (i / len) * 2 * len + (i % len);
-            const float a = s_u[j], b = s_u[j + len];
-            s_u[j] = a + b;
-            s_u[j + len] = a - b;
+    float u = 0.f;
+    if (g.Q) {
+        // Haar rotation: u = sqrt(d) Q x
+        if (tid < D) s_e[tid] = load_dt(src, src_off + tid, dt);
+        __syncthreads();
+        if (tid < D) {
+            const float *row = g.Q + ((int64_t)h * D + tid) * D;
+            float a = 0.f;
+            for (int j = 0; j < D; ++j) a = fmaf(__ldg(row + j), s_e[j], a);
+            u = a * sqrtf((float)D);
         }
         __syncthreads();
+    } else {
+        if (tid < D) {
+            const float x = load_dt(src, src_off + tid, dt);
+            s_u[tid] = ((g.signs[(int64_t)h * (D / 32) + tid / 32] >> (tid % 32)) & 1) ? -x : x;
+        }
+        __syncthreads();
+        for (int len = 1; len < D; len <<= 1) {
+            for (int i = tid; i < D / 2; i += blockDim.x) {
+                const int j = (i / len) * 2 * len + (i % len);
+                const float a = s_u[j], b = s_u[j + len];
+                s_u[j] = a + b;
+                s_u[j + len] = a - b;
+            }
+            __syncthreads();
+        }
+        u = tid < D ? s_u[tid] : 0.f;
     }
-    const float u = tid < D ? s_u[tid] : 0.f;
     const float n2 = block_sum(u * u, s_red);
     const bool nonfinite = !(n2 <= 3.0e38f);
     const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
@@ -398,7 +443,8 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_cons
     const int h = j / P.G;
     for (int i = threadIdx.x; i < D; i += blockDim.x) s_in[i] = load_as_float<Tq>(q, ((int64_t)seq * P.Hq + j) * D + i);
     __syncthreads();
-    prep_query<D>(s_in, g.signs + (int64_t)h * (D / 32), g.S + (int64_t)h * g.m * D, g.m, s_qr, s_sq);
+    prep_query<D>(s_in, g.signs + (int64_t)h * (D / 32), g.S + (int64_t)h * g.m * D, g.m, s_qr, s_sq,
+                  g.Q ? g.Q + (int64_t)h * D * D : nullptr);
     float *dst = P.qprep + g.qprep_base + ((int64_t)seq_local * P.Hq + j) * (D + g.m);
     for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = s_qr[i];
     for (int i = threadIdx.x; i < g.m; i += blockDim.x) dst[D + i] = s_sq[i];
@@ -462,6 +508,7 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
     p.scores = scores;
     p.signs = ctx->d_signs;
     p.S = ctx->d_S;
+    p.Q = ctx->rotation == TQ_ROT_HAAR ? ctx->d_Q32 : nullptr;
     p.capacity = codes->capacity;
     p.T = T;
     p.Hq = Hq;
@@ -485,6 +532,7 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
     p.vh = v_hat;
     p.signs = ctx->d_signs;
     p.S = ctx->d_S;
+    p.Q = ctx->rotation == TQ_ROT_HAAR ? ctx->d_Q32 : nullptr;
     p.capacity = codes->capacity;
     p.T = T;
     p.H = codes->n_kv_heads;

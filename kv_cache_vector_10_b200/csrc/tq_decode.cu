@@ -415,6 +415,28 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         }
     }
     __syncthreads();
+    if (g.Q) {
+        // Haar rotation: out = Q^T acc / sqrt(d)
+        const float *Qh = g.Q + (int64_t)h * D * D;
+        const float isd = rsqrtf((float)D);
+        for (int i = tid; i < QC * D; i += blockDim.x) {
+            const int qq = i / D, j = i % D;
+            const int qi = qchunk * QC + qq;
+            if (qi >= nq) continue;
+            const int seq_local = qi / P.G, jh = h * P.G + qi % P.G;
+            float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
+            float v = 0.f;
+            for (int r = 0; r < D; ++r) v = fmaf(Qh[r * D + j], acc[qq * D + r], v);
+            dst[4 + j] = v * isd;
+            if (j == 0) {
+                dst[0] = ml[2 * qq];
+                dst[1] = ml[2 * qq + 1];
+                dst[2] = 0.f;
+                dst[3] = 0.f;
+            }
+        }
+        return;
+    }
     // Pi^T with the 1/sqrt(d) of the value scale: out = D H acc / d
     for (int len = 1; len < D; len <<= 1) {
         for (int i = tid; i < QC * D / 2; i += blockDim.x) {
@@ -611,6 +633,7 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         d.S = c->d_S;
         d.status = c->d_status;
         d.book = c->d_book;
+        d.Q = c->rotation == TQ_ROT_HAAR ? c->d_Q32 : nullptr;
         d.append = app && app->flags[s] ? 1 : 0;
         if (d.append) P.n_append_blocks += Hkv;
         d.capacity = sg.codes.capacity;

@@ -17,6 +17,7 @@ struct SegDesc {
     const __half *S;           // [H_kv][m][d]
     unsigned long long *status;  // the segment context's status word
     const TqBook *book;        // the segment context's codebooks (device)
+    const float *Q;            // Haar rotation [H_kv][d][d] fp32, or nullptr (Walsh-Hadamard)
     int64_t capacity;
     int64_t T;
     int64_t part_base;         // first partial slot of this segment

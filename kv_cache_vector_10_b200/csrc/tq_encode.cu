@@ -430,15 +430,177 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
     return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : cols <= 256 ? 256u : 512u;
 }
 
+// ------------------------------------------------- dense (Haar) rotation
+// The Haar rotation u = sqrt(d) Q x runs on the tensor cores: each thread
+// writes its row, scaled by 2^e so that max_j |x_j| lies in [2^14, 2^15), as
+// binary16 into the 128-byte-swizzled K-major operand layout (16-byte unit kk
+// of row r at (kk / 8) * ATOM + r * 128 + ((kk % 8) ^ (r % 8)) * 16); the
+// scaling is a power of two, so binary16 and bfloat16 rows are exact (up to
+// binary16 subnormals below 2^-14 of the row maximum) and float32 rows are
+// split into hi + lo.  The MMA against sqrt(d) Q (binary16 hi + lo) leaves
+// 2^e u in TMEM; quantization is scale-free, and the stored norms are
+// multiplied back by 2^-e.
+struct DenseRow {
+    float n2;          // d |2^e x|^2 = |2^e u|^2
+    float inv_scale;   // 2^-e
+    bool nonfinite;    // some x_j is Inf or NaN
+    bool zero;         // zero operand: non-finite, all zero, or max |x_j| < 2^-100 (or past the end)
+};
+
+template <typename Tin>
+__device__ __forceinline__ float2 word_to_float2(uint32_t w) {
+    if constexpr (std::is_same<Tin, __half>::value)
+        return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    else
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+template <int D, typename Tin>
+__device__ __forceinline__ DenseRow stage_dense_row(const RowWords<D> &raw, const Tin *rowp, bool valid, int r,
+                                                    uint8_t *xHi, uint8_t *xLo) {
+    constexpr int ATOM = ENC_ROWS * 128;
+    constexpr bool H16 = sizeof(Tin) == 2;
+    DenseRow out;
+    float mx = 0.f;
+    bool bad = false;
+    if constexpr (H16) {
+        uint32_t mb = 0u;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            const uint4 q = raw.w[i];
+            mb = __vmaxu2(mb, q.x & 0x7FFF7FFFu);
+            mb = __vmaxu2(mb, q.y & 0x7FFF7FFFu);
+            mb = __vmaxu2(mb, q.z & 0x7FFF7FFFu);
+            mb = __vmaxu2(mb, q.w & 0x7FFF7FFFu);
+        }
+        const uint32_t m16 = max(mb & 0xFFFFu, mb >> 16);
+        if constexpr (std::is_same<Tin, __half>::value) {
+            bad = m16 >= 0x7C00u;
+            mx = __half2float(__ushort_as_half((unsigned short)m16));
+        } else {
+            bad = m16 >= 0x7F80u;
+            mx = __uint_as_float(m16 << 16);
+        }
+    } else if (valid) {
+        uint32_t mb = 0u;
+        const uint4 *p4 = reinterpret_cast<const uint4 *>(rowp);
+#pragma unroll 4
+        for (int i = 0; i < D / 4; ++i) {
+            const uint4 q = __ldg(p4 + i);
+            mb = max(mb, max(max(q.x & 0x7FFFFFFFu, q.y & 0x7FFFFFFFu), max(q.z & 0x7FFFFFFFu, q.w & 0x7FFFFFFFu)));
+        }
+        bad = mb >= 0x7F800000u;
+        mx = __uint_as_float(mb);
+    }
+    if (!valid) {
+        bad = false;
+        mx = 0.f;
+    }
+    out.nonfinite = bad;
+    out.zero = bad || !(mx >= 0x1p-100f);
+    const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
+    const int e = out.zero ? 0 : 14 - ex;               // in [-113, 114]
+    const float sc = __uint_as_float((uint32_t)(e + 127) << 23);
+    out.inv_scale = __uint_as_float((uint32_t)(127 - e) << 23);
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int kk = 0; kk < D / 8; ++kk) {
+        float v[8];
+        if constexpr (H16) {
+            const uint4 q = raw.w[kk];
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                const float2 f = word_to_float2<Tin>(w4[e2]);
+                v[2 * e2] = f.x;
+                v[2 * e2 + 1] = f.y;
+            }
+        } else {
+            if (valid) {
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(rowp) + 2 * kk);
+                const float4 b2 = __ldg(reinterpret_cast<const float4 *>(rowp) + 2 * kk + 1);
+                v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+                v[4] = b2.x; v[5] = b2.y; v[6] = b2.z; v[7] = b2.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = 0.f;
+            }
+        }
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 a = out.zero ? make_float2(0.f, 0.f) : mul2(make_float2(v[2 * e2], v[2 * e2 + 1]), dup2(sc));
+            acc = fma2(a, a, acc);
+            const __half2 hh = __floats2half2_rn(a.x, a.y);
+            hw[e2] = *reinterpret_cast<const uint32_t *>(&hh);
+            if constexpr (!H16) {
+                const float2 l = sub2(a, __half22float2(hh));
+                const __half2 ll = __floats2half2_rn(l.x, l.y);
+                lw[e2] = *reinterpret_cast<const uint32_t *>(&ll);
+            }
+        }
+        const int off = (kk / 8) * ATOM + r * 128 + (((kk % 8) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4 *>(xHi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        if constexpr (!H16) *reinterpret_cast<uint4 *>(xLo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    out.n2 = (acc.x + acc.y) * (float)D;
+    return out;
+}
+
+// Issued by one thread: 2^e u = X (sqrt(d) Q)^T into TMEM columns [0, d):
+// passes (X hi, Q hi), (X hi, Q lo) and, for float32 rows, (X lo, Q hi).
+template <int D, typename Tin>
+__device__ __forceinline__ void issue_dense_rotation(uint32_t tmem_base, const uint8_t *xHi, const uint8_t *xLo,
+                                                     const uint8_t *sQ, uint64_t *bar) {
+    constexpr int ATOM = ENC_ROWS * 128;
+    constexpr int PASSES = sizeof(Tin) == 2 ? 2 : 3;
+    const uint32_t idesc = tqdev::idesc_f16_f32(D);
+#pragma unroll
+    for (int pass = 0; pass < PASSES; ++pass) {
+        const uint32_t abase = tqdev::smem_u32(pass == 2 ? xLo : xHi);
+        const uint32_t bbase = tqdev::smem_u32(sQ + (pass == 1 ? (D / 64) * D * 128 : 0));
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t a_addr = abase + (ks / 4) * ATOM + (ks % 4) * 32;
+            const uint32_t b_addr = bbase + (ks / 4) * (D * 128) + (ks % 4) * 32;
+            tqdev::mma_f16_ss(tmem_base, tqdev::smem_desc_sw128(a_addr), tqdev::smem_desc_sw128(b_addr), idesc,
+                              (pass | ks) != 0);
+        }
+    }
+    tqdev::mma_commit(bar);
+}
+
+// TMA of head h's two binary16 pieces of sqrt(d) Q into sQ [2][d/64][d][128 B].
+template <int D>
+__device__ __forceinline__ void load_q_tiles(uint8_t *sQ, const CUtensorMap *tmapQ, int head, uint64_t *bar) {
+    tqdev::mbar_expect_tx(bar, (uint32_t)(2 * D * D * 2));
+#pragma unroll
+    for (int piece = 0; piece < 2; ++piece)
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+            tqdev::tma_load_2d(sQ + (piece * (D / 64) + a) * D * 128, tmapQ, a * 64, (head * 2 + piece) * D, bar);
+}
+
 // ------------------------------------------------------------------ values
-template <int D, int BV, typename Tin>
-__global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_constant__ EncodeParams p) {
+// ROT: 0 = Walsh-Hadamard rotation in registers and TMEM; 1 = dense (Haar)
+// rotation on the tensor cores.
+template <int D, int BV, typename Tin, int ROT>
+__global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_constant__ EncodeParams p,
+                                                               const __grid_constant__ CUtensorMap tmapQ) {
     constexpr int HV = (1 << BV) / 2;
     constexpr int NC = D / 32;
     constexpr uint32_t FMASK = (1u << BV) - 1u;
+    constexpr int ATOM = ENC_ROWS * 128;
     __shared__ __align__(16) uint32_t s_mask[Chunk<Tin>::MASK_WORDS * NC];
     __shared__ float s_mag2[16];
     __shared__ uint32_t s_tmem;
+    // dense rotation only: [sQ: 2 x d/64 x d x 128 B][X: pieces x d/64 x ATOM], 1024-aligned
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t s_bars[2];    // [0] Q loaded, [1] rotation MMA done
+    __shared__ int s_abort;
+    uint8_t *sQ = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xHi = sQ + 2 * (D / 64) * D * 128;
+    uint8_t *xLo = xHi + (D / 64) * ATOM;
     const int tid = threadIdx.x, warp = tid / 32;
     const int64_t blk = blockIdx.x;
     const int64_t bh = blk / p.blocks_per_bh;
@@ -447,12 +609,23 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
     const int64_t tb0 = (blk % p.blocks_per_bh) * (int64_t)ENC_TILES * ENC_ROWS;
     build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
     if (tid < 16) s_mag2[tid] = tid < HV ? p.mag[tid] * p.mag[tid] : 0.f;
+    if constexpr (ROT == 1) {
+        if (tid == 0) {
+            tqdev::mbar_init(&s_bars[0], 1);
+            tqdev::mbar_init(&s_bars[1], 1);
+            s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
+            tqdev::fence_barrier_init();
+        }
+    }
     if (warp == 0) tqdev::tmem_alloc(&s_tmem, tmem_cols_for(D));
     tqdev::tc_fence_before();
     __syncthreads();
     tqdev::tc_fence_after();
     const uint32_t tlane = s_tmem + ((uint32_t)(warp * 32) << 16);
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
+    if constexpr (ROT == 1) {
+        if (tid == 0 && !s_abort) load_q_tiles<D>(sQ, &tmapQ, head, &s_bars[0]);
+    }
     // 16-bit inputs: each tile's rows are loaded into registers during the
     // previous tile's quantization
     constexpr bool PF = sizeof(Tin) == 2;
@@ -466,16 +639,48 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
         if (t0 >= p.T) break;
         const int64_t t = t0 + tid;
         const bool valid = t < p.T;
-        float n2;
-        if constexpr (PF) {
-            n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
-            if (tile + 1 < ENC_TILES && t0 + ENC_ROWS < p.T)
-                load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+        float n2, inv_scale = 1.f;
+        bool nonfinite, degenerate;
+        if constexpr (ROT == 1) {
+            const DenseRow dr = stage_dense_row<D, Tin>(raw, src + t * p.st, valid, tid, xHi, xLo);
+            if constexpr (PF) {
+                if (tile + 1 < ENC_TILES && t0 + ENC_ROWS < p.T)
+                    load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+            }
+            tqdev::fence_proxy_async_smem();
+            tqdev::tc_fence_before();
+            __syncthreads();
+            if (tid == 0 && !s_abort) {
+                if (tile > 0 || tqdev::mbar_wait_bounded(&s_bars[0], 0)) {
+                    tqdev::tc_fence_after();
+                    issue_dense_rotation<D, Tin>(s_tmem, xHi, xLo, sQ, &s_bars[1]);
+                } else {
+                    atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+                    s_abort = 1;
+                    tqdev::mbar_arrive(&s_bars[1]);   // release the wait below
+                }
+            }
+            const bool done = s_abort ? true : tqdev::mbar_wait_bounded(&s_bars[1], (uint32_t)(tile & 1));
+            if (__syncthreads_or(!done || s_abort)) {
+                if (tid == 0 && !done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+                break;
+            }
+            tqdev::tc_fence_after();
+            n2 = dr.n2;
+            inv_scale = dr.inv_scale;
+            nonfinite = dr.nonfinite;
+            degenerate = dr.zero;
         } else {
-            n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+            if constexpr (PF) {
+                n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
+                if (tile + 1 < ENC_TILES && t0 + ENC_ROWS < p.T)
+                    load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+            } else {
+                n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, valid, s_mask, tlane);
+            }
+            nonfinite = !(n2 <= 3.0e38f);
+            degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         }
-        const bool nonfinite = !(n2 <= 3.0e38f);
-        const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
         const float n = sqrtf(n2 * (1.f / D));
@@ -561,7 +766,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
                 }
             }
         }
-        if (valid) dst[BV * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2));
+        if (valid) dst[BV * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2) * inv_scale);
     }
     tqdev::tc_fence_before();
     __syncthreads();
@@ -572,9 +777,10 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
 }
 
 // -------------------------------------------------------------------- keys
-template <int D, int BK, typename Tin>
+template <int D, int BK, typename Tin, int ROT>
 __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_constant__ EncodeParams p,
-                                                               const __grid_constant__ CUtensorMap tmapS) {
+                                                               const __grid_constant__ CUtensorMap tmapS,
+                                                               const __grid_constant__ CUtensorMap tmapQ) {
     constexpr int HK = (1 << BK) / 2;
     constexpr int NC = D / 32;                 // chunks = 32-bit words per bit plane
     constexpr int ATOM = ENC_ROWS * 128;       // bytes of one 128-row x 128-byte swizzle column
@@ -585,12 +791,14 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // <= 512 B
     float *s_mag = reinterpret_cast<float *>(smem + 512);                   // [16]
     float *s_mag2 = s_mag + 16;                                             // [16]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);              // [0] S loaded, [1] MMA done
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 2);
+    // [0] S loaded, [1] QJL MMA done, [2] Q loaded, [3] rotation MMA done (dense rotation)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 4);
     int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
     const int M = p.M;
     uint8_t *sS = smem + 1024;                                              // [D/64][M rows][128 B]
     uint8_t *sA = sS + (D / 64) * M * 128;                                   // [pass][D/64][128 rows][128 B]
+    uint8_t *sQ = sA + 2 * A_BYTES;                                          // dense rotation: [2][D/64][D][128 B]
     const int tid = threadIdx.x, warp = tid / 32;
     const int64_t blk = blockIdx.x;
     const int64_t bh = blk / p.blocks_per_bh;
@@ -607,8 +815,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         s_mag2[tid] = mg * mg;
     }
     if (tid == 0) {
-        tqdev::mbar_init(&bars[0], 1);
-        tqdev::mbar_init(&bars[1], 1);
+        for (int i = 0; i < 4; ++i) tqdev::mbar_init(&bars[i], 1);
         *s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
         tqdev::fence_barrier_init();
     }
@@ -622,6 +829,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         tqdev::mbar_expect_tx(&bars[0], (uint32_t)(M * D * 2));
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) tqdev::tma_load_2d(sS + a * M * 128, &tmapS, a * 64, head * M, &bars[0]);
+        if constexpr (ROT == 1) load_q_tiles<D>(sQ, &tmapQ, head, &bars[2]);
     }
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
@@ -635,11 +843,10 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     float n2 = 0.f;
     if (ntiles > 0 && !*s_abort) {
         const int64_t t = tb0 + tid;
-        if constexpr (PF) {
-            load_row_words<D, Tin>(src + t * p.st, t < p.T, raw);
-            n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
-        } else {
-            n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, t < p.T, s_mask, tlane);
+        if constexpr (PF) load_row_words<D, Tin>(src + t * p.st, t < p.T, raw);
+        if constexpr (ROT == 0) {
+            if constexpr (PF) n2 = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
+            else n2 = rotate_row_to_tmem<D, Tin>(src + t * p.st, t < p.T, s_mask, tlane);
         }
     }
 #pragma unroll 1
@@ -647,12 +854,44 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         if (*s_abort) break;   // uniform: set before the barrier that ends the previous tile
         const int64_t t = tb0 + tile * ENC_ROWS + tid;
         const bool valid = t < p.T;
-        if constexpr (PF) {
+        float inv_scale = 1.f;
+        bool dense_nonfinite = false, dense_zero = false;
+        if constexpr (ROT == 1) {
+            // A, B: the dense rotation of this tile on the tensor cores
+            const DenseRow dr = stage_dense_row<D, Tin>(raw, src + t * p.st, valid, tid, aHi, aLo);
+            tqdev::fence_proxy_async_smem();
+            tqdev::tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                if (tile > 0 || tqdev::mbar_wait_bounded(&bars[2], 0)) {
+                    tqdev::tc_fence_after();
+                    issue_dense_rotation<D, Tin>(tmem_base, aHi, aLo, sQ, &bars[3]);
+                } else {
+                    atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+                    *s_abort = 1;
+                    tqdev::mbar_arrive(&bars[3]);   // release the wait below
+                }
+            }
+            if constexpr (PF) {
+                if (tile + 1 < ntiles) load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
+            }
+            const bool rdone = tqdev::mbar_wait_bounded(&bars[3], (uint32_t)(tile & 1));
+            if (__syncthreads_or(!rdone || *s_abort)) {
+                if (tid == 0 && !rdone) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+                if (tid == 0) *s_abort = 1;
+                break;
+            }
+            tqdev::tc_fence_after();
+            n2 = dr.n2;
+            inv_scale = dr.inv_scale;
+            dense_nonfinite = dr.nonfinite;
+            dense_zero = dr.zero;
+        } else if constexpr (PF) {
             if (tile + 1 < ntiles) load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
         }
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
-        const bool nonfinite = !(n2 <= 3.0e38f);
-        const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
+        const bool nonfinite = ROT == 1 ? dense_nonfinite : !(n2 <= 3.0e38f);
+        const bool degenerate = ROT == 1 ? dense_zero : (nonfinite || !(n2 >= 1.17549435e-38f));
         if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
         const float n = sqrtf(n2 * (1.f / D));
         float rb[8];
@@ -759,8 +998,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         const float e2 = e2p.x + e2p.y;
         if (valid) {
             const int tail = BK * NC + M / 32;
-            dst[tail] = __float_as_uint(ns);
-            dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)));
+            dst[tail] = __float_as_uint(ns * inv_scale);
+            dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)) * inv_scale);
         }
         // E: the QJL projection on the tensor cores (TMEM columns [d, d + m))
         tqdev::fence_proxy_async_smem();
@@ -792,7 +1031,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         }
         // A, B of the next tile while the MMA runs (they touch only U)
         float n2_next = 0.f;
-        if (tile + 1 < ntiles) {
+        if (ROT == 0 && tile + 1 < ntiles) {
             const int64_t tn = t + ENC_ROWS;
             if constexpr (PF) n2_next = rotate_words_to_tmem<D, Tin>(raw, s_mask, tlane);
             else n2_next = rotate_row_to_tmem<D, Tin>(src + tn * p.st, tn < p.T, s_mask, tlane);
@@ -831,11 +1070,13 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     }
 }
 
-template <int D, typename Tin>
-cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, int64_t grid, cudaStream_t s) {
+template <int D, typename Tin, int ROT>
+cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &mapS, const CUtensorMap &mapQ, int64_t grid,
+                     cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     auto go = [&](auto kern) {
         size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+        if (ROT == 1) smem += 2 * (size_t)(D / 64) * D * 128;   // sqrt(d) Q, hi + lo
         // a CTA holding all 512 TMEM columns (d + m > 256) gets an SM to itself
         if (D + p.M > 256 && smem < 120 * 1024) smem = 120 * 1024;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -843,37 +1084,59 @@ cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &map, in
             cudaGetLastError();   // do not leave the failure as the thread's sticky last error
             return;
         }
-        kern<<<(unsigned)grid, ENC_ROWS, smem, s>>>(p, map);
+        kern<<<(unsigned)grid, ENC_ROWS, smem, s>>>(p, mapS, mapQ);
         e = cudaGetLastError();
     };
     switch (bits) {
-        case 2: go(tq_encode_k_kernel<D, 1, Tin>); break;
-        case 3: go(tq_encode_k_kernel<D, 2, Tin>); break;
-        case 4: go(tq_encode_k_kernel<D, 3, Tin>); break;
-        case 5: go(tq_encode_k_kernel<D, 4, Tin>); break;
+        case 2: go(tq_encode_k_kernel<D, 1, Tin, ROT>); break;
+        case 3: go(tq_encode_k_kernel<D, 2, Tin, ROT>); break;
+        case 4: go(tq_encode_k_kernel<D, 3, Tin, ROT>); break;
+        case 5: go(tq_encode_k_kernel<D, 4, Tin, ROT>); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return e;
+}
+
+template <int D, typename Tin, int ROT>
+cudaError_t launch_v(int bits, const EncodeParams &p, const CUtensorMap &mapQ, int64_t grid, cudaStream_t s) {
+    cudaError_t e = cudaSuccess;
+    auto go = [&](auto kern) {
+        size_t smem = 0;
+        if (ROT == 1)   // 1024-byte alignment slack, sqrt(d) Q (hi + lo), the row operand (hi [+ lo])
+            smem = 1024 + 2 * (size_t)(D / 64) * D * 128 + (sizeof(Tin) == 2 ? 1 : 2) * (size_t)(D / 64) * ENC_ROWS * 128;
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return;
+            }
+        }
+        kern<<<(unsigned)grid, ENC_ROWS, smem, s>>>(p, mapQ);
+        e = cudaGetLastError();
+    };
+    switch (bits) {
+        case 2: go(tq_encode_v_kernel<D, 2, Tin, ROT>); break;
+        case 3: go(tq_encode_v_kernel<D, 3, Tin, ROT>); break;
+        case 4: go(tq_encode_v_kernel<D, 4, Tin, ROT>); break;
+        case 5: go(tq_encode_v_kernel<D, 5, Tin, ROT>); break;
         default: return cudaErrorInvalidValue;
     }
     return e;
 }
 
 template <int D, typename Tin>
-cudaError_t launch_v(int bits, const EncodeParams &p, int64_t grid, cudaStream_t s) {
-    switch (bits) {
-        case 2: tq_encode_v_kernel<D, 2, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
-        case 3: tq_encode_v_kernel<D, 3, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
-        case 4: tq_encode_v_kernel<D, 4, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
-        case 5: tq_encode_v_kernel<D, 5, Tin><<<(unsigned)grid, ENC_ROWS, 0, s>>>(p); break;
-        default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
+cudaError_t launch_dim(const tq_ctx *ctx, bool keys, const EncodeParams &p, int64_t grid, cudaStream_t s) {
+    if (ctx->rotation == TQ_ROT_HAAR)
+        return keys ? launch_k<D, Tin, 1>(ctx->bits, p, ctx->tmap_S, ctx->tmap_Q, grid, s)
+                    : launch_v<D, Tin, 1>(ctx->bits, p, ctx->tmap_Q, grid, s);
+    return keys ? launch_k<D, Tin, 0>(ctx->bits, p, ctx->tmap_S, ctx->tmap_Q, grid, s)
+                : launch_v<D, Tin, 0>(ctx->bits, p, ctx->tmap_Q, grid, s);
 }
 
 template <typename Tin>
 cudaError_t launch_side(const tq_ctx *ctx, bool keys, const EncodeParams &p, int64_t grid, cudaStream_t s) {
-    if (ctx->d == 128)
-        return keys ? launch_k<128, Tin>(ctx->bits, p, ctx->tmap_S, grid, s) : launch_v<128, Tin>(ctx->bits, p, grid, s);
-    if (ctx->d == 64)
-        return keys ? launch_k<64, Tin>(ctx->bits, p, ctx->tmap_S, grid, s) : launch_v<64, Tin>(ctx->bits, p, grid, s);
+    if (ctx->d == 128) return launch_dim<128, Tin>(ctx, keys, p, grid, s);
+    if (ctx->d == 64) return launch_dim<64, Tin>(ctx, keys, p, grid, s);
     return cudaErrorInvalidValue;
 }
 

@@ -30,6 +30,13 @@ struct tq_ctx {
     // Lloyd-Max codebooks of N(0,1): centroids ascending and boundaries.
     float ck[TQ_MAX_LEVELS], bk[TQ_MAX_LEVELS], cv[TQ_MAX_LEVELS], bv[TQ_MAX_LEVELS];
     struct TqBook *d_book;          // device copy of the positive halves (TqBook)
+    int rotation;                   // tq_rotation
+    // Haar rotation tables (rotation == TQ_ROT_HAAR): Q [heads][d][d] fp32,
+    // and sqrt(d) Q as binary16 hi + lo [heads][2][d][d] with its TMA map
+    // (inner d, outer heads*2*d rows, box 64 x d, 128-byte swizzle).
+    float *d_Q32;
+    __half *d_Qh;
+    CUtensorMap tmap_Q;
 };
 
 // Positive halves of the codebooks: magnitudes of the centroids and the

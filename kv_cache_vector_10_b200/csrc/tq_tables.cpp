@@ -7,6 +7,12 @@
 //    and fill the QJL matrix S row-major [m][d], each rounded to binary16
 //    (nearest, ties to even) -- the rounded value is the matrix the codec
 //    uses, which also makes it exact as a tensor-core operand.
+//  * Haar rotations (turboquant-plus-rs README, Modules: rotation --
+//    "Haar-distributed rotation via QR"): Q = the orthogonal factor of the
+//    QR factorization of a d x d Gaussian matrix G with R's diagonal
+//    positive.  G's entries are Box-Muller pairs continuing head h's stream
+//    after the sign and S draws.  The factorization here is Gram-Schmidt run
+//    twice per column (its R diagonal is a norm, hence positive), in fp64.
 //  * Lloyd-Max codebooks of N(0,1) (turboquant-plus-rs README, Modules:
 //    "codebook -- optimal MSE centroids, closed-form (1-2 bit) and Lloyd's
 //    algorithm (3+ bit)"): the iteration runs on the positive half-line,
@@ -59,6 +65,40 @@ extern "C" __attribute__((visibility("hidden"))) void tq_host_head_tables(int d,
         S_bits[i] = to_binary16_bits(rad * std::cos(ang));
         if (i + 1 < total) S_bits[i + 1] = to_binary16_bits(rad * std::sin(ang));
     }
+}
+
+extern "C" __attribute__((visibility("hidden"))) void tq_host_haar(int d, int m, uint64_t seed, int h, double *Q) {
+    SplitMix64 g{seed + (uint64_t)(int64_t)h};
+    for (int j = 0; j < d; ++j) g.next();                    // rotation signs
+    const int64_t sdraws = (int64_t)m * d + (((int64_t)m * d) & 1);
+    for (int64_t i = 0; i < sdraws; ++i) g.next();            // S, drawn in pairs
+    const int64_t n = (int64_t)d * d;
+    double *G = new double[n];
+    for (int64_t i = 0; i < n; i += 2) {
+        const uint64_t a = g.next(), b = g.next();
+        const double u1 = (double)((a >> 11) + 1) * 0x1.0p-53;
+        const double u2 = (double)(b >> 11) * 0x1.0p-53;
+        const double rad = std::sqrt(-2.0 * std::log(u1));
+        const double ang = 2.0 * M_PI * u2;
+        G[i] = rad * std::cos(ang);
+        if (i + 1 < n) G[i + 1] = rad * std::sin(ang);
+    }
+    double *v = new double[d];
+    for (int k = 0; k < d; ++k) {
+        for (int i = 0; i < d; ++i) v[i] = G[(int64_t)i * d + k];
+        for (int pass = 0; pass < 2; ++pass)
+            for (int c = 0; c < k; ++c) {
+                double r = 0.0;
+                for (int i = 0; i < d; ++i) r += Q[(int64_t)i * d + c] * v[i];
+                for (int i = 0; i < d; ++i) v[i] -= r * Q[(int64_t)i * d + c];
+            }
+        double nv = 0.0;
+        for (int i = 0; i < d; ++i) nv += v[i] * v[i];
+        nv = std::sqrt(nv);
+        for (int i = 0; i < d; ++i) Q[(int64_t)i * d + k] = v[i] / nv;
+    }
+    delete[] v;
+    delete[] G;
 }
 
 // Centroids c[L] (ascending) and boundaries beta[L-1] of the 2^B-level
