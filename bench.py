@@ -97,8 +97,8 @@ def arm_config(workload):
 # holding that kernel when the counters were taken: once the source changes
 # the entry no longer applies (traffic: null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): ("tq_encode.cu", "c5bf4a225cbdb7e1b79fa72f7f4140215e6c26ca", 326849024),
-    ("encode_values", "mha_decode"): ("tq_encode.cu", "c5bf4a225cbdb7e1b79fa72f7f4140215e6c26ca", 321014272),
+    ("encode_keys", "mha_decode"): ("tq_encode.cu", "f99a18f2572104ce3e0252f1739063f8a49ec903", 326895872),
+    ("encode_values", "mha_decode"): ("tq_encode.cu", "f99a18f2572104ce3e0252f1739063f8a49ec903", 320783360),
     ("decode", "mha_decode"): ("tq_decode.cu", "420aa8ed6238705ffaaea7f0431d3414d93fcb44", 151321344),
 }
 
