@@ -900,7 +900,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         // cell counts (for sum C[idx]^2) and sum |u| C[idx]
         int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         float2 ucp = make_float2(0.f, 0.f);
-#pragma unroll 1
+#pragma unroll 2
         for (int c = 0; c < NC; ++c) {
             float u[32];
             tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
@@ -968,7 +968,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
         // D: residual u - n_s C[idx] as binary16 hi + lo, swizzled K-major operand
         float2 e2p = make_float2(0.f, 0.f);
-#pragma unroll 1
+#pragma unroll 2
         for (int c = 0; c < NC; ++c) {
             float u[32], cv[32];
             tqdev::tmem_ld_32x32b_x32_nowait(tlane + 32 * c, u);
@@ -1045,7 +1045,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         }
         tqdev::tc_fence_after();
         uint32_t *sdst = dst + BK * NC;
-#pragma unroll 1
+#pragma unroll 2
         for (int c = 0; c < M / 32; ++c) {
             float pv[32];
             tqdev::tmem_ld_32x32b_x32_nowait(tP + (uint32_t)(c * 32), pv);
