@@ -272,6 +272,17 @@ tq_status tq_decode_attention_static(const tq_segment *segs, int n_segs, const v
  * wait inside a kernel gave up; its outputs for that tile are invalid). */
 tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags);
 
+/* Failure-detection self-test (the paper has no counterpart): enqueue one
+ * kernel that waits, bounded by timeout_us of wall time (1..100000), on an
+ * mbarrier phase nothing completes, and records the timeout in the
+ * context's status word exactly as the library's kernels do when one of
+ * their waits runs out.  Afterwards tq_get_status reports error flag bit 0,
+ * kernels of this context skip their work (key encode and decode; their
+ * outputs are invalid) until tq_reset_status clears the word, and the
+ * context is usable again.  No fault, trap or unbounded wait is involved.
+ * TQ_ERR_LIMIT for a timeout outside the range. */
+tq_status tq_selftest_wait_timeout(tq_ctx *ctx, uint32_t timeout_us, void *stream);
+
 /* Zero the status word (enqueued on `stream`). */
 tq_status tq_reset_status(tq_ctx *ctx, void *stream);
 

@@ -36,7 +36,8 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
 EXPORTED = ["tq_create", "tq_create_ex", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
-            "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes"]
+            "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes",
+            "tq_selftest_wait_timeout"]
 
 
 class TQError(RuntimeError):
@@ -81,6 +82,7 @@ def _load():
         "tq_decode_append_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
         "tq_get_status": (I, [V, V, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32)]),
         "tq_reset_status": (I, [V, V]),
+        "tq_selftest_wait_timeout": (I, [V, ctypes.c_uint32, V]),
         "tq_status_string": (ctypes.c_char_p, [I]),
         "tq_last_cuda_error": (ctypes.c_char_p, []),
     }
@@ -227,6 +229,11 @@ def tq_get_status(ctx: int, stream=None):
     f = ctypes.c_uint32()
     _check(_lib.tq_get_status(ctx, _stream(stream), ctypes.byref(n), ctypes.byref(f)), "tq_get_status")
     return n.value, f.value
+
+
+def tq_selftest_wait_timeout(ctx: int, timeout_us: int, stream=None):
+    """Make one bounded wait run out on purpose (see include/tq.h)."""
+    _check(_lib.tq_selftest_wait_timeout(ctx, timeout_us, _stream(stream)), "tq_selftest_wait_timeout")
 
 
 def tq_reset_status(ctx: int, stream=None):

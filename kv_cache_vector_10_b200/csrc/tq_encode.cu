@@ -787,10 +787,9 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // misc region [0, 1024): sign masks, centroid magnitudes, barriers
+    // misc region [0, 1024): sign masks, squared centroid magnitudes, barriers
     uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // <= 512 B
-    float *s_mag = reinterpret_cast<float *>(smem + 512);                   // [16]
-    float *s_mag2 = s_mag + 16;                                             // [16]
+    float *s_mag2 = reinterpret_cast<float *>(smem + 512);                  // [16]
     // [0] S loaded, [1] QJL MMA done, [2] Q loaded, [3] rotation MMA done (dense rotation)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 4);
@@ -809,11 +808,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     // tile's rotation fills U)
     const uint32_t tmem_cols = tmem_cols_for(D + (M > D ? M : D));
     build_sign_masks<Tin, D>(p.signs + (int64_t)head * (D / 32), s_mask);
-    if (tid < 16) {
-        const float mg = tid < HK ? p.mag[tid] : 0.f;
-        s_mag[tid] = mg;
-        s_mag2[tid] = mg * mg;
-    }
+    if (tid < 16) s_mag2[tid] = tid < HK ? p.mag[tid] * p.mag[tid] : 0.f;
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) tqdev::mbar_init(&bars[i], 1);
         *s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
@@ -851,7 +846,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     }
 #pragma unroll 1
     for (int tile = 0; tile < ntiles; ++tile) {
-        if (*s_abort) break;   // uniform: set before the barrier that ends the previous tile
+        if (tile == 0 && *s_abort) break;   // uniform: set before the set-up barrier
         const int64_t t = tb0 + tile * ENC_ROWS + tid;
         const bool valid = t < p.T;
         float inv_scale = 1.f;
@@ -1001,10 +996,11 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
             dst[tail] = __float_as_uint(ns * inv_scale);
             dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)) * inv_scale);
         }
-        // E: the QJL projection on the tensor cores (TMEM columns [d, d + m))
+        // E: the QJL projection on the tensor cores (TMEM columns [d, d + m));
+        // an abort flag set by any thread ends the loop here, for all threads
         tqdev::fence_proxy_async_smem();
         tqdev::tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(*s_abort)) break;
         if (tid == 0) {
             const bool ok = tile > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
             if (!ok) {
@@ -1038,10 +1034,12 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         }
         // F: sign epilogue
         const bool done = tqdev::mbar_wait_bounded(&bars[1], (uint32_t)(tile & 1));
-        if (__syncthreads_or(!done || *s_abort)) {
-            if (tid == 0 && !done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
-            if (tid == 0) *s_abort = 1;
-            break;
+        if (!done || *s_abort) {
+            // this thread skips the epilogue; the flag ends the loop for every
+            // thread at the next pre-MMA barrier
+            if (!done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+            *s_abort = 1;
+            continue;
         }
         tqdev::tc_fence_after();
         uint32_t *sdst = dst + BK * NC;
