@@ -97,8 +97,8 @@ def arm_config(workload):
 # holding that kernel when the counters were taken: once the source changes
 # the entry no longer applies (traffic: null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): ("tq_encode.cu", "f99a18f2572104ce3e0252f1739063f8a49ec903", 326895872),
-    ("encode_values", "mha_decode"): ("tq_encode.cu", "f99a18f2572104ce3e0252f1739063f8a49ec903", 320783360),
+    ("encode_keys", "mha_decode"): ("tq_encode.cu", "0090ee5f532343ec656f1565a641d05b552cea39", 326150912),
+    ("encode_values", "mha_decode"): ("tq_encode.cu", "0090ee5f532343ec656f1565a641d05b552cea39", 320644352),
     ("decode", "mha_decode"): ("tq_decode.cu", "420aa8ed6238705ffaaea7f0431d3414d93fcb44", 151321344),
 }
 
