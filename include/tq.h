@@ -25,6 +25,10 @@
  *    and returned as tq_status; nothing runs in that case.
  *  - There is no CPU fallback: if the device is not an sm_100 GPU or the
  *    kernels cannot launch, the call returns TQ_ERR_DEVICE / TQ_ERR_CUDA.
+ *  - Threads: different contexts may be used from different host threads at
+ *    once.  Calls on one context from several threads must be serialized
+ *    by the caller when any of them may build head tables (tq_ensure_heads,
+ *    or a call using more heads than built so far).
  *  - d = head_dim, m = projections, b = bits, B_K = b-1, B_V = b.
  *
  * Packed row formats (the pages give no layout; this is the library's):

@@ -2,6 +2,7 @@
 // table upload and kernel dispatch.  No computation on the data path
 // happens on the host; every step runs in the kernels of tq_encode.cu,
 // tq_decode.cu and tq_aux.cu.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -35,14 +36,16 @@ tq_status tq_check_cuda(cudaError_t e) {
 }
 
 static int device_sms(int dev) {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];   // zero-initialized; concurrent fills store the same value
     if (dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
+    int v = cached[dev].load(std::memory_order_relaxed);
+    if (!v) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 148;
+        v = n > 0 ? n : 148;
+        cached[dev].store(v, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return v;
 }
 
 tq_status tq_check_device(const tq_ctx *ctx) {
@@ -58,14 +61,15 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32
                                     CUtensorMapFloatOOBfill);
 
 static PFN_encodeTiled get_encode_tiled() {
-    static PFN_encodeTiled fn = nullptr;
-    if (!fn) {
+    // looked up once, thread-safely (function-local static initialization)
+    static const PFN_encodeTiled fn = [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_encodeTiled>(p);
-    }
+            return reinterpret_cast<PFN_encodeTiled>(p);
+        return static_cast<PFN_encodeTiled>(nullptr);
+    }();
     return fn;
 }
 

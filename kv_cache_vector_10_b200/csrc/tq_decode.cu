@@ -609,7 +609,9 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
     (void)ws_bytes;
     std::vector<SegPlan> pl;
     plan_segments(segs, n_segs, Hq, Hkv, n_sms, pl);
-    static DecodePlan P;   // large; filled per call on the host
+    // large (it is the kernels' parameter block); one per host thread, so
+    // calls from different threads do not share it
+    thread_local DecodePlan P;
     P = DecodePlan{};
     P.n_segs = n_segs;
     P.Hq = Hq;
