@@ -79,6 +79,8 @@ def _load():
         _lib.tqo_scores_fused.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, ctypes.c_int64, P]
         _lib.tqo_scores_dequant.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, ctypes.c_int64, P]
         _lib.tqo_attend.argtypes = [ctypes.c_int, P, P, P, P, P, P, P, P]
+        _lib.tqo_attend_split.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, ctypes.POINTER(_Cfg), P, P, P, P,
+                                          ctypes.c_int64, P, P]
         _lib.tqo_streaming_softmax_sum.argtypes = [ctypes.c_int64, ctypes.c_int, P, P, ctypes.c_int64, P]
         _lib.tqo_packed_bytes.restype = ctypes.c_int64
         _lib.tqo_packed_bytes.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64]
@@ -303,4 +305,19 @@ def streaming_softmax_sum(scores, vals, blk: int) -> np.ndarray:
     vals = _f64(vals)
     out = np.zeros(vals.shape[1])
     _load().tqo_streaming_softmax_sum(scores.shape[0], vals.shape[1], _p(scores), _p(vals), blk, _p(out))
+    return out
+
+
+def attention_split(q, part_o, part_n) -> np.ndarray:
+    """Decode attention of one query q [d_o + d_n] over a split cache: part_x =
+    (codec, h, krows, vrows) for the outlier group (channels first) and the
+    normal group; both hold the same tokens."""
+    q = _f64(q)
+    (co, ho, ko, vo), (cn, hn, kn, vn) = part_o, part_n
+    ro, So = co.tables(ho)
+    rn, Sn = cn.tables(hn)
+    ko, vo, kn, vn = (np.ascontiguousarray(a, dtype=np.uint8) for a in (ko, vo, kn, vn))
+    out = np.zeros(co.d + cn.d)
+    _load().tqo_attend_split(ctypes.byref(co.cfg), _p(_f64(ro)), _p(So), _p(ko), _p(vo), ctypes.byref(cn.cfg),
+                             _p(_f64(rn)), _p(Sn), _p(kn), _p(vn), ko.shape[0], _p(q), _p(out))
     return out

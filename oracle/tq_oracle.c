@@ -51,6 +51,15 @@
  *       pairs (not rounded) from the head's SplitMix64 stream continued after
  *       the d sign draws and the draws of S.  The rest of the method is
  *       unchanged: z = sqrt(d) Q x / ||x||, reconstruction Q^T (...).
+ *   R10 Outlier/normal channel splitting ([TQ] Modules, outlier: "Non-integer
+ *       bit rates via outlier/normal channel splitting"): a head's d channels
+ *       are split into two groups, outliers first (the caller orders the
+ *       channels); each group is a codec of its own (its own rotation over the
+ *       group's channels, its own bits), so the bits per value are the
+ *       channel-weighted mean.  A key's score is the full inner product
+ *       q.k_hat / sqrt(d) = (sum over groups g of q_g . k_hat_g) / sqrt(d); one
+ *       softmax covers the token; the value is the concatenation of the groups'
+ *       reconstructions.
  *   R8  Packed layout (the pages give none):
  *       K row: B_K index bit planes (plane p holds bit p of every index;
  *       coordinate j -> byte j/8, bit j%8), then the m-bit sign plane, then
@@ -655,4 +664,40 @@ void tqo_streaming_softmax_sum(int64_t T, int d, const double *scores, const dou
  * [BP] compression_ratio = original bytes / compressed bytes). */
 int64_t tqo_packed_bytes(const tqo_cfg *cfg, int64_t n_rows) {
     return n_rows * (int64_t)(tqo_k_row_bytes(cfg) + tqo_v_row_bytes(cfg));
+}
+
+/* Decode attention of one query q[d_o + d_n] over T tokens of a split cache
+ * (R10): group o (channels [0, d_o)) and group n (channels [d_o, d)) with
+ * their own configs, rotation tables and packed rows.  Scores from each
+ * group's dequantized keys (materialized), one softmax over the token's
+ * total score, values concatenated. */
+void tqo_attend_split(const tqo_cfg *co, const double *rot_o, const double *S_o, const uint8_t *krows_o,
+                      const uint8_t *vrows_o, const tqo_cfg *cn, const double *rot_n, const double *S_n,
+                      const uint8_t *krows_n, const uint8_t *vrows_n, int64_t T, const double *q, double *out) {
+    const int d_o = co->d, d_n = cn->d, d = d_o + d_n;
+    for (int j = 0; j < d; ++j) out[j] = 0.0;
+    if (T == 0) return;
+    double *sc = (double *)malloc(sizeof(double) * (size_t)T);
+    double *kh = (double *)malloc(sizeof(double) * d);
+    double *vh = (double *)malloc(sizeof(double) * d);
+    const int rko = tqo_k_row_bytes(co), rkn = tqo_k_row_bytes(cn);
+    const int rvo = tqo_v_row_bytes(co), rvn = tqo_v_row_bytes(cn);
+    for (int64_t t = 0; t < T; ++t) {
+        tqo_dequant_k(co, rot_o, S_o, krows_o + t * rko, kh);
+        tqo_dequant_k(cn, rot_n, S_n, krows_n + t * rkn, kh + d_o);
+        double a = 0.0;
+        for (int j = 0; j < d; ++j) a += q[j] * kh[j];
+        sc[t] = a / sqrt((double)d);
+    }
+    double mx = -INFINITY;
+    for (int64_t t = 0; t < T; ++t) if (sc[t] > mx) mx = sc[t];
+    double den = 0.0;
+    for (int64_t t = 0; t < T; ++t) { sc[t] = exp(sc[t] - mx); den += sc[t]; }
+    for (int64_t t = 0; t < T; ++t) {
+        tqo_dequant_v(co, rot_o, vrows_o + t * rvo, vh);
+        tqo_dequant_v(cn, rot_n, vrows_n + t * rvn, vh + d_o);
+        const double p = sc[t] / den;
+        for (int j = 0; j < d; ++j) out[j] += p * vh[j];
+    }
+    free(sc); free(kh); free(vh);
 }

@@ -503,3 +503,52 @@ def test_compression_table_arithmetic():
     for bits, bpv_ours in ((4, 4.375), (3, 3.375), (2, 2.375)):
         codec = oracle.Codec(128, bits, 128, 0)
         assert codec.packed_bytes(1) * 8 / (2 * 128) == bpv_ours
+
+
+# ------------------------------------------------------ outlier splitting
+
+def _split_parts(seed=3, T=60, bits=(4, 3)):
+    rng = np.random.default_rng(seed)
+    co, cn = oracle.Codec(64, bits[0], 64, 11), oracle.Codec(64, bits[1], 64, 29)
+    K = rng.standard_normal((T, 128)) * np.r_[np.full(64, 4.0), np.ones(64)]
+    V = rng.standard_normal((T, 128))
+    eko, evo = co.encode(K[:, :64], 2, True), co.encode(V[:, :64], 2, False)
+    ekn, evn = cn.encode(K[:, 64:], 2, True), cn.encode(V[:, 64:], 2, False)
+    return rng, co, cn, (co, 2, eko["rows"], evo["rows"]), (cn, 2, ekn["rows"], evn["rows"])
+
+
+def test_split_attention_is_softmax_over_the_concatenated_reconstruction():
+    """Brute force: keys and values are the concatenations of the two groups'
+    dequantized rows; scores q.k_hat / sqrt(128); one softmax over tokens."""
+    rng, co, cn, po, pn = _split_parts()
+    kh = np.concatenate([co.dequant(po[2], 2, True), cn.dequant(pn[2], 2, True)], axis=1)
+    vh = np.concatenate([co.dequant(po[3], 2, False), cn.dequant(pn[3], 2, False)], axis=1)
+    for _ in range(3):
+        q = rng.standard_normal(128)
+        s = kh @ q / math.sqrt(128)
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        assert np.allclose(oracle.attention_split(q, po, pn), p @ vh, atol=1e-12)
+
+
+def test_split_scores_are_the_groups_scores_rescaled():
+    """With q zero on the normal group, every token's split score is the outlier
+    group's own score times sqrt(64 / 128): the attention equals a softmax of the
+    group's scores scaled by 1/sqrt(2)."""
+    rng, co, cn, po, pn = _split_parts(seed=5)
+    q = np.r_[rng.standard_normal(64), np.zeros(64)]
+    so = co.scores(q[:64], po[2], 2) * math.sqrt(64 / 128)
+    p = np.exp(so - so.max())
+    p /= p.sum()
+    vh = np.concatenate([co.dequant(po[3], 2, False), cn.dequant(pn[3], 2, False)], axis=1)
+    assert np.allclose(oracle.attention_split(q, po, pn), p @ vh, atol=1e-12)
+
+
+def test_split_bits_per_value():
+    """Channel-weighted bits: 64 outlier channels at b + 1 and 64 at b give b + 1/2
+    index bits per value (the non-integer rates the module names)."""
+    for b in (2, 3, 4):
+        co, cn = oracle.Codec(64, b + 1, 64, 1), oracle.Codec(64, b, 64, 1)
+        idx_bits = 64 * co.bits + 64 * cn.bits   # value rows: b index bits per coordinate
+        assert idx_bits / 128 == b + 0.5
+        assert co.v_row_bytes - 4 + cn.v_row_bytes - 4 == (64 * (b + 1) + 64 * b) // 8
