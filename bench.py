@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha_decode",
                     choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head",
-                             "mha_append", "mha_decode_haar"])
+                             "mha_append", "mha_decode_haar", "mha_split"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -76,6 +76,9 @@ WORKLOAD_DESC = {
                   "(sequence, kv head), d128, m128, bits 4 (K 3+1, V 4), float16",
     "mha_decode_haar": "mha_decode_haar: the mha_decode workload with the Haar-QR rotation (batch 8, 32 heads, "
                        "4096 tokens, d128, m128, bits 4, float16)",
+    "mha_split": "mha_split: the mha_decode data (batch 8, 32 heads, 4096 tokens, d128, fp16) split per head into "
+                 "64 outlier channels (largest RMS) at bits 4 and 64 normal channels at bits 3 (3.5 index bits per "
+                 "value), m64 per group",
 }
 
 
@@ -83,6 +86,7 @@ STEP_DESC = {w: "encode all K/V rows + one decode step per query head"
              for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head", "mha_decode_haar")}
 STEP_DESC["bulk_encode"] = "encode all K/V rows of 32 layers"
 STEP_DESC["mha_append"] = "append one token per (sequence, kv head) + one decode step per query head"
+STEP_DESC["mha_split"] = "encode both channel groups of all K/V rows + one split decode step per query head"
 L2_DESC = ("flushed (256 MiB write) before every timed piece, outside its CUDA events; "
            "ms_per_step = sum of the pieces")
 
@@ -171,6 +175,29 @@ class Workload:
                 self.pieces = [("encode_keys", B * Hkv * T * (D * es + kr), 1),
                                ("encode_values", B * Hkv * T * (D * es + vr), 1),
                                ("decode", B * Hkv * T * (kr + vr) + qb, 3)]
+        elif name == "mha_split":
+            w = W.mha_decode(device=device, data_seed=2 + seed_shift)
+            B, H, T, _ = w["k"].shape
+            # channels ordered per head by RMS over the cached keys: outliers first
+            order = w["k"].float().pow(2).mean(dim=(0, 2)).argsort(dim=-1, descending=True)   # [H, d]
+            idx = order[None, :, None, :]
+            k = torch.gather(w["k"], 3, idx.expand_as(w["k"])).contiguous()
+            v = torch.gather(w["v"], 3, idx.expand_as(w["v"])).contiguous()
+            q = torch.gather(w["q"], 2, order[None].expand_as(w["q"])).contiguous()
+            self.codec_o = tq.Codec(64, 4, 64, w["seed"])
+            self.codec_n = tq.Codec(64, 3, 64, w["seed"] + 1000)
+            self.cache_o = self.codec_o.alloc(B, H, T, device)
+            self.cache_n = self.codec_n.alloc(B, H, T, device)
+            self.inputs = dict(k=k, v=v, q=q)
+            self.B, self.Hq, self.Hkv, self.T = B, H, H, T
+            self.tokens_scored = B * H * T
+            es = k.element_size()
+            ko, vo = 3 * 8 + 8 + 8, 4 * 8 + 4
+            kn, vn = 2 * 8 + 8 + 8, 3 * 8 + 4
+            qb = B * H * D * 2 * es
+            self.pieces = [("encode_keys", B * H * T * (D * es + ko + kn), 2),
+                           ("encode_values", B * H * T * (D * es + vo + vn), 2),
+                           ("decode_split", B * H * T * (ko + kn + vo + vn) + qb, 5)]
         elif name == "shared_prefix":
             w = W.shared_prefix(device=device, data_seed=5 + seed_shift)
             self.w = w
@@ -232,8 +259,24 @@ class Workload:
             tq.tq_decode_attention(self.segments, inp["q"], self.B, self.Hq, self.Hkv, self.out, self.ws)
 
     def _run_piece(self, name, inp):
+        if name == "decode_split":
+            if self.out is None:
+                torch = self.torch
+                need = self.tq.lib.tq_decode_split_workspace_bytes(self.codec_o.ctx, self.codec_n.ctx, self.B,
+                                                                   self.Hq, self.T)
+                self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=inp["q"].device)
+            self.out = self.tq.decode_split(self.codec_o, self.cache_o, self.codec_n, self.cache_n, self.T, inp["q"],
+                                            workspace=self.ws)
+            return
         if name == "encode_keys" or name == "encode_values":
             side = "k" if name == "encode_keys" else "v"
+            if self.name == "mha_split":
+                x = inp[side]
+                a = (x[..., :64], None) if side == "k" else (None, x[..., :64])
+                self.codec_o.encode_kv(*a, self.cache_o)
+                a = (x[..., 64:], None) if side == "k" else (None, x[..., 64:])
+                self.codec_n.encode_kv(*a, self.cache_n)
+                return
             if self.name == "shared_prefix":
                 args_p = (inp["pk"], None) if side == "k" else (None, inp["pv"])
                 args_t = (inp["tk"], None) if side == "k" else (None, inp["tv"])
@@ -358,6 +401,18 @@ def oracle_unit(wl_name, rank_seed=0):
                              [(pc, 0, ekp["rows"], evp["rows"]), (tc, 0, ekt["rows"], evt["rows"])])
         dt = time.perf_counter() - t0
         return dt, 4 * (1024 + 256), "tokens", "1 agent x 1 kv head (4 q heads), prefix 1024 + tail 256 tokens"
+    if wl_name == "mha_split":
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=512)
+        order = w["k"][0, 0].pow(2).mean(dim=0).argsort(descending=True)
+        k, v, q = (w["k"][0, 0][:, order].double().numpy(), w["v"][0, 0][:, order].double().numpy(),
+                   w["q"][0, 0][order].double().numpy())
+        oo, on = oracle.Codec(64, 4, 64, w["seed"]), oracle.Codec(64, 3, 64, w["seed"] + 1000)
+        t0 = time.perf_counter()
+        eko, evo = oo.encode(k[:, :64], 0, True), oo.encode(v[:, :64], 0, False)
+        ekn, evn = on.encode(k[:, 64:], 0, True), on.encode(v[:, 64:], 0, False)
+        oracle.attention_split(q, (oo, 0, eko["rows"], evo["rows"]), (on, 0, ekn["rows"], evn["rows"]))
+        dt = time.perf_counter() - t0
+        return dt, 512, "tokens", "1 kv head x 1 query head x 512 tokens: encode both channel groups + split decode"
     if wl_name == "mha_append":
         w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1025)
         oc = oracle.Codec(D, w["bits"], M, w["seed"])

@@ -276,6 +276,29 @@ tq_status tq_decode_attention_static(const tq_segment *segs, int n_segs, const v
  * wait inside a kernel gave up; its outputs for that tile are invalid). */
 tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags);
 
+/* Decode attention over an outlier/normal channel-split cache
+ * (turboquant-plus-rs README, Modules: outlier -- "Non-integer bit rates via
+ * outlier/normal channel splitting").  A head's channels are split into an
+ * outlier group (the first d_o channels, codec ctx_o) and a normal group (the
+ * next d_n channels, codec ctx_n); each group is encoded with tq_encode_kv
+ * of its own codec (e.g. 64 channels at b+1 bits and 64 at b: b + 1/2 index
+ * bits per value), so the caller orders the channels outliers first.  For
+ * every sequence b and query head j:
+ *   s_t = q . k_hat_t / sqrt(d_o + d_n)  (k_hat_t: both groups' keys),
+ *   out[b][j] = sum_t softmax_t(s_t) v_hat_t  (v_hat_t: both groups' values).
+ *  codes_o, codes_n : the groups' caches, same batch, kv heads and capacity;
+ *                     tokens [0, n_tokens) of batch slot b are sequence b's.
+ *  q, out           : device [batch][n_q_heads][d_o + d_n], outliers first.
+ *  workspace        : >= tq_decode_split_workspace_bytes(...), 16-byte aligned.
+ * Query head j reads kv head j / (n_q_heads / n_kv_heads).  Launches four
+ * kernels: the query's groups as fp32, each group's exact scores, and one
+ * softmax-and-value kernel. */
+size_t tq_decode_split_workspace_bytes(const tq_ctx *ctx_o, const tq_ctx *ctx_n, int batch, int n_q_heads,
+                                       int64_t n_tokens);
+tq_status tq_decode_attention_split(tq_ctx *ctx_o, const tq_codes *codes_o, tq_ctx *ctx_n, const tq_codes *codes_n,
+                                    int64_t n_tokens, const void *q, tq_dtype q_dtype, int batch, int n_q_heads,
+                                    void *out, tq_dtype out_dtype, void *workspace, size_t ws_bytes, void *stream);
+
 /* Failure-detection self-test (the paper has no counterpart): enqueue one
  * kernel that waits, bounded by timeout_us of wall time (1..100000), on an
  * mbarrier phase nothing completes, and records the timeout in the

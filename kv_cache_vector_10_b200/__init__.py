@@ -37,7 +37,7 @@ EXPORTED = ["tq_create", "tq_create_ex", "tq_destroy", "tq_ensure_heads", "tq_ro
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
             "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes",
-            "tq_selftest_wait_timeout"]
+            "tq_selftest_wait_timeout", "tq_decode_attention_split", "tq_decode_split_workspace_bytes"]
 
 
 class TQError(RuntimeError):
@@ -83,6 +83,9 @@ def _load():
         "tq_get_status": (I, [V, V, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint32)]),
         "tq_reset_status": (I, [V, V]),
         "tq_selftest_wait_timeout": (I, [V, ctypes.c_uint32, V]),
+        "tq_decode_split_workspace_bytes": (SZ, [V, V, I, I, I64]),
+        "tq_decode_attention_split": (I, [V, ctypes.POINTER(tq_codes), V, ctypes.POINTER(tq_codes), I64, V, I, I, I,
+                                          V, I, V, SZ, V]),
         "tq_status_string": (ctypes.c_char_p, [I]),
         "tq_last_cuda_error": (ctypes.c_char_p, []),
     }
@@ -345,6 +348,27 @@ def decode_append(segments, k_new, v_new, q, n_kv_heads: int, out_dtype=None, wo
     for s in segments:
         if s.n_seqs == 1:
             s.n_tokens += 1
+    return out
+
+
+def decode_split(codec_o, cache_o, codec_n, cache_n, n_tokens: int, q, out_dtype=None, workspace=None,
+                 stream=None):
+    """Decode attention over an outlier/normal channel-split cache: q [batch,
+    n_q_heads, d_o + d_n] with the outlier channels first; cache_o / cache_n
+    hold the two groups' codes (codecs codec_o / codec_n)."""
+    import torch
+    B, Hq, d = q.shape
+    out = torch.empty(B, Hq, d, dtype=out_dtype or q.dtype, device=q.device)
+    need = _lib.tq_decode_split_workspace_bytes(codec_o.ctx, codec_n.ctx, B, Hq, n_tokens)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    qc = q.contiguous()
+    co, cn = cache_o.struct(), cache_n.struct()
+    _check(_lib.tq_decode_attention_split(codec_o.ctx, ctypes.byref(co), codec_n.ctx, ctypes.byref(cn), n_tokens,
+                                          qc.data_ptr(), _dtype_code(qc.dtype), B, Hq, out.data_ptr(),
+                                          _dtype_code(out.dtype), workspace.data_ptr(),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tq_decode_attention_split")
     return out
 
 

@@ -23,6 +23,10 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
 tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float *k_hat, float *v_hat,
                             cudaStream_t stream);
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
+size_t tq_split_ws(int batch, int Hq, int d_o, int d_n, int64_t T);
+tq_status tq_launch_split(tq_ctx *co, const tq_codes *ko, tq_ctx *cn, const tq_codes *kn, int64_t T, const void *q,
+                          tq_dtype q_dtype, int batch, int Hq, void *out, tq_dtype out_dtype, void *ws,
+                          cudaStream_t stream);
 tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,
                            int Hq, int Hkv, void *out, tq_dtype out_dtype, void *ws, size_t ws_bytes,
                            cudaStream_t stream, int n_sms, const TqAppend *app = nullptr);
@@ -455,6 +459,37 @@ tq_status tq_decode_append(const tq_segment *segs, int n_segs, const void *k_new
     const TqAppend app{k_new, v_new, kv_dtype, flags.data()};
     return tq_launch_decode(grown.data(), n_segs, q, q_dtype, batch, n_q_heads, n_kv_heads, out, out_dtype,
                             workspace, ws_bytes, static_cast<cudaStream_t>(stream), device_sms(dev), &app);
+}
+
+size_t tq_decode_split_workspace_bytes(const tq_ctx *ctx_o, const tq_ctx *ctx_n, int batch, int n_q_heads,
+                                       int64_t n_tokens) {
+    if (!ctx_o || !ctx_n || batch <= 0 || n_q_heads <= 0 || n_tokens < 0) return 0;
+    return tq_split_ws(batch, n_q_heads, ctx_o->d, ctx_n->d, n_tokens);
+}
+
+tq_status tq_decode_attention_split(tq_ctx *ctx_o, const tq_codes *codes_o, tq_ctx *ctx_n, const tq_codes *codes_n,
+                                    int64_t n_tokens, const void *q, tq_dtype q_dtype, int batch, int n_q_heads,
+                                    void *out, tq_dtype out_dtype, void *workspace, size_t ws_bytes, void *stream) {
+    if (!ctx_o || !ctx_n || !q || !out) return TQ_ERR_NULL;
+    tq_status st = check_codes(ctx_o, codes_o, true, true);
+    if (st == TQ_OK) st = check_codes(ctx_n, codes_n, true, true);
+    if (st != TQ_OK) return st;
+    if (batch <= 0 || n_q_heads <= 0 || n_tokens <= 0) return TQ_ERR_EMPTY;
+    if (codes_o->batch != batch || codes_n->batch != batch || codes_o->n_kv_heads != codes_n->n_kv_heads ||
+        codes_o->capacity != codes_n->capacity || n_q_heads % codes_o->n_kv_heads ||
+        n_tokens > codes_o->capacity)
+        return TQ_ERR_DIM_MISMATCH;
+    if ((q_dtype != TQ_F32 && q_dtype != TQ_F16 && q_dtype != TQ_BF16) ||
+        (out_dtype != TQ_F32 && out_dtype != TQ_F16 && out_dtype != TQ_BF16))
+        return TQ_ERR_DIM_MISMATCH;
+    if ((st = tq_check_device(ctx_o)) != TQ_OK || (st = tq_check_device(ctx_n)) != TQ_OK) return st;
+    if ((st = tq_ensure_heads(ctx_o, codes_o->n_kv_heads)) != TQ_OK) return st;
+    if ((st = tq_ensure_heads(ctx_n, codes_n->n_kv_heads)) != TQ_OK) return st;
+    const size_t need = tq_split_ws(batch, n_q_heads, ctx_o->d, ctx_n->d, n_tokens);
+    if (!workspace || ws_bytes < need) return TQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return TQ_ERR_ALIGN;
+    return tq_launch_split(ctx_o, codes_o, ctx_n, codes_n, n_tokens, q, q_dtype, batch, n_q_heads, out, out_dtype,
+                           workspace, static_cast<cudaStream_t>(stream));
 }
 
 tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags) {

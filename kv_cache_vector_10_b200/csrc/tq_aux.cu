@@ -117,32 +117,54 @@ struct ScoresParams {
     float ck[16];
 };
 
+// One block per (token block, query head, sequence); every thread scores
+// SCORE_TPT tokens, so the query preparation is amortized over
+// SCORE_TPT * AUX_THREADS tokens.
+constexpr int SCORE_TPT = 8;
+
 template <int D>
 __global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_constant__ ScoresParams p) {
     __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
+    __shared__ float s_ck[16];
     const int j = blockIdx.y, b = blockIdx.z;
     const int h = j / (p.Hq / p.Hkv);
+    if (threadIdx.x < 16) s_ck[threadIdx.x] = p.ck[threadIdx.x];
     prep_query<D>(p.q + ((int64_t)b * p.Hq + j) * D, p.signs + (int64_t)h * (D / 32), p.S + (int64_t)h * p.M * D,
-                  p.M, s_qr, s_sq, p.Q ? p.Q + (int64_t)h * D * D : nullptr);
-    const int64_t t = (int64_t)blockIdx.x * AUX_THREADS + threadIdx.x;
-    if (t >= p.T) return;
-    const uint8_t *row = p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) * p.krow;
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
-    float a = 0.f;
-    for (int jj = 0; jj < D; ++jj) {
-        int idx = 0;
-        for (int q = 0; q < p.bk; ++q) idx |= ((w[q * (D / 32) + jj / 32] >> (jj % 32)) & 1) << q;
-        a = fmaf(s_qr[jj], p.ck[idx], a);
-    }
-    const uint32_t *sg = w + p.bk * (D / 32);
-    float bq = 0.f;
-    for (int i = 0; i < p.M; ++i) bq += ((sg[i / 32] >> (i % 32)) & 1) ? s_sq[i] : -s_sq[i];
-    const float ns = __uint_as_float(sg[p.M / 32]);
-    const float gamma = __uint_as_float(sg[p.M / 32 + 1]);
+                  p.M, s_qr, s_sq, p.Q ? p.Q + (int64_t)h * D * D : nullptr);   // its barriers publish s_ck
     const float isd = rsqrtf((float)D);
     const float cq = 1.2533141373155003f / (float)p.M;   // sqrt(pi/2) / m
-    p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (ns * a * isd + cq * gamma * bq) * isd;
+    for (int k = 0; k < SCORE_TPT; ++k) {
+        const int64_t t = ((int64_t)blockIdx.x * SCORE_TPT + k) * AUX_THREADS + threadIdx.x;
+        if (t >= p.T) break;
+        const uint8_t *row = p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) * p.krow;
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
+        float a = 0.f;
+#pragma unroll 1
+        for (int wd = 0; wd < D / 32; ++wd) {
+            uint32_t pl[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pl[q] = q < p.bk ? w[q * (D / 32) + wd] : 0u;
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                int idx = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) idx |= (int)((pl[q] >> i) & 1u) << q;
+                a = fmaf(s_qr[wd * 32 + i], s_ck[idx], a);
+            }
+        }
+        const uint32_t *sg = w + p.bk * (D / 32);
+        float bq = 0.f;
+#pragma unroll 1
+        for (int wd = 0; wd < p.M / 32; ++wd) {
+            const uint32_t sw = sg[wd];
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) bq += ((sw >> i) & 1u) ? s_sq[wd * 32 + i] : -s_sq[wd * 32 + i];
+        }
+        const float ns = __uint_as_float(sg[p.M / 32]);
+        const float gamma = __uint_as_float(sg[p.M / 32 + 1]);
+        p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (ns * a * isd + cq * gamma * bq) * isd;
+    }
 }
 
 struct DequantParams {
@@ -517,7 +539,8 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
     p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
     p.bk = ctx->BK;
     for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
-    dim3 grid((unsigned)((T + AUX_THREADS - 1) / AUX_THREADS), (unsigned)Hq, (unsigned)codes->batch);
+    const int64_t per_block = (int64_t)AUX_THREADS * SCORE_TPT;
+    dim3 grid((unsigned)((T + per_block - 1) / per_block), (unsigned)Hq, (unsigned)codes->batch);
     if (ctx->d == 128) tq_scores_kernel<128><<<grid, AUX_THREADS, 0, stream>>>(p);
     else tq_scores_kernel<64><<<grid, AUX_THREADS, 0, stream>>>(p);
     return tq_check_cuda(cudaGetLastError());
