@@ -109,20 +109,37 @@ def test_encode_deterministic():
     assert torch.equal(c1.k, c2.k) and torch.equal(c1.v, c2.v)
 
 
-def test_encode_nonfinite_and_zero_rows():
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+def test_encode_nonfinite_and_zero_rows(dtype):
     k = torch.randn(1, 2, 40, 128)
     v = torch.randn(1, 2, 40, 128)
     k[0, 0, 3, 5] = float("nan")
     k[0, 1, 7] = 0.0
     v[0, 1, 9, 0] = float("inf")
     v[0, 0, 11] = 0.0
-    gc, oc, cache, ek, ev, rep = _encode_and_compare(k, v, 128, 3, 128, 3)
+    gc, oc, cache, ek, ev, rep = _encode_and_compare(k.to(dtype), v.to(dtype), 128, 3, 128, 3)
     n, flags = gc.status()
     assert n == 2 and flags == 0
     kh, vh = gc.dequantize(cache, 40)
     assert float(kh[0, 0, 3].abs().max()) == 0.0 and float(vh[0, 1, 9].abs().max()) == 0.0
     tq.tq_reset_status(gc.ctx)
     assert gc.status() == (0, 0)
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -18, 2.0 ** -10, 2.0 ** 13])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_encode_16bit_extreme_magnitudes(scale, dtype):
+    """16-bit rows go through the tensor-core chunk transforms with the row in
+    its own type: binary16 subnormals (2^-18), rows mixing subnormal and
+    normal entries (2^-10) and rows near the binary16 maximum (2^13) encode
+    like the oracle."""
+    g = torch.Generator().manual_seed(int(math.log2(scale)) + 40)
+    k = (torch.randn(1, 2, 260, 128, generator=g) * scale).to(dtype)
+    v = (torch.randn(1, 2, 260, 128, generator=g) * scale).to(dtype)
+    for d in (128, 64):
+        gc, *_ , rep = _encode_and_compare(k[..., :d].contiguous(), v[..., :d].contiguous(), d, 4, 64, 21)
+        assert gc.status() == (0, 0)
+        assert rep.get("k_rows_flipped", 0) <= 3 and rep.get("v_index_flips", 0) <= 3, rep
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 5])
