@@ -39,7 +39,7 @@ class _Cfg(ctypes.Structure):
                 ("LV", ctypes.c_int), ("norm_correct", ctypes.c_int),
                 ("ck", ctypes.c_double * 64), ("bk", ctypes.c_double * 64),
                 ("cv", ctypes.c_double * 64), ("bv", ctypes.c_double * 64),
-                ("rotation", ctypes.c_int)]
+                ("rotation", ctypes.c_int), ("norm_f16", ctypes.c_int)]
 
 ROTATIONS = {"hadamard": 0, "haar": 1}
 
@@ -167,18 +167,25 @@ def unrotate(rot, y) -> np.ndarray:
 
 # ------------------------------------------------------------------- codec
 
+NORM_FORMATS = {"f32": 0, "f16": 1}
+
+
 class Codec:
-    """One codec configuration (head_dim, bits, projections, seed, rotation)
-    on the CPU; rotation is "hadamard" (FWHT with random signs) or "haar"."""
+    """One codec configuration (head_dim, bits, projections, seed, rotation,
+    key-norm format) on the CPU; rotation is "hadamard" (FWHT with random
+    signs) or "haar"; norms is "f32" or "f16" (key rows' n_s and gamma as
+    binary16)."""
 
     def __init__(self, head_dim: int, bits: int, projections: int, seed: int, norm_correct: bool = True,
-                 rotation: str = "hadamard"):
+                 rotation: str = "hadamard", norms: str = "f32"):
         self.d, self.bits, self.m, self.seed = head_dim, bits, projections, seed
         self.rotation = rotation
+        self.norms = norms
         self.cfg = _Cfg()
         if _load().tqo_cfg_init(ctypes.byref(self.cfg), head_dim, bits, projections, int(norm_correct)) != 0:
             raise ValueError("invalid oracle configuration")
         self.cfg.rotation = ROTATIONS[rotation]
+        self.cfg.norm_f16 = NORM_FORMATS[norms]
         self.k_row_bytes = _lib.tqo_k_row_bytes(ctypes.byref(self.cfg))
         self.v_row_bytes = _lib.tqo_v_row_bytes(ctypes.byref(self.cfg))
         self._tables = {}

@@ -66,6 +66,15 @@
  *       n_s (fp32), then gamma (fp32).
  *       V row: B_V-bit index fields, coordinate j at bit B_V*j of a
  *       little-endian bit stream, then n_s (fp32).
+ *   R11 Binary16 key norms (turboquant-plus-rs "Compression formats": turbo4
+ *       at 4.25 bits per value): with norm_f16 set, the K row ends in n_s
+ *       and gamma each rounded to binary16 (ties to even), 2 bytes apiece,
+ *       little-endian, instead of the two fp32 values; the index planes and
+ *       sign bits are those of the fp32 format (computed from the unrounded
+ *       norms), and every consumer reads the rounded norms.  A row whose
+ *       rounded n_s or gamma is infinite (at or above 65520) is stored as the
+ *       degenerate row of R7 and counted with the non-finite rows.  V rows
+ *       keep their fp32 n_s: the row length stays a multiple of 4 bytes.
  */
 #include <math.h>
 #include <stdint.h>
@@ -308,6 +317,7 @@ typedef struct {
     int norm_correct;          /* 1: n_s = n/||yhat|| (R5); 0: n_s = n */
     double ck[TQO_MAXL], bk[TQO_MAXL], cv[TQO_MAXL], bv[TQO_MAXL];
     int rotation;              /* 0: Hadamard (R3), rot = d signs; 1: Haar (R9), rot = Q (d x d) */
+    int norm_f16;              /* 1: K row norms as binary16 (R11); 0: fp32 (R8) */
 } tqo_cfg;
 
 /* Pi x and Pi^T y for the configured rotation; `rot` is the head's signs
@@ -335,7 +345,7 @@ int tqo_cfg_init(tqo_cfg *cfg, int d, int bits, int m, int norm_correct) {
     return 0;
 }
 
-int tqo_k_row_bytes(const tqo_cfg *c) { return c->BK * c->d / 8 + c->m / 8 + 8; }
+int tqo_k_row_bytes(const tqo_cfg *c) { return c->BK * c->d / 8 + c->m / 8 + (c->norm_f16 ? 4 : 8); }
 int tqo_v_row_bytes(const tqo_cfg *c) { return c->BV * c->d / 8 + 4; }
 
 /* ---------------------------------------------------------------- encode -- */
@@ -356,6 +366,37 @@ static double get_f32(const uint8_t *src) {
     memcpy(&f, src, 4);
     return (double)f;
 }
+
+/* Bits of a binary16 value h (a value tqo_round_fp16 returns: finite or
+ * +-inf): sign, 5-bit biased exponent, 10-bit fraction. */
+static uint16_t fp16_bits(double h) {
+    const uint16_t sg = signbit(h) ? 0x8000u : 0u;
+    const double a = fabs(h);
+    if (isinf(a)) return (uint16_t)(sg | 0x7C00u);
+    if (a < 0x1p-14) return (uint16_t)(sg | (uint16_t)(a * 0x1p24));     /* subnormal or zero */
+    int e;
+    frexp(a, &e);                                                       /* a in [2^(e-1), 2^e) */
+    const int ex = e - 1;
+    const uint16_t frac = (uint16_t)(ldexp(a, 10 - ex) - 1024.0);
+    return (uint16_t)(sg | (uint16_t)((ex + 15) << 10) | frac);
+}
+
+static double fp16_value(uint16_t b) {
+    const int ex = (b >> 10) & 31, frac = b & 1023;
+    double v;
+    if (ex == 0) v = ldexp((double)frac, -24);
+    else if (ex == 31) v = frac ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + frac), ex - 25);
+    return (b & 0x8000u) ? -v : v;
+}
+
+static void put_f16(uint8_t *dst, double h) {
+    const uint16_t b = fp16_bits(h);
+    dst[0] = (uint8_t)(b & 0xFFu);
+    dst[1] = (uint8_t)(b >> 8);
+}
+
+static double get_f16(const uint8_t *src) { return fp16_value((uint16_t)(src[0] | (src[1] << 8))); }
 
 /* Encode one row.  is_key selects TurboQuant (K) or MSE-only (V).
  * signs, S[m*d]: the head's tables (signs: the d rotation signs, or Q
@@ -435,6 +476,20 @@ int tqo_encode_row(const tqo_cfg *cfg, int is_key, const double *signs, const do
         }
     }
     (void)B;
+    /* R11: binary16 key norms; a norm that overflows makes the row degenerate */
+    double ns16 = 0.0, gamma16 = 0.0;
+    if (is_key && cfg->norm_f16) {
+        ns16 = tqo_round_fp16(ns);
+        gamma16 = tqo_round_fp16(gamma);
+        if (isinf(ns16) || isinf(gamma16)) {
+            nonfinite = 1;
+            ns = gamma = ns16 = gamma16 = 0.0;
+            for (int j = 0; j < d; ++j) idx[j] = L / 2;
+            for (int i = 0; i < m; ++i) bit[i] = 1;
+            if (z_out) for (int j = 0; j < d; ++j) z_out[j] = HUGE_VAL;
+            if (pn_out) for (int i = 0; i < m; ++i) pn_out[i] = HUGE_VAL;
+        }
+    }
     /* a7: bit packing (R8) */
     if (is_key) {
         const int pb = d / 8;
@@ -444,8 +499,13 @@ int tqo_encode_row(const tqo_cfg *cfg, int is_key, const double *signs, const do
         uint8_t *sg = row + cfg->BK * pb;
         for (int i = 0; i < m; ++i)
             if (bit[i]) sg[i / 8] |= (uint8_t)(1u << (i % 8));
-        put_f32(row + cfg->BK * pb + m / 8, ns);
-        put_f32(row + cfg->BK * pb + m / 8 + 4, gamma);
+        if (cfg->norm_f16) {
+            put_f16(row + cfg->BK * pb + m / 8, ns16);
+            put_f16(row + cfg->BK * pb + m / 8 + 2, gamma16);
+        } else {
+            put_f32(row + cfg->BK * pb + m / 8, ns);
+            put_f32(row + cfg->BK * pb + m / 8 + 4, gamma);
+        }
     } else {
         for (int j = 0; j < d; ++j)
             for (int k = 0; k < cfg->BV; ++k) {
@@ -487,8 +547,13 @@ void tqo_unpack_k(const tqo_cfg *cfg, const uint8_t *row, int *idx, int *bit, do
     }
     const uint8_t *sg = row + cfg->BK * pb;
     for (int i = 0; i < m; ++i) bit[i] = (sg[i / 8] >> (i % 8)) & 1;
-    *ns = get_f32(row + cfg->BK * pb + m / 8);
-    *gamma = get_f32(row + cfg->BK * pb + m / 8 + 4);
+    if (cfg->norm_f16) {
+        *ns = get_f16(row + cfg->BK * pb + m / 8);
+        *gamma = get_f16(row + cfg->BK * pb + m / 8 + 2);
+    } else {
+        *ns = get_f32(row + cfg->BK * pb + m / 8);
+        *gamma = get_f32(row + cfg->BK * pb + m / 8 + 4);
+    }
 }
 
 void tqo_unpack_v(const tqo_cfg *cfg, const uint8_t *row, int *idx, double *ns) {

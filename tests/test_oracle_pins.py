@@ -552,3 +552,67 @@ def test_split_bits_per_value():
         idx_bits = 64 * co.bits + 64 * cn.bits   # value rows: b index bits per coordinate
         assert idx_bits / 128 == b + 0.5
         assert co.v_row_bytes - 4 + cn.v_row_bytes - 4 == (64 * (b + 1) + 64 * b) // 8
+
+
+# -------------------------------------------------- binary16 key norms (R11)
+
+@pytest.mark.parametrize("rotation", ["hadamard", "haar"])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5])
+def test_f16_norm_rows_are_f32_rows_with_ieee_rounded_norms(bits, rotation):
+    """The binary16-norm key row is the fp32-norm row with its tail replaced
+    by n_s and gamma rounded to binary16 by numpy's own IEEE conversion;
+    value rows are unchanged."""
+    rng = np.random.default_rng(bits)
+    x = rng.standard_normal((24, 64)) * rng.uniform(0.01, 300.0, size=(24, 1))
+    a = oracle.Codec(64, bits, 64, 5, rotation=rotation)
+    b = oracle.Codec(64, bits, 64, 5, rotation=rotation, norms="f16")
+    assert b.k_row_bytes == a.k_row_bytes - 4 and b.v_row_bytes == a.v_row_bytes
+    ea, eb = a.encode(x, 1, True), b.encode(x, 1, True)
+    body = a.k_row_bytes - 8
+    assert np.array_equal(ea["rows"][:, :body], eb["rows"][:, :body])
+    tail = eb["rows"][:, body:].copy().view(np.uint16)           # [T, 2] little-endian halves
+    assert np.array_equal(tail[:, 0], ea["ns"].astype(np.float16).view(np.uint16))
+    assert np.array_equal(tail[:, 1], ea["gamma"].astype(np.float16).view(np.uint16))
+    assert np.array_equal(a.encode(x, 1, False)["rows"], b.encode(x, 1, False)["rows"])
+
+
+def test_f16_norm_consumers_read_the_rounded_norms():
+    """Dequantization and scores of binary16-norm rows equal those of the
+    fp32-norm rows whose two norms are overwritten by the binary16-rounded
+    values (exact in fp32)."""
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((16, 128)) * 3.0
+    q = rng.standard_normal(128)
+    a = oracle.Codec(128, 4, 128, 9)
+    b = oracle.Codec(128, 4, 128, 9, norms="f16")
+    ra, rb = a.encode(x, 0, True)["rows"].copy(), b.encode(x, 0, True)["rows"]
+    body = a.k_row_bytes - 8
+    nsg = ra[:, body:].copy().view(np.float32)
+    ra[:, body:] = nsg.astype(np.float16).astype(np.float32).view(np.uint8).reshape(ra.shape[0], 8)
+    assert np.allclose(b.dequant(rb, 0, True), a.dequant(ra, 0, True), rtol=0, atol=1e-13)
+    assert np.allclose(b.scores(q, rb, 0), a.scores(q, ra, 0), rtol=0, atol=1e-12)
+    assert np.allclose(b.scores(q, rb, 0, fused=False), b.scores(q, rb, 0), rtol=0, atol=1e-11)
+
+
+def test_f16_norm_overflow_rows_are_degenerate_and_counted():
+    """A key row whose n_s or gamma rounds to binary16 infinity (>= 65520) is
+    stored as the zero row and counted; just below, it is kept."""
+    rng = np.random.default_rng(6)
+    u = rng.standard_normal(128)
+    u /= np.linalg.norm(u)
+    b = oracle.Codec(128, 3, 128, 2, norms="f16")
+    zero = b.encode(np.zeros((1, 128)), 0, True)["rows"][0]
+    big = b.encode(u[None] * 1e6, 0, True)
+    assert big["nonfinite"] == 1 and np.array_equal(big["rows"][0], zero)
+    ok = b.encode(u[None] * 3e4, 0, True)
+    assert ok["nonfinite"] == 0 and not np.array_equal(ok["rows"][0], zero)
+    idx, bit, ns, g = b.unpack_k(ok["rows"][0])
+    assert ns == float(np.float16(ok["ns"][0])) and np.isfinite(ns)
+
+
+def test_f16_norm_turbo4_key_rate():
+    """Binary16 key norms give the pages' turbo4 rate for keys: 3 index planes
+    + 128 sign bits + 2 x 16 bits over 128 values = 4.25 bits per value
+    (turboquant-plus-rs "Compression formats"); fp32 norms give 4.5."""
+    assert oracle.Codec(128, 4, 128, 0, norms="f16").k_row_bytes * 8 / 128 == 4.25
+    assert oracle.Codec(128, 4, 128, 0).k_row_bytes * 8 / 128 == 4.5
