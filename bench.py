@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha_decode",
                     choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head",
-                             "mha_append", "mha_decode_haar", "mha_split"])
+                             "mha_append", "mha_decode_haar", "mha_split", "mha_decode_f16norms"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -74,6 +74,8 @@ WORKLOAD_DESC = {
                    "(K 2+1, V 3), float32",
     "mha_append": "mha_append: batch 8, 32 query heads over 32 kv heads, 4096 cached tokens + 1 appended per "
                   "(sequence, kv head), d128, m128, bits 4 (K 3+1, V 4), float16",
+    "mha_decode_f16norms": "mha_decode_f16norms: the mha_decode workload (batch 8, 32 heads, 4096 tokens, d128, "
+                           "fp16, bits 4, m128) with binary16 key norms (68-byte key rows, 4.25 bits per key value)",
     "mha_decode_haar": "mha_decode_haar: the mha_decode workload with the Haar-QR rotation (batch 8, 32 heads, "
                        "4096 tokens, d128, m128, bits 4, float16)",
     "mha_split": "mha_split: the mha_decode data (batch 8, 32 heads, 4096 tokens, d128, fp16) split per head into "
@@ -83,7 +85,8 @@ WORKLOAD_DESC = {
 
 
 STEP_DESC = {w: "encode all K/V rows + one decode step per query head"
-             for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head", "mha_decode_haar")}
+             for w in ("mha_decode", "gqa_decode", "shared_prefix", "single_head", "mha_decode_haar",
+                       "mha_decode_f16norms")}
 STEP_DESC["bulk_encode"] = "encode all K/V rows of 32 layers"
 STEP_DESC["mha_append"] = "append one token per (sequence, kv head) + one decode step per query head"
 STEP_DESC["mha_split"] = "encode both channel groups of all K/V rows + one split decode step per query head"
@@ -121,8 +124,8 @@ def measured_traffic(piece, workload):
     return nbytes if cur == sha else None
 
 
-def row_bytes(bits):
-    return (bits - 1) * D // 8 + M // 8 + 8, bits * D // 8 + 4
+def row_bytes(bits, norms="f32"):
+    return (bits - 1) * D // 8 + M // 8 + (4 if norms == "f16" else 8), bits * D // 8 + 4
 
 
 # ------------------------------------------------------------------ workloads
@@ -139,8 +142,8 @@ class Workload:
         from kv_cache_vector_10_b200 import workloads as W
         self.name, self.tq, self.torch = name, tq, torch
         seed_shift = 1000 * rank
-        if name in ("mha_decode", "gqa_decode", "single_head", "mha_append", "mha_decode_haar"):
-            if name in ("mha_decode", "mha_append", "mha_decode_haar"):
+        if name in ("mha_decode", "gqa_decode", "single_head", "mha_append", "mha_decode_haar", "mha_decode_f16norms"):
+            if name in ("mha_decode", "mha_append", "mha_decode_haar", "mha_decode_f16norms"):
                 w = W.mha_decode(device=device, data_seed=2 + seed_shift,
                                  n_tokens=4097 if name == "mha_append" else 4096)
             elif name == "gqa_decode":
@@ -151,10 +154,12 @@ class Workload:
             B, Hkv, T, _ = w["k"].shape
             Hq = w["q"].shape[1]
             bits = w["bits"]
-            kr, vr = row_bytes(bits)
+            norms = "f16" if name == "mha_decode_f16norms" else "f32"
+            kr, vr = row_bytes(bits, norms)
             es = w["k"].element_size()
             qb = B * Hq * D * 2 * w["q"].element_size()          # query in + output out
-            self.codec = tq.Codec(D, bits, M, w["seed"], rotation="haar" if name == "mha_decode_haar" else "hadamard")
+            self.codec = tq.Codec(D, bits, M, w["seed"], rotation="haar" if name == "mha_decode_haar" else "hadamard",
+                                  norms=norms)
             self.B, self.Hq, self.Hkv = B, Hq, Hkv
             if name == "mha_append":
                 T -= 1                                            # history; row T is the step's new row
@@ -424,7 +429,7 @@ def oracle_unit(wl_name, rank_seed=0):
                          [(oc, 0, np.concatenate([ek["rows"], nk["rows"]]), np.concatenate([ev["rows"], nv["rows"]]))])
         dt = time.perf_counter() - t0
         return dt, 1025, "tokens", "1 kv head x 1 query head: append 1 token to 1024 + decode over 1025"
-    if wl_name in ("mha_decode", "mha_decode_haar"):
+    if wl_name in ("mha_decode", "mha_decode_haar", "mha_decode_f16norms"):
         w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024)
         G = 1
     elif wl_name == "gqa_decode":
@@ -433,7 +438,8 @@ def oracle_unit(wl_name, rank_seed=0):
     else:
         w = W.single_head(device="cpu")
         G = 4
-    oc = oracle.Codec(D, w["bits"], M, w["seed"], rotation="haar" if wl_name == "mha_decode_haar" else "hadamard")
+    oc = oracle.Codec(D, w["bits"], M, w["seed"], rotation="haar" if wl_name == "mha_decode_haar" else "hadamard",
+                      norms="f16" if wl_name == "mha_decode_f16norms" else "f32")
     T = w["k"].shape[2]
     t0 = time.perf_counter()
     ek = oc.encode(w["k"][0, 0].double().numpy(), 0, True)

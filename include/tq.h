@@ -37,6 +37,9 @@
  *    coordinate j at byte j/8, bit j%8), then the m-bit QJL sign plane
  *    (projection i at byte i/8, bit i%8; 1 = non-negative), then n_s
  *    (float32, the corrected norm), then gamma (float32, the residual norm).
+ *    With binary16 key norms (tq_create_format, TQ_NORMS_F16) the tail is
+ *    one 32-bit word instead: n_s and gamma rounded to binary16 (ties to
+ *    even), n_s in the low half; k_row_bytes = B_K*d/8 + m/8 + 4.
  *  V row (v_row_bytes = B_V*d/8 + 4):
  *    B_V-bit index fields, coordinate j at bit B_V*j of a little-endian bit
  *    stream, then n_s (float32).
@@ -75,6 +78,14 @@ typedef enum tq_which { TQ_KEYS = 0, TQ_VALUES = 1, TQ_BOTH = 2 } tq_which;
 
 /* The random rotation Pi (turboquant-plus-rs README, Architecture: "random
  * rotation (Haar-distributed or fast Walsh-Hadamard)"; Modules: rotation). */
+/* Storage of the two key-row norms (turboquant-plus-rs README,
+ * "Compression formats": turbo4 is 4.25 bits per value, which binary16
+ * norms give a key row at b = 4, d = m = 128). */
+typedef enum tq_norm_format {
+    TQ_NORMS_F32 = 0,      /* n_s, gamma as float32 (8 bytes) */
+    TQ_NORMS_F16 = 1       /* n_s, gamma as binary16 in one 32-bit word */
+} tq_norm_format;
+
 typedef enum tq_rotation {
     TQ_ROT_HADAMARD = 0,   /* Pi = H D / sqrt(d): Sylvester Walsh-Hadamard, random signs D */
     TQ_ROT_HAAR = 1        /* Pi = Q: orthogonal factor of the QR of a d x d Gaussian matrix,
@@ -137,6 +148,17 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
  * Returns TQ_ERR_DIM for an unknown rotation. */
 tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
                        tq_ctx **out);
+
+/* tq_create_ex with a choice of key-norm storage.  TQ_NORMS_F32 is
+ * tq_create_ex.  TQ_NORMS_F16: key rows store n_s and gamma rounded to
+ * binary16 (ties to even) in one 32-bit word; indices and sign bits are
+ * those of the float32 format, and scores, dequantization and decode read
+ * the rounded norms.  A key row whose n_s or gamma rounds to binary16
+ * infinity (>= 65520) is stored as a zero row and counted with the
+ * non-finite rows (tq_get_status).  Value rows keep their float32 n_s.
+ * Returns TQ_ERR_DIM for an unknown rotation or norm format. */
+tq_status tq_create_format(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
+                           tq_norm_format key_norms, tq_ctx **out);
 
 /* Release a context and its device tables (synchronizes the device). NULL is a no-op. */
 void tq_destroy(tq_ctx *ctx);

@@ -26,6 +26,8 @@ TQ_F32, TQ_F16, TQ_BF16 = 0, 1, 2
 TQ_KEYS, TQ_VALUES, TQ_BOTH = 0, 1, 2
 TQ_ROT_HADAMARD, TQ_ROT_HAAR = 0, 1
 ROTATIONS = {"hadamard": TQ_ROT_HADAMARD, "haar": TQ_ROT_HAAR}
+TQ_NORMS_F32, TQ_NORMS_F16 = 0, 1
+NORM_FORMATS = {"f32": TQ_NORMS_F32, "f16": TQ_NORMS_F16}
 TQ_MAX_SEGMENTS = 64
 
 STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_DIM", 4: "TQ_ERR_BITS",
@@ -33,7 +35,7 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
                 9: "TQ_ERR_WORKSPACE", 10: "TQ_ERR_ALIGN", 11: "TQ_ERR_CUDA", 12: "TQ_ERR_DEVICE",
                 13: "TQ_ERR_LIMIT"}
 
-EXPORTED = ["tq_create", "tq_create_ex", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
+EXPORTED = ["tq_create", "tq_create_ex", "tq_create_format", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
             "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
             "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes",
@@ -68,6 +70,7 @@ def _load():
     sig = {
         "tq_create": (I, [I, I, I, U64, ctypes.POINTER(V)]),
         "tq_create_ex": (I, [I, I, I, U64, I, ctypes.POINTER(V)]),
+        "tq_create_format": (I, [I, I, I, U64, I, I, ctypes.POINTER(V)]),
         "tq_destroy": (None, [V]),
         "tq_ensure_heads": (I, [V, I]),
         "tq_row_bytes": (I64, [V, I]),
@@ -129,6 +132,13 @@ def tq_create_ex(head_dim: int, bits: int, projections: int, seed: int, rotation
     out = ctypes.c_void_p()
     _check(_lib.tq_create_ex(head_dim, bits, projections, seed & 0xFFFFFFFFFFFFFFFF, rotation, ctypes.byref(out)),
            "tq_create_ex")
+    return out.value
+
+
+def tq_create_format(head_dim: int, bits: int, projections: int, seed: int, rotation: int, key_norms: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.tq_create_format(head_dim, bits, projections, seed & 0xFFFFFFFFFFFFFFFF, rotation, key_norms,
+                                 ctypes.byref(out)), "tq_create_format")
     return out.value
 
 
@@ -246,13 +256,16 @@ def tq_reset_status(ctx: int, stream=None):
 # -------------------------------------------------------------- conveniences
 
 class Codec:
-    """A codec context: KvCacheConfig {head_dim, bits, projections, seed}, and
-    the rotation ("hadamard": FWHT with random signs; "haar": QR rotation)."""
+    """A codec context: KvCacheConfig {head_dim, bits, projections, seed}, the
+    rotation ("hadamard": FWHT with random signs; "haar": QR rotation) and the
+    key-norm storage ("f32", or "f16": n_s and gamma as binary16)."""
 
-    def __init__(self, head_dim: int, bits: int, projections: int, seed: int, rotation: str = "hadamard"):
+    def __init__(self, head_dim: int, bits: int, projections: int, seed: int, rotation: str = "hadamard",
+                 norms: str = "f32"):
         self.head_dim, self.bits, self.projections, self.seed = head_dim, bits, projections, seed
         self.rotation = rotation
-        self.ctx = tq_create_ex(head_dim, bits, projections, seed, ROTATIONS[rotation])
+        self.norms = norms
+        self.ctx = tq_create_format(head_dim, bits, projections, seed, ROTATIONS[rotation], NORM_FORMATS[norms])
         self.k_row_bytes = tq_row_bytes(self.ctx, TQ_KEYS)
         self.v_row_bytes = tq_row_bytes(self.ctx, TQ_VALUES)
 

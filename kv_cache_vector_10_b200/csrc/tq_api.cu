@@ -107,8 +107,14 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
 
 tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
                        tq_ctx **out) {
+    return tq_create_format(head_dim, bits, projections, seed, rotation, TQ_NORMS_F32, out);
+}
+
+tq_status tq_create_format(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
+                           tq_norm_format key_norms, tq_ctx **out) {
     if (!out) return TQ_ERR_NULL;
-    if (rotation != TQ_ROT_HADAMARD && rotation != TQ_ROT_HAAR) {
+    if ((rotation != TQ_ROT_HADAMARD && rotation != TQ_ROT_HAAR) ||
+        (key_norms != TQ_NORMS_F32 && key_norms != TQ_NORMS_F16)) {
         *out = nullptr;
         return TQ_ERR_DIM;
     }
@@ -133,6 +139,7 @@ tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, t
     c->seed = seed;
     c->device = dev;
     c->rotation = (int)rotation;
+    c->norm_f16 = key_norms == TQ_NORMS_F16 ? 1 : 0;
     c->LK = tq_host_codebook(c->BK, c->ck, c->bk);
     c->LV = tq_host_codebook(c->BV, c->cv, c->bv);
     TqBook book;
@@ -265,7 +272,7 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
 
 int64_t tq_row_bytes(const tq_ctx *ctx, tq_which which) {
     if (!ctx) return 0;
-    const int64_t kb = (int64_t)ctx->BK * ctx->d / 8 + ctx->m / 8 + 8;
+    const int64_t kb = (int64_t)ctx->BK * ctx->d / 8 + ctx->m / 8 + (ctx->norm_f16 ? 4 : 8);
     const int64_t vb = (int64_t)ctx->BV * ctx->d / 8 + 4;
     return which == TQ_KEYS ? kb : which == TQ_VALUES ? vb : kb + vb;
 }

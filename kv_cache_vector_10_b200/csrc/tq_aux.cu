@@ -114,6 +114,7 @@ struct ScoresParams {
     const float *Q;            // Haar rotation, or nullptr
     int64_t capacity, T;
     int Hq, Hkv, M, krow, bk;
+    int kf16;                  // key norms as binary16
     float ck[16];
 };
 
@@ -161,9 +162,8 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_con
 #pragma unroll 8
             for (int i = 0; i < 32; ++i) bq += ((sw >> i) & 1u) ? s_sq[wd * 32 + i] : -s_sq[wd * 32 + i];
         }
-        const float ns = __uint_as_float(sg[p.M / 32]);
-        const float gamma = __uint_as_float(sg[p.M / 32 + 1]);
-        p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (ns * a * isd + cq * gamma * bq) * isd;
+        const float2 nrm = tqdev::key_norms(sg + p.M / 32, p.kf16 != 0);
+        p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (nrm.x * a * isd + cq * nrm.y * bq) * isd;
     }
 }
 
@@ -177,6 +177,7 @@ struct DequantParams {
     const float *Q;            // Haar rotation, or nullptr
     int64_t capacity, T;
     int H, M, krow, vrow, bk, bv;
+    int kf16;                  // key norms as binary16
     float ck[16];
     float cv[32];
 };
@@ -253,9 +254,9 @@ __global__ void __launch_bounds__(AUX_THREADS) tq_dequant_kernel(const __grid_co
     if (p.kh) {
         const uint32_t *w = reinterpret_cast<const uint32_t *>(p.kc + rowi * p.krow);
         const uint32_t *sgn = w + p.bk * (D / 32);
-        const float ns = __uint_as_float(sgn[p.M / 32]);
-        const float gamma = __uint_as_float(sgn[p.M / 32 + 1]);
-        const float cq = 1.2533141373155003f / (float)p.M * gamma;
+        const float2 nrm = tqdev::key_norms(sgn + p.M / 32, p.kf16 != 0);
+        const float ns = nrm.x;
+        const float cq = 1.2533141373155003f / (float)p.M * nrm.y;
         float x[D];
 #pragma unroll
         for (int j = 0; j < D; ++j) {
@@ -376,10 +377,21 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
         const float e = tid < D && !degenerate ? u - ns * (u < 0.f ? -cm : cm) : 0.f;
         if (tid < D) s_e[tid] = e;
         const float e2 = block_sum(e * e, s_red);   // its barriers publish s_e
+        const float gv = degenerate ? 0.f : sqrtf(e2 * (1.f / D));
+        // binary16 norms: a row whose norms overflow is the zero row, counted
+        // with the non-finite rows (ns and e2 are block-wide, so is this)
+        bool zero_row = degenerate;
+        uint32_t nw = 0u;
+        if (g.kf16 && !tqdev::pack_norms_f16(ns, gv, nw)) {
+            zero_row = true;
+            nw = 0u;
+            if (tid == 0) atomicAdd(&g.status[0], 1ull);
+        }
+        const uint32_t kidx = zero_row ? (uint32_t)HB : idx;
         // index bit planes: warp w holds coordinates [32w, 32w + 32)
 #pragma unroll 1
         for (int q = 0; q < B; ++q) {
-            const uint32_t w = __ballot_sync(0xffffffffu, (idx >> q) & 1u);
+            const uint32_t w = __ballot_sync(0xffffffffu, (kidx >> q) & 1u);
             if (lane == 0 && tid < D) row[q * (D / 32) + warp] = w;
         }
         // QJL signs: projection i on thread i (and i + blockDim.x, ...)
@@ -403,12 +415,16 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
                 }
             }
             const uint32_t w = __ballot_sync(0xffffffffu, p >= 0.f);
-            if (lane == 0 && i0 + 32 * warp < g.m) row[sw0 + (i0 + 32 * warp) / 32] = degenerate ? ~0u : w;
+            if (lane == 0 && i0 + 32 * warp < g.m) row[sw0 + (i0 + 32 * warp) / 32] = zero_row ? ~0u : w;
         }
         if (tid == 0) {
             const int tail = sw0 + g.m / 32;
-            row[tail] = __float_as_uint(ns);
-            row[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)));
+            if (g.kf16) {
+                row[tail] = nw;
+            } else {
+                row[tail] = __float_as_uint(ns);
+                row[tail + 1] = __float_as_uint(gv);
+            }
         }
     } else {
         if (tid < D) s_idx[tid] = (uint8_t)idx;
@@ -538,6 +554,7 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
     p.M = ctx->m;
     p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
     p.bk = ctx->BK;
+    p.kf16 = ctx->norm_f16;
     for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
     const int64_t per_block = (int64_t)AUX_THREADS * SCORE_TPT;
     dim3 grid((unsigned)((T + per_block - 1) / per_block), (unsigned)Hq, (unsigned)codes->batch);
@@ -564,6 +581,7 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
     p.vrow = (int)tq_row_bytes(ctx, TQ_VALUES);
     p.bk = ctx->BK;
     p.bv = ctx->BV;
+    p.kf16 = ctx->norm_f16;
     for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
     for (int i = 0; i < ctx->LV; ++i) p.cv[i] = ctx->cv[i];
     dim3 grid((unsigned)((T + AUX_THREADS - 1) / AUX_THREADS), (unsigned)codes->n_kv_heads, (unsigned)codes->batch);

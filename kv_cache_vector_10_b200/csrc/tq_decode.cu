@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int h = (int)(local / ((int64_t)g.n_qchunks * g.n_splits));
     const int M = MT > 0 ? MT : g.m;
     const int NGS = M / 8, RS = (NGS + 15) / 16;
-    const int krow = MT > 0 ? BK * D / 8 + MT / 8 + 8 : g.krow;
+    const int krow = MT > 0 ? BK * D / 8 + MT / 8 + (g.kf16 ? 4 : 8) : g.krow;
     const int vrow = MT > 0 ? BV * D / 8 + 4 : g.vrow;
     const int64_t t_begin = (int64_t)split * g.split_len;
     const int64_t t_end = std::min<int64_t>(g.T, t_begin + g.split_len);
@@ -220,6 +220,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const float cqs = 1.2533141373155003f / (float)M * rsqrtf((float)D);   // sqrt(pi/2)/m/sqrt(d)
     const int off_sign = BK * (D / 8);
     const int off_ns = off_sign + M / 8;
+    const bool kf16 = g.kf16 != 0;
     const int voff_ns = BV * D / 8;
     // value bits of this lane's 8 coordinates: [8*BV*slot, 8*BV*slot + 8*BV)
     const int vbit = 8 * BV * slot;
@@ -285,9 +286,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                     for (int qq = 0; qq < QC; ++qq) as[qq] += Vec<QC>::get(e, qq);
                 }
             }
-            const float ns = *reinterpret_cast<const float *>(kr + off_ns);
-            const float gm = *reinterpret_cast<const float *>(kr + off_ns + 4);
-            const float a1 = ns * inv_d, a2 = gm * cqs;
+            const float2 nrm = tqdev::key_norms(reinterpret_cast<const uint32_t *>(kr + off_ns), kf16);
+            const float a1 = nrm.x * inv_d, a2 = nrm.y * cqs;
 #pragma unroll
             for (int qq = 0; qq < QC; ++qq) part[qq][st] = fmaf(a1, am[qq], a2 * as[qq]);
         }
@@ -645,6 +645,7 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         d.first_seq = sg.first_seq;
         d.n_seqs = sg.n_seqs;
         d.krow = (int)krow;
+        d.kf16 = c->norm_f16;
         d.vrow = (int)vrow;
         d.m = c->m;
         d.bk = c->BK;
@@ -666,15 +667,19 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
     }
     cudaError_t e = tq_launch_qprep(P, q, q_dtype, stream);
     if (e != cudaSuccess) return tq_check_cuda(e);
-    // one launch per (bits, queries per CTA) group
+    // one launch per (bits, queries per CTA, row format) group: the CTA's
+    // shared memory is sized by the group's row lengths
     std::vector<int> done(n_segs, 0);
     for (int s0 = 0; s0 < n_segs; ++s0) {
         if (done[s0]) continue;
-        const int bk = P.seg[s0].bk, qc = pl[s0].qc, m = P.seg[s0].m;
+        const int bk = P.seg[s0].bk, qc = pl[s0].qc, m = P.seg[s0].m, kr = P.seg[s0].krow;
+        auto same = [&](int s) {
+            return P.seg[s].bk == bk && pl[s].qc == qc && P.seg[s].m == m && P.seg[s].krow == kr;
+        };
         int64_t items = 0;
         for (int s = 0; s < n_segs; ++s) {
             SegDesc &d = P.seg[s];
-            if (!done[s] && d.bk == bk && pl[s].qc == qc && d.m == m) {
+            if (!done[s] && same(s)) {
                 d.item_base = items;
                 items += (int64_t)Hkv * d.n_splits * d.n_qchunks;
             } else if (!done[s]) {
@@ -685,7 +690,7 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         for (int s = 0; s < n_segs; ++s)
             if (done[s]) Pg.seg[s].item_base = -(int64_t)1 << 62;
         for (int s = 0; s < n_segs; ++s)
-            if (!done[s] && P.seg[s].bk == bk && pl[s].qc == qc && P.seg[s].m == m) done[s] = 1;
+            if (!done[s] && same(s)) done[s] = 1;
         if (items == 0) continue;
         e = P.d == 128 ? launch_decode_dim<128>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
                        : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);

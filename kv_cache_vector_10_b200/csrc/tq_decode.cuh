@@ -28,6 +28,7 @@ struct SegDesc {
     int n_splits, split_len, n_qchunks;
     int n_planes;              // odd subsets of the key index bits
     int append;                // 1: this step's new key/value rows go to row T-1
+    int kf16;                  // 1: key norms as binary16 (one word)
     uint32_t plane_sets[8];    // bit mask of index planes XOR-ed into sigma-plane s
     float alpha[8];            // Walsh coefficient of sigma-plane s
     float vtab[32];            // value centroids, indexed by code

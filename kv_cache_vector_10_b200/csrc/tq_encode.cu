@@ -65,6 +65,7 @@ struct EncodeParams {
     float mag[16];          // positive-half centroid magnitudes
     float pb[16];           // positive boundaries
     float cl[8];            // keys: centroid magnitude as a multilinear form in the search bits
+    int norm_f16;           // keys: n_s and gamma as binary16 in one word
 };
 
 // ------------------------------------------------------------- row loading
@@ -991,10 +992,31 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
             }
         }
         const float e2 = e2p.x + e2p.y;
-        if (valid) {
+        bool zero_row = degenerate;
+        {
             const int tail = BK * NC + M / 32;
-            dst[tail] = __float_as_uint(ns * inv_scale);
-            dst[tail + 1] = __float_as_uint(degenerate ? 0.f : sqrtf(e2 * (1.f / D)) * inv_scale);
+            const float nsv = ns * inv_scale, gv = degenerate ? 0.f : sqrtf(e2 * (1.f / D)) * inv_scale;
+            if (p.norm_f16) {
+                uint32_t w;
+                if (!tqdev::pack_norms_f16(nsv, gv, w)) {
+                    // binary16 overflow: the zero row, counted with the non-finite rows
+                    zero_row = true;
+                    w = 0u;
+                    if (valid) {
+                        atomicAdd(&p.status[0], 1ull);
+#pragma unroll 1
+                        for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                            for (int q = 0; q < BK - 1; ++q) dst[q * NC + c] = ((HK >> q) & 1) ? ~0u : 0u;
+                            dst[(BK - 1) * NC + c] = ~0u;
+                        }
+                    }
+                }
+                if (valid) dst[tail] = w;
+            } else if (valid) {
+                dst[tail] = __float_as_uint(nsv);
+                dst[tail + 1] = __float_as_uint(gv);
+            }
         }
         // E: the QJL projection on the tensor cores (TMEM columns [d, d + m));
         // an abort flag set by any thread ends the loop here, for all threads
@@ -1056,7 +1078,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 neg = push_sign(neg, q.y);
                 neg = push_sign(neg, q.x);
             }
-            if (valid) sdst[c] = degenerate ? ~0u : ~neg;
+            if (valid) sdst[c] = zero_row ? ~0u : ~neg;
         }
         n2 = n2_next;
     }
@@ -1167,6 +1189,7 @@ tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype d
         p.blocks_per_bh = blocks_per_bh;
         p.signs = ctx->d_signs;
         p.status = ctx->d_status;
+        p.norm_f16 = ctx->norm_f16;
         const int B = keys ? ctx->BK : ctx->BV;
         const float *cb = keys ? ctx->ck : ctx->cv;
         const float *bd = keys ? ctx->bk : ctx->bv;

@@ -31,6 +31,7 @@ struct tq_ctx {
     float ck[TQ_MAX_LEVELS], bk[TQ_MAX_LEVELS], cv[TQ_MAX_LEVELS], bv[TQ_MAX_LEVELS];
     struct TqBook *d_book;          // device copy of the positive halves (TqBook)
     int rotation;                   // tq_rotation
+    int norm_f16;                   // 1: key rows end in n_s, gamma as binary16 (tq_norm_format)
     // Haar rotation tables (rotation == TQ_ROT_HAAR): Q [heads][d][d] fp32,
     // and sqrt(d) Q as binary16 hi + lo [heads][2][d][d] with its TMA map
     // (inner d, outer heads*2*d rows, box 64 x d, 128-byte swizzle).
@@ -269,6 +270,24 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 
 // Instruction descriptor: kind::f16, A and B binary16, K-major, fp32
 // accumulator, M = 128, N = n.
+// Key-row norms.  Binary16 format: n_s and gamma rounded to binary16 (ties
+// to even) in one 32-bit word, n_s in the low half; pack returns false if
+// either rounds to infinity (the row is then stored as a zero row).
+__device__ __forceinline__ bool pack_norms_f16(float ns, float g, uint32_t &w) {
+    const __half hn = __float2half_rn(ns), hg = __float2half_rn(g);
+    w = (uint32_t)__half_as_ushort(hn) | ((uint32_t)__half_as_ushort(hg) << 16);
+    return !(__hisinf(hn) || __hisinf(hg));
+}
+// (n_s, gamma) from a key row's tail words.
+__device__ __forceinline__ float2 key_norms(const uint32_t *tail, bool f16) {
+    if (f16) {
+        const uint32_t w = tail[0];
+        return make_float2(__half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))),
+                           __half2float(__ushort_as_half((unsigned short)(w >> 16))));
+    }
+    return make_float2(__uint_as_float(tail[0]), __uint_as_float(tail[1]));
+}
+
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }

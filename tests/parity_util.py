@@ -19,8 +19,9 @@ REL = 1e-4           # dequantized vectors, scores, stored norms
 ATTN_ABS = 2e-3      # attention outputs
 
 
-def unpack_k(rows: np.ndarray, d: int, bk: int, m: int):
-    """rows [N, k_row_bytes] uint8 -> idx [N, d], bits [N, m], ns [N], gamma [N]."""
+def unpack_k(rows: np.ndarray, d: int, bk: int, m: int, norms: str = "f32"):
+    """rows [N, k_row_bytes] uint8 -> idx [N, d], bits [N, m], ns [N], gamma [N].
+    norms "f16": the tail is n_s, gamma as binary16 (one 32-bit word)."""
     rows = np.ascontiguousarray(rows)
     N = rows.shape[0]
     pb = d // 8
@@ -29,8 +30,18 @@ def unpack_k(rows: np.ndarray, d: int, bk: int, m: int):
     for p in range(bk):
         idx |= bits[:, p * d:(p + 1) * d].astype(np.int64) << p
     sg = bits[:, bk * d: bk * d + m].astype(np.int64)
-    tail = rows[:, bk * pb + m // 8: bk * pb + m // 8 + 8].copy().view(np.float32)
+    nb = 4 if norms == "f16" else 8
+    tail = rows[:, bk * pb + m // 8: bk * pb + m // 8 + nb].copy().view(np.float16 if norms == "f16" else np.float32)
     return idx, sg, tail[:, 0].astype(np.float64), tail[:, 1].astype(np.float64)
+
+
+def norm_slack(ref: np.ndarray, norms: str) -> np.ndarray:
+    """Extra tolerance of a stored norm: one binary16 step at the oracle's
+    value when norms are binary16 (the kernel rounds its fp32 norm, the
+    oracle its fp64 norm), else 0."""
+    if norms != "f16":
+        return np.zeros_like(ref)
+    return np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
 
 
 def unpack_v(rows: np.ndarray, d: int, bv: int):
@@ -53,8 +64,9 @@ def _near_boundary(z: np.ndarray, beta: np.ndarray) -> np.ndarray:
 def compare_k(gpu_rows, ora, codec: oracle.Codec, report: dict):
     """Compare packed key rows.  ora: dict from Codec.encode(..., is_key=True)."""
     d, m, bk = codec.d, codec.m, codec.bits - 1
-    gi, gb, gns, gg = unpack_k(gpu_rows, d, bk, m)
-    oi, ob, ons, og = unpack_k(ora["rows"], d, bk, m)
+    norms = getattr(codec, "norms", "f32")
+    gi, gb, gns, gg = unpack_k(gpu_rows, d, bk, m, norms)
+    oi, ob, ons, og = unpack_k(ora["rows"], d, bk, m, norms)
     near = _near_boundary(ora["z"], codec.bk)
     bad_idx = (gi != oi) & ~near
     assert not bad_idx.any(), f"key index mismatch outside the boundary band at rows {np.nonzero(bad_idx.any(1))[0][:10]}"
@@ -69,8 +81,10 @@ def compare_k(gpu_rows, ora, codec: oracle.Codec, report: dict):
     report["k_sign_flips"] = report.get("k_sign_flips", 0) + int(((gb != ob) & ok_rows[:, None]).sum())
     report["k_rows_flipped"] = report.get("k_rows_flipped", 0) + int(flipped.sum())
     nf = ~flipped
-    assert np.all(np.abs(gns[nf] - ons[nf]) <= REL * np.abs(ons[nf]) + 1e-30), "n_s mismatch"
-    assert np.all(np.abs(gg[nf] - og[nf]) <= REL * np.maximum(np.abs(og[nf]), 1e-3 * ons[nf]) + 1e-30), "gamma mismatch"
+    assert np.all(np.abs(gns[nf] - ons[nf]) <= REL * np.abs(ons[nf]) + norm_slack(ons[nf], norms) + 1e-30), \
+        "n_s mismatch"
+    assert np.all(np.abs(gg[nf] - og[nf]) <= REL * np.maximum(np.abs(og[nf]), 1e-3 * ons[nf]) +
+                  norm_slack(og[nf], norms) + 1e-30), "gamma mismatch"
     return report
 
 
