@@ -99,14 +99,14 @@ def arm_config(workload):
 
 
 # DRAM traffic of a piece's main kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum of one launch, ncu --set full, caches flushed before
+# dram__bytes_write.sum of one launch, one ncu capture, caches flushed before
 # the launch), keyed by (piece, workload), with the SHA-1 of the source file
 # holding that kernel when the counters were taken: once the source changes
 # the entry no longer applies (traffic: null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): ("tq_encode.cu", "0090ee5f532343ec656f1565a641d05b552cea39", 326150912),
-    ("encode_values", "mha_decode"): ("tq_encode.cu", "0090ee5f532343ec656f1565a641d05b552cea39", 320644352),
-    ("decode", "mha_decode"): ("tq_decode.cu", "420aa8ed6238705ffaaea7f0431d3414d93fcb44", 151321344),
+    ("encode_keys", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 327339776),
+    ("encode_values", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 320737792),
+    ("decode", "mha_decode"): ("tq_decode.cu", "f344464501af8ebb494252e10449a289bb4ca771", 151534848),
 }
 
 

@@ -94,8 +94,10 @@ __host__ __device__ constexpr int vpair_copies() { return BV <= 4 ? 16 : 1; }
 template <int BV>
 __host__ __device__ constexpr int vpair_entries() { return 1 << (2 * BV); }
 
-// MT = number of QJL projections when known at compile time (128), else 0.
-template <int D, int BK, int BV, int QC, int MT>
+// MT = number of QJL projections when known at compile time (128), else 0;
+// KF = key norms as binary16 (1) or fp32 (0) when MT > 0 (else read from the
+// segment).
+template <int D, int BK, int BV, int QC, int MT, int KF>
 __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const __grid_constant__ DecodePlan P) {
     using VT = typename Vec<QC>::T;
     constexpr int NGK = D / 8;                    // byte groups of an index plane = value slots
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int h = (int)(local / ((int64_t)g.n_qchunks * g.n_splits));
     const int M = MT > 0 ? MT : g.m;
     const int NGS = M / 8, RS = (NGS + 15) / 16;
-    const int krow = MT > 0 ? BK * D / 8 + MT / 8 + (g.kf16 ? 4 : 8) : g.krow;
+    const int krow = MT > 0 ? BK * D / 8 + MT / 8 + (KF ? 4 : 8) : g.krow;
     const int vrow = MT > 0 ? BV * D / 8 + 4 : g.vrow;
     const int64_t t_begin = (int64_t)split * g.split_len;
     const int64_t t_end = std::min<int64_t>(g.T, t_begin + g.split_len);
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const float cqs = 1.2533141373155003f / (float)M * rsqrtf((float)D);   // sqrt(pi/2)/m/sqrt(d)
     const int off_sign = BK * (D / 8);
     const int off_ns = off_sign + M / 8;
-    const bool kf16 = g.kf16 != 0;
+    const bool kf16 = MT > 0 ? KF != 0 : g.kf16 != 0;
     const int voff_ns = BV * D / 8;
     // value bits of this lane's 8 coordinates: [8*BV*slot, 8*BV*slot + 8*BV)
     const int vbit = 8 * BV * slot;
@@ -541,7 +543,11 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
 template <int D, int BK, int BV, int QC>
 cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vrow, int M, cudaStream_t stream) {
     const size_t smem = decode_smem_bytes(D, BV, QC, krow, vrow, M);
-    auto kern = M == 128 ? tq_decode_kernel<D, BK, BV, QC, 128> : tq_decode_kernel<D, BK, BV, QC, 0>;
+    // the launch's segments share one key-row length, hence one norm format
+    const bool kf16 = krow == BK * D / 8 + M / 8 + 4;
+    auto kern = M != 128 ? tq_decode_kernel<D, BK, BV, QC, 0, 0>
+                : kf16   ? tq_decode_kernel<D, BK, BV, QC, 128, 1>
+                         : tq_decode_kernel<D, BK, BV, QC, 128, 0>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
         cudaGetLastError();   // do not leave the failure as the thread's sticky last error
