@@ -15,7 +15,8 @@
 // query head, chunk of tokens) combines the scores, takes the chunk's softmax
 // terms and accumulates each group's values in its rotated frame from the
 // packed codes (128-token tiles of probabilities and of both groups' value
-// rows staged in shared memory by coalesced copies); a last kernel merges the
+// rows staged in shared memory, the next tile's rows copied with cp.async
+// while the current one is accumulated); a last kernel merges the
 // chunks by their maxima and sums (log-sum-exp) and rotates each group back.
 #include <cmath>
 
@@ -28,7 +29,6 @@ tq_status tq_check_cuda(cudaError_t e);
 namespace {
 
 constexpr int SPLIT_TILE = 128;    // tokens per pass: probabilities and both groups' value rows in smem
-constexpr int SPLIT_VROW_MAX = 5 * 128 / 8 + 4;   // largest value row (5 bits, d = 128)
 
 struct SplitGroup {
     const uint8_t *vc;        // packed value rows [batch][H_kv][capacity][vrow]
@@ -72,7 +72,7 @@ __global__ void tq_split_q_kernel(const __grid_constant__ SplitParams P) {
     }
 }
 
-constexpr int SPLIT_SLICES = 4;      // token slices per coordinate in a block
+constexpr int SPLIT_SLICES = 8;      // token slices per coordinate pair in a block
 constexpr int SPLIT_TARGET_BLOCKS = 1184;   // 8 blocks per SM of 148
 
 // Tokens per chunk: a multiple of SPLIT_TILE, chosen so that (rows x chunks)
@@ -86,22 +86,40 @@ int64_t split_chunk_len(int rows, int64_t T) {
     return per * SPLIT_TILE;
 }
 
+// Both groups' value rows of a tile, [group 0 rows][group 1 rows], copied
+// with 4-byte cp.async by all threads (one commit group per tile).
+__device__ __forceinline__ void split_stage_tile(const SplitParams &P, int b, int h, int64_t base, int n, uint8_t *dst,
+                                                 int ltid, int nthr) {
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(
+            P.g[gg].vc + (((int64_t)b * P.Hkv + h) * P.capacity + base) * P.g[gg].vrow);
+        const uint32_t d = tqdev::smem_u32(dst + (gg ? SPLIT_TILE * P.g[0].vrow : 0));
+        const int words = n * (P.g[gg].vrow / 4);
+        for (int i = ltid; i < words; i += nthr)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d + 4u * (uint32_t)i), "l"(src + i)
+                         : "memory");
+    }
+}
+
 // Partial attention of one chunk of tokens for one (sequence, query head):
-// grid (rows, chunks), SPLIT_SLICES * (d_o + d_n) threads; thread (slice, t)
-// accumulates coordinate t of the concatenated output (group 0 first), in its
-// group's rotated frame, over the chunk's tokens i = slice (mod SPLIT_SLICES).
+// grid (rows, chunks), SPLIT_SLICES * (d_o + d_n) / 2 threads; thread
+// (slice, q) accumulates coordinates 2q and 2q + 1 of the concatenated output
+// (group 0 first; d_o is even, so both are in one group), in that group's
+// rotated frame, over the chunk's tokens i = slice (mod SPLIT_SLICES).
 // Writes the chunk's max combined score m, sum of exp(s - m) and the
 // unnormalised accumulator sum_i exp(s_i - m) n_s,i c[idx_i,t].
 __global__ void __launch_bounds__(1024) tq_split_attend_kernel(const __grid_constant__ SplitParams P,
                                                                int64_t chunk_len, float *part) {
-    __shared__ float s_p[SPLIT_TILE];
-    __shared__ __align__(16) uint32_t s_v[2][SPLIT_TILE * SPLIT_VROW_MAX / 4];
+    // value rows of two tiles (double-buffered): [buf][SPLIT_TILE x (vrow_0 + vrow_1) bytes]
+    extern __shared__ __align__(16) uint8_t s_rows[];
+    __shared__ float s_w[2][SPLIT_TILE];     // exp(s_i - m) n_s,i of this tile, per group
     __shared__ float s_red[32];
     __shared__ float s_acc[SPLIT_SLICES][256];
     __shared__ float s_cv[2][32];
     const int nthr = blockDim.x, ltid = threadIdx.x;
-    const int d0 = P.g[0].d, d1 = P.g[1].d, dt = d0 + d1;
-    const int slice = ltid / dt, tid = ltid % dt;
+    const int d0 = P.g[0].d, d1 = P.g[1].d, dt = d0 + d1, np = dt / 2;
+    const int slice = ltid / np, q = ltid % np;
     const int row = blockIdx.x, b = row / P.Hq, j = row % P.Hq;
     const int h = j / (P.Hq / P.Hkv);
     const int64_t t0 = (int64_t)blockIdx.y * chunk_len;
@@ -117,51 +135,67 @@ __global__ void __launch_bounds__(1024) tq_split_attend_kernel(const __grid_cons
     __syncthreads();
     mx = -INFINITY;
     for (int w = 0; w < nthr / 32; ++w) mx = fmaxf(mx, s_red[w]);
-    const int g = tid < d0 ? 0 : 1;
-    const int jj = g == 0 ? tid : tid - d0;
+    const int c0 = 2 * q;
+    const int g = c0 < d0 ? 0 : 1;
+    const int jj = g == 0 ? c0 : c0 - d0;
     const SplitGroup &G = P.g[g];
     const int bit = G.bv * jj, wi = bit / 32, sh = bit % 32;
+    const bool straddle = sh + 2 * G.bv > 32;
     const uint32_t fm = (1u << G.bv) - 1u;
-    const int vw = G.vrow / 4, nsw = G.bv * G.d / 32;   // row words, word of n_s
-    float acc = 0.f, lsum = 0.f;
-    for (int64_t base = t0; base < t1; base += SPLIT_TILE) {
+    const int vw = G.vrow / 4;
+    float acc0 = 0.f, acc1 = 0.f, lsum = 0.f;
+    // tile k's rows land while tile k - 1 is accumulated
+    const int buf_bytes = SPLIT_TILE * (P.g[0].vrow + P.g[1].vrow);
+    const int goff = g ? SPLIT_TILE * P.g[0].vrow : 0;
+    split_stage_tile(P, b, h, t0, (int)min((int64_t)SPLIT_TILE, t1 - t0), s_rows, ltid, nthr);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    int k = 0;
+    for (int64_t base = t0; base < t1; base += SPLIT_TILE, ++k) {
         const int n = (int)min((int64_t)SPLIT_TILE, t1 - base);
+        const int buf = k & 1;
+        // the other buffer was last read in iteration k - 1, which ended with a barrier
+        if (base + SPLIT_TILE < t1)
+            split_stage_tile(P, b, h, base + SPLIT_TILE, (int)min((int64_t)SPLIT_TILE, t1 - base - SPLIT_TILE),
+                             s_rows + (buf ^ 1) * buf_bytes, ltid, nthr);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 1;" ::: "memory");   // this tile's copies (not the next's)
         __syncthreads();
-        for (int i = ltid; i < n; i += nthr) {
+        // per-token weights of both groups: exp(s_i - m) n_s,i
+        for (int e = ltid; e < 2 * n; e += nthr) {
+            const int gg = e >= n ? 1 : 0, i = e - gg * n;
             const float p = __expf(w0 * s0[base + i] + w1 * s1[base + i] - mx);
-            s_p[i] = p;
-            lsum += p;
-        }
-        // both groups' value rows of the tile, coalesced 4-byte copies
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(
-                P.g[gg].vc + (((int64_t)b * P.Hkv + h) * P.capacity + base) * P.g[gg].vrow);
-            const int words = n * (P.g[gg].vrow / 4);
-            for (int i = ltid; i < words; i += nthr) s_v[gg][i] = __ldg(src + i);
+            if (gg == 0) lsum += p;
+            const uint32_t *r = reinterpret_cast<const uint32_t *>(s_rows + buf * buf_bytes +
+                                                                   (gg ? SPLIT_TILE * P.g[0].vrow : 0)) +
+                                i * (P.g[gg].vrow / 4);
+            s_w[gg][i] = p * __uint_as_float(r[P.g[gg].bv * P.g[gg].d / 32]);
         }
         __syncthreads();
-        const uint32_t *sv = s_v[g];
+        const uint32_t *sv = reinterpret_cast<const uint32_t *>(s_rows + buf * buf_bytes + goff);
+        const float *sw = s_w[g];
 #pragma unroll 4
         for (int i = slice; i < n; i += SPLIT_SLICES) {
             const uint32_t *vr = sv + i * vw;
-            uint32_t code = vr[wi] >> sh;
-            if (sh + G.bv > 32) code |= vr[wi + 1] << (32 - sh);
-            const float ns = __uint_as_float(vr[nsw]);
-            acc = fmaf(s_p[i] * ns, s_cv[g][code & fm], acc);
+            uint32_t raw = vr[wi] >> sh;
+            if (straddle) raw |= vr[wi + 1] << (32 - sh);
+            const float w = sw[i];
+            acc0 = fmaf(w, s_cv[g][raw & fm], acc0);
+            acc1 = fmaf(w, s_cv[g][(raw >> G.bv) & fm], acc1);
         }
+        __syncthreads();
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    __syncthreads();
     if ((ltid & 31) == 0) s_red[ltid >> 5] = lsum;
-    s_acc[slice][tid] = acc;
+    s_acc[slice][c0] = acc0;
+    s_acc[slice][c0 + 1] = acc1;
     __syncthreads();
     float *dst = part + ((int64_t)blockIdx.y * gridDim.x + row) * (dt + 2);
-    if (slice == 0) {
+    for (int c = ltid; c < dt; c += nthr) {
         float a2 = 0.f;
 #pragma unroll
-        for (int sl = 0; sl < SPLIT_SLICES; ++sl) a2 += s_acc[sl][tid];
-        dst[2 + tid] = a2;
+        for (int sl = 0; sl < SPLIT_SLICES; ++sl) a2 += s_acc[sl][c];
+        dst[2 + c] = a2;
     }
     if (ltid == 0) {
         float l = 0.f;
@@ -260,7 +294,12 @@ tq_status tq_launch_split(tq_ctx *co, const tq_codes *ko, tq_ctx *cn, const tq_c
     const int64_t L = split_chunk_len((int)rows, T), chunks = (T + L - 1) / L;
     float *part = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sc) +
                                             ((2 * (size_t)rows * (size_t)T * 4 + 255) & ~size_t(255)));
-    tq_split_attend_kernel<<<dim3(rows, (unsigned)chunks), SPLIT_SLICES * (d0 + d1), 0, stream>>>(P, L, part);
+    const size_t rows_smem = 2 * (size_t)SPLIT_TILE * (P.g[0].vrow + P.g[1].vrow);
+    if ((st = tq_check_cuda(cudaFuncSetAttribute(tq_split_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)rows_smem))) != TQ_OK)
+        return st;
+    tq_split_attend_kernel<<<dim3(rows, (unsigned)chunks), SPLIT_SLICES * (d0 + d1) / 2, rows_smem, stream>>>(P, L,
+                                                                                                        part);
     if ((st = tq_check_cuda(cudaGetLastError())) != TQ_OK) return st;
     tq_split_combine_kernel<<<rows, d0 + d1, 0, stream>>>(P, (int)chunks, part);
     return tq_check_cuda(cudaGetLastError());
