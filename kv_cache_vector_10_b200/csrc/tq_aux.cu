@@ -115,52 +115,85 @@ struct ScoresParams {
     int64_t capacity, T;
     int Hq, Hkv, M, krow, bk;
     int kf16;                  // key norms as binary16
-    float ck[16];
+    int n_planes;              // sigma-planes: odd subsets of the index bits
+    uint32_t plane_sets[8];    // index planes XOR-ed into sigma-plane s
+    float alpha[8];            // Walsh coefficient of sigma-plane s
 };
 
-// One block per (token block, query head, sequence); every thread scores
-// SCORE_TPT tokens, so the query preparation is amortized over
-// SCORE_TPT * AUX_THREADS tokens.
-constexpr int SCORE_TPT = 8;
+// One block of SCORE_THREADS per (token block, query head, sequence); every
+// thread scores SCORE_TPT tokens, so the query preparation and the tables
+// are amortized over SCORE_TPT * SCORE_THREADS tokens, and many resident
+// warps cover the latency of each thread's row loads.
+constexpr int SCORE_THREADS = 512;
+constexpr int SCORE_TPT = 4;
 
+// Scores from byte tables (the decode kernel's method, one thread per token):
+// the codebook is antisymmetric, so C[idx_j] = sum_s alpha_s sigma_s,j with
+// sigma_s,j = +-1 the parity of the index bits in the odd set s; for byte
+// position g of a plane, T_g[x] = sum_{i<8} v[8g + i] (2 bit_i(x) - 1) with v =
+// q_rot gives sum_j q_rot,j sigma_s,j as sum_g T_g[sigma-byte_g], and v = S q_rot
+// gives <S q_rot, 2b - 1> from the sign plane's bytes.  Tables: [position][256]
+// in dynamic shared memory, index positions (d/8) first, then sign positions
+// (m/8).
 template <int D>
-__global__ void __launch_bounds__(AUX_THREADS) tq_scores_kernel(const __grid_constant__ ScoresParams p) {
+__global__ void __launch_bounds__(SCORE_THREADS) tq_scores_kernel(const __grid_constant__ ScoresParams p) {
     __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
-    __shared__ float s_ck[16];
+    extern __shared__ float s_tab[];
+    constexpr int PK = D / 8, NW = D / 32;
     const int j = blockIdx.y, b = blockIdx.z;
     const int h = j / (p.Hq / p.Hkv);
-    if (threadIdx.x < 16) s_ck[threadIdx.x] = p.ck[threadIdx.x];
     prep_query<D>(p.q + ((int64_t)b * p.Hq + j) * D, p.signs + (int64_t)h * (D / 32), p.S + (int64_t)h * p.M * D,
-                  p.M, s_qr, s_sq, p.Q ? p.Q + (int64_t)h * D * D : nullptr);   // its barriers publish s_ck
+                  p.M, s_qr, s_sq, p.Q ? p.Q + (int64_t)h * D * D : nullptr);   // ends with a barrier
+    const int PS = p.M / 8;
+    for (int e = threadIdx.x; e < (PK + PS) * 256; e += blockDim.x) {
+        const int g = e >> 8, x = e & 255;
+        const float *v = g < PK ? s_qr + 8 * g : s_sq + 8 * (g - PK);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a += ((x >> i) & 1) ? v[i] : -v[i];
+        s_tab[e] = a;
+    }
+    __syncthreads();
+    const float *ts = s_tab + PK * 256;
     const float isd = rsqrtf((float)D);
     const float cq = 1.2533141373155003f / (float)p.M;   // sqrt(pi/2) / m
+    const int bk = p.bk, np = p.n_planes;
     for (int k = 0; k < SCORE_TPT; ++k) {
-        const int64_t t = ((int64_t)blockIdx.x * SCORE_TPT + k) * AUX_THREADS + threadIdx.x;
+        const int64_t t = ((int64_t)blockIdx.x * SCORE_TPT + k) * SCORE_THREADS + threadIdx.x;
         if (t >= p.T) break;
-        const uint8_t *row = p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) * p.krow;
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(row);
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(p.kc + (((int64_t)b * p.Hkv + h) * p.capacity + t) *
+                                                                   p.krow);
+        uint32_t pl[4][NW];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int wd = 0; wd < NW; ++wd) pl[q][wd] = q < bk ? w[q * NW + wd] : 0u;
         float a = 0.f;
-#pragma unroll 1
-        for (int wd = 0; wd < D / 32; ++wd) {
-            uint32_t pl[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) pl[q] = q < p.bk ? w[q * (D / 32) + wd] : 0u;
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                int idx = 0;
+        for (int g = 0; g < PK; ++g) {
+            uint32_t by[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) idx |= (int)((pl[q] >> i) & 1u) << q;
-                a = fmaf(s_qr[wd * 32 + i], s_ck[idx], a);
+            for (int q = 0; q < 4; ++q) by[q] = (pl[q][g / 4] >> (8 * (g % 4))) & 0xFFu;
+            const float *tg = s_tab + g * 256;
+#pragma unroll
+            for (int sp = 0; sp < 8; ++sp) {
+                if (sp < np) {
+                    const uint32_t set = p.plane_sets[sp];
+                    uint32_t x = 0u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if ((set >> q) & 1u) x ^= by[q];
+                    a = fmaf(p.alpha[sp], tg[x], a);
+                }
             }
         }
-        const uint32_t *sg = w + p.bk * (D / 32);
+        const uint32_t *sg = w + bk * NW;
         float bq = 0.f;
-#pragma unroll 1
         for (int wd = 0; wd < p.M / 32; ++wd) {
             const uint32_t sw = sg[wd];
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) bq += ((sw >> i) & 1u) ? s_sq[wd * 32 + i] : -s_sq[wd * 32 + i];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) bq += ts[(4 * wd + r) * 256 + ((sw >> (8 * r)) & 0xFFu)];
         }
         const float2 nrm = tqdev::key_norms(sg + p.M / 32, p.kf16 != 0);
         p.scores[((int64_t)b * p.Hq + j) * p.T + t] = (nrm.x * a * isd + cq * nrm.y * bq) * isd;
@@ -555,11 +588,17 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
     p.krow = (int)tq_row_bytes(ctx, TQ_KEYS);
     p.bk = ctx->BK;
     p.kf16 = ctx->norm_f16;
-    for (int i = 0; i < ctx->LK; ++i) p.ck[i] = ctx->ck[i];
-    const int64_t per_block = (int64_t)AUX_THREADS * SCORE_TPT;
+    tq_sigma_planes(ctx, &p.n_planes, p.plane_sets, p.alpha);
+    const int64_t per_block = (int64_t)SCORE_THREADS * SCORE_TPT;
     dim3 grid((unsigned)((T + per_block - 1) / per_block), (unsigned)Hq, (unsigned)codes->batch);
-    if (ctx->d == 128) tq_scores_kernel<128><<<grid, AUX_THREADS, 0, stream>>>(p);
-    else tq_scores_kernel<64><<<grid, AUX_THREADS, 0, stream>>>(p);
+    const size_t tab = (size_t)(ctx->d / 8 + ctx->m / 8) * 256 * sizeof(float);
+    auto kern = ctx->d == 128 ? tq_scores_kernel<128> : tq_scores_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return tq_check_cuda(e);
+    }
+    kern<<<grid, SCORE_THREADS, tab, stream>>>(p);
     return tq_check_cuda(cudaGetLastError());
 }
 

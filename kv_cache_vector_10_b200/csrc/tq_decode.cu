@@ -597,6 +597,12 @@ void sigma_alphas(const tq_ctx *ctx, float *alpha) {
 
 }  // namespace
 
+void tq_sigma_planes(const tq_ctx *ctx, int *n_planes, uint32_t *sets, float *alpha) {
+    *n_planes = n_sigma_planes(ctx->BK);
+    for (int i = 0; i < *n_planes; ++i) sets[i] = sigma_set(ctx->BK, i);
+    sigma_alphas(ctx, alpha);
+}
+
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms) {
     (void)batch;
     std::vector<SegPlan> pl;

@@ -297,3 +297,6 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
 // ------------------------------------------------------------ host helpers
 tq_status tq_check_cuda(cudaError_t e);
 tq_status tq_check_device(const tq_ctx *ctx);
+// Sigma-plane decomposition of the key codebook (odd subsets of the B_K index
+// bits and their Walsh coefficients), as the decode kernel uses it.
+void tq_sigma_planes(const tq_ctx *ctx, int *n_planes, uint32_t *sets, float *alpha);
