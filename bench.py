@@ -170,8 +170,9 @@ class Workload:
                 self.inputs = dict(k_new=w["k"][:, :, T].contiguous(), v_new=w["v"][:, :, T].contiguous(),
                                    q=w["q"])
                 self.tokens_scored = B * Hq * (T + 1)
+                grown = [tq.Segment(self.cache, T + 1, b, 1, codes_batch=b) for b in range(B)]
                 self.pieces = [("decode_append", B * Hkv * (T + 1) * (kr + vr) + B * Hkv * (2 * D * es + kr + vr)
-                                + qb, 3)]
+                                + qb, tq.tq_decode_launch_count(grown, B, Hq, Hkv))]
             else:
                 self.cache = self.codec.alloc(B, Hkv, (T + 15) // 16 * 16, device)
                 self.segments = [tq.Segment(self.cache, T, b, 1, codes_batch=b) for b in range(B)]
@@ -179,7 +180,8 @@ class Workload:
                 self.tokens_scored = B * Hq * T
                 self.pieces = [("encode_keys", B * Hkv * T * (D * es + kr), 1),
                                ("encode_values", B * Hkv * T * (D * es + vr), 1),
-                               ("decode", B * Hkv * T * (kr + vr) + qb, 3)]
+                               ("decode", B * Hkv * T * (kr + vr) + qb,
+                                tq.tq_decode_launch_count(self.segments, B, Hq, Hkv))]
         elif name == "mha_split":
             w = W.mha_decode(device=device, data_seed=2 + seed_shift)
             B, H, T, _ = w["k"].shape
@@ -223,7 +225,8 @@ class Workload:
             es = w["prefix_k"].element_size()
             self.pieces = [("encode_keys", Hkv * P * (D * es + pkr) + A * Hkv * Tt * (D * es + tkr), 2),
                            ("encode_values", Hkv * P * (D * es + pvr) + A * Hkv * Tt * (D * es + tvr), 2),
-                           ("decode", Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + 2 * A * Hq * D * es, 4)]
+                           ("decode", Hkv * P * (pkr + pvr) + A * Hkv * Tt * (tkr + tvr) + 2 * A * Hq * D * es,
+                            tq.tq_decode_launch_count(self.segments, A, Hq, Hkv))]
         elif name == "bulk_encode":
             w = W.bulk_encode(device=device, data_seed=4 + seed_shift)
             self.w = w

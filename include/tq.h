@@ -214,6 +214,15 @@ tq_status tq_dequantize(tq_ctx *ctx, const tq_codes *codes, int64_t n_tokens, fl
 size_t tq_decode_workspace_bytes(const tq_segment *segs, int n_segs, int batch, int n_q_heads,
                                  int n_kv_heads);
 
+/* Number of kernels one tq_decode_attention (or tq_decode_append) call with
+ * this segment list launches on the current device: the query preparation,
+ * one split-K decode launch per group of segments sharing bits, queries per
+ * CTA, m and row length, and the combine step, which is left out when every
+ * sequence is covered by exactly one segment holding tokens that the plan
+ * does not split (the decode kernel then writes the output itself).  -1 if
+ * the arguments are invalid.  Host-only; no device work. */
+int tq_decode_launch_count(const tq_segment *segs, int n_segs, int batch, int n_q_heads, int n_kv_heads);
+
 /* One decode step: for every sequence b and query head j,
  *   out[b][j] = sum_t softmax_t(s_t) v_hat_t
  * over the concatenation of all segments that sequence b attends to, with

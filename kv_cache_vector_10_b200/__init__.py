@@ -36,7 +36,8 @@ STATUS_NAMES = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_ZERO_DIM", 3: "TQ_ERR_D
                 13: "TQ_ERR_LIMIT"}
 
 EXPORTED = ["tq_create", "tq_create_ex", "tq_create_format", "tq_destroy", "tq_ensure_heads", "tq_row_bytes", "tq_packed_bytes", "tq_encode_kv",
-            "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_attention",
+            "tq_attention_scores", "tq_dequantize", "tq_decode_workspace_bytes", "tq_decode_launch_count",
+            "tq_decode_attention",
             "tq_get_status", "tq_reset_status", "tq_status_string", "tq_last_cuda_error",
             "tq_decode_attention_static", "tq_decode_append", "tq_decode_append_workspace_bytes",
             "tq_selftest_wait_timeout", "tq_decode_attention_split", "tq_decode_split_workspace_bytes"]
@@ -79,6 +80,7 @@ def _load():
         "tq_attention_scores": (I, [V, ctypes.POINTER(tq_codes), V, I, I64, V, V]),
         "tq_dequantize": (I, [V, ctypes.POINTER(tq_codes), I64, V, V, V]),
         "tq_decode_workspace_bytes": (SZ, [ctypes.POINTER(tq_segment), I, I, I, I]),
+        "tq_decode_launch_count": (I, [ctypes.POINTER(tq_segment), I, I, I, I]),
         "tq_decode_attention": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V, SZ, V]),
         "tq_decode_attention_static": (I, [ctypes.POINTER(tq_segment), I, V, I, I, I, I, V, I, V]),
         "tq_decode_append": (I, [ctypes.POINTER(tq_segment), I, V, V, I, V, I, I, I, I, V, I, V, SZ, V]),
@@ -201,6 +203,12 @@ def _segment_array(segments):
 def tq_decode_workspace_bytes(segments, batch: int, n_q_heads: int, n_kv_heads: int) -> int:
     arr = _segment_array(segments)
     return _lib.tq_decode_workspace_bytes(arr, len(segments), batch, n_q_heads, n_kv_heads)
+
+
+def tq_decode_launch_count(segments, batch: int, n_q_heads: int, n_kv_heads: int) -> int:
+    """Kernels one decode call with these segments launches (host-only)."""
+    arr = _segment_array(segments)
+    return _lib.tq_decode_launch_count(arr, len(segments), batch, n_q_heads, n_kv_heads)
 
 
 def tq_decode_attention(segments, q, batch: int, n_q_heads: int, n_kv_heads: int, out, workspace, stream=None):

@@ -23,6 +23,7 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
 tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float *k_hat, float *v_hat,
                             cudaStream_t stream);
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
+int tq_decode_launches(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms);
 size_t tq_split_ws(int batch, int Hq, int d_o, int d_n, int64_t T);
 tq_status tq_launch_split(tq_ctx *co, const tq_codes *ko, tq_ctx *cn, const tq_codes *kn, int64_t T, const void *q,
                           tq_dtype q_dtype, int batch, int Hq, void *out, tq_dtype out_dtype, void *ws,
@@ -373,6 +374,13 @@ size_t tq_decode_workspace_bytes(const tq_segment *segs, int n_segs, int batch, 
     int dev = 0;
     cudaGetDevice(&dev);
     return tq_decode_ws(segs, n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
+}
+
+int tq_decode_launch_count(const tq_segment *segs, int n_segs, int batch, int n_q_heads, int n_kv_heads) {
+    if (check_segments(segs, n_segs, batch, n_q_heads, n_kv_heads) != TQ_OK) return -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return tq_decode_launches(segs, n_segs, batch, n_q_heads, n_kv_heads, device_sms(dev));
 }
 
 tq_status tq_decode_attention(const tq_segment *segs, int n_segs, const void *q, tq_dtype q_dtype, int batch,

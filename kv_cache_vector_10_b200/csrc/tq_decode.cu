@@ -94,6 +94,13 @@ __host__ __device__ constexpr int vpair_copies() { return BV <= 4 ? 16 : 1; }
 template <int BV>
 __host__ __device__ constexpr int vpair_entries() { return 1 << (2 * BV); }
 
+// One output element in the caller's type.
+__device__ __forceinline__ void store_out_dt(void *p, int64_t i, float v, int dt) {
+    if (dt == TQ_F32) static_cast<float *>(p)[i] = v;
+    else if (dt == TQ_F16) static_cast<__half *>(p)[i] = __float2half_rn(v);
+    else static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+}
+
 // MT = number of QJL projections when known at compile time (128), else 0;
 // KF = key norms as binary16 (1) or fp32 (0) when MT > 0 (else read from the
 // segment).
@@ -426,10 +433,17 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             const int qi = qchunk * QC + qq;
             if (qi >= nq) continue;
             const int seq_local = qi / P.G, jh = h * P.G + qi % P.G;
-            float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
             float v = 0.f;
             for (int r = 0; r < D; ++r) v = fmaf(Qh[r * D + j], acc[qq * D + r], v);
-            dst[4 + j] = v * isd;
+            v *= isd;
+            if (P.direct) {
+                const float l = ml[2 * qq + 1];
+                store_out_dt(P.out, ((int64_t)(g.first_seq + seq_local) * P.Hq + jh) * D + j, l > 0.f ? v / l : 0.f,
+                             P.out_dtype);
+                continue;
+            }
+            float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
+            dst[4 + j] = v;
             if (j == 0) {
                 dst[0] = ml[2 * qq];
                 dst[1] = ml[2 * qq + 1];
@@ -457,9 +471,15 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         const int qi = qchunk * QC + qq;
         if (qi >= nq) continue;
         const int seq_local = qi / P.G, jh = h * P.G + qi % P.G;
-        float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
         float v = acc[qq * D + j] * inv_d;
         if ((sg[j / 32] >> (j % 32)) & 1) v = -v;
+        if (P.direct) {
+            const float l = ml[2 * qq + 1];
+            store_out_dt(P.out, ((int64_t)(g.first_seq + seq_local) * P.Hq + jh) * D + j, l > 0.f ? v / l : 0.f,
+                         P.out_dtype);
+            continue;
+        }
+        float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + seq_local) * P.Hq + jh) * tq_part_floats(D);
         dst[4 + j] = v;
         if (j == 0) {
             dst[0] = ml[2 * qq];
@@ -603,6 +623,42 @@ void tq_sigma_planes(const tq_ctx *ctx, int *n_planes, uint32_t *sets, float *al
     sigma_alphas(ctx, alpha);
 }
 
+namespace {
+// Direct output: every sequence is covered by exactly one (segment, split)
+// holding tokens, so the decode kernel can write out = o / l itself.
+bool direct_output(const tq_segment *segs, int n_segs, int batch, const std::vector<SegPlan> &pl) {
+    std::vector<int> cover((size_t)batch, 0);
+    for (int s = 0; s < n_segs; ++s) {
+        if (pl[s].n_splits != 1 || segs[s].n_tokens <= 0) return false;
+        for (int b = segs[s].first_seq; b < segs[s].first_seq + segs[s].n_seqs; ++b)
+            if (b >= 0 && b < batch) ++cover[(size_t)b];
+    }
+    for (int b = 0; b < batch; ++b)
+        if (cover[(size_t)b] != 1) return false;
+    return true;
+}
+}  // namespace
+
+int tq_decode_launches(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms) {
+    std::vector<SegPlan> pl;
+    plan_segments(segs, n_segs, Hq, Hkv, n_sms, pl);
+    // one decode launch per (bits, queries per CTA, m, key-row length) group
+    std::vector<int> done(n_segs, 0);
+    int groups = 0;
+    for (int s0 = 0; s0 < n_segs; ++s0) {
+        if (done[s0]) continue;
+        const tq_ctx *c0 = segs[s0].ctx;
+        for (int s = 0; s < n_segs; ++s) {
+            const tq_ctx *c = segs[s].ctx;
+            if (!done[s] && c->BK == c0->BK && pl[s].qc == pl[s0].qc && c->m == c0->m &&
+                tq_row_bytes(c, TQ_KEYS) == tq_row_bytes(c0, TQ_KEYS))
+                done[s] = 1;
+        }
+        ++groups;
+    }
+    return 1 + groups + (direct_output(segs, n_segs, batch, pl) ? 0 : 1);
+}
+
 size_t tq_decode_ws(const tq_segment *segs, int n_segs, int batch, int Hq, int Hkv, int n_sms) {
     (void)batch;
     std::vector<SegPlan> pl;
@@ -631,6 +687,9 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
     P.G = Hq / Hkv;
     P.d = segs[0].ctx->d;
     P.batch = batch;
+    P.out = out;
+    P.out_dtype = (int)out_dtype;
+    P.direct = direct_output(segs, n_segs, batch, pl) ? 1 : 0;
     size_t qtot = 0;
     for (auto &x : pl) qtot += x.qprep_floats;
     P.qprep = static_cast<float *>(ws);
@@ -708,6 +767,7 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
                        : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);
         if (e != cudaSuccess) return tq_check_cuda(e);
     }
+    if (P.direct) return TQ_OK;   // the decode kernel wrote the output
     e = tq_launch_combine(P, out, out_dtype, stream);
     return tq_check_cuda(e);
 }

@@ -47,6 +47,11 @@ struct DecodePlan {
     const void *v_new;
     int kv_dtype;
     int n_append_blocks;
+    // Direct output: every sequence is covered by exactly one (segment, split),
+    // so the decode kernel writes out = o / l itself and no combine runs.
+    void *out;
+    int out_dtype;
+    int direct;
 };
 static_assert(sizeof(DecodePlan) <= 32764, "the plan is passed as a kernel parameter");
 

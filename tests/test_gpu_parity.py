@@ -357,3 +357,36 @@ def test_argument_errors():
     ws = torch.empty(16, dtype=torch.uint8, device=DEV)
     with pytest.raises(tq.TQError, match="WORKSPACE"):
         tq.tq_decode_attention(seg, q[:1], 1, 4, 2, torch.empty(1, 4, 128, device=DEV), ws)
+
+
+@pytest.mark.parametrize("rotation,out_dtype", [("hadamard", torch.float32), ("haar", torch.bfloat16),
+                                                ("hadamard", torch.float16)])
+def test_decode_direct_output_equals_combined(rotation, out_dtype):
+    """When every sequence has one segment and the plan does not split it, the
+    decode kernel writes the output itself (one launch fewer); adding an
+    empty segment per sequence forces the combine step, which must give the
+    same values (for one split it is the same o / l)."""
+    g = torch.Generator().manual_seed(17)
+    B, H, Hq, T, d = 8, 32, 32, 700, 128       # 256 (sequence, kv head) items: one split each
+    k = torch.randn(B, H, T, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, T, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    gc = tq.Codec(d, 4, 128, 5, rotation=rotation)
+    cache = gc.alloc(B, H, 704)
+    gc.encode_kv(k.to(DEV), v.to(DEV), cache)
+    segs = [tq.Segment(cache, T, b, 1, codes_batch=b) for b in range(B)]
+    with_empty = segs + [tq.Segment(cache, 0, b, 1, codes_batch=b) for b in range(B)]
+    assert tq.tq_decode_launch_count(segs, B, Hq, H) == 2              # query prep + decode
+    assert tq.tq_decode_launch_count(with_empty, B, Hq, H) == 3        # + combine
+    out1 = tq.decode_attention(segs, q.to(DEV), H, out_dtype=out_dtype)
+    out2 = tq.decode_attention(with_empty, q.to(DEV), H, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+    # and against the oracle on a few (sequence, head) pairs
+    oc = oracle.Codec(d, 4, 128, 5, rotation=rotation)
+    for b, j in ((0, 0), (5, 17), (7, 31)):
+        ek = oc.encode(k[b, j].double().numpy(), j, True)
+        ev = oc.encode(v[b, j].double().numpy(), j, False)
+        ref = oracle.attention(q[b, j].double().numpy(), [(oc, j, ek["rows"], ev["rows"])])
+        tol = pu.ATTN_ABS + (2 ** -8 if out_dtype == torch.bfloat16 else 2 ** -11 if out_dtype == torch.float16 else 0)
+        assert np.max(np.abs(out1[b, j].float().cpu().numpy() - ref)) <= tol
