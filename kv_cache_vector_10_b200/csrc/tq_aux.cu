@@ -481,6 +481,7 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
 // kv head), the append step's new key and value rows.
 template <int D, typename Tq>
 __global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
+    tqdev::grid_dep_trigger();   // the decode CTAs may start their set-up now
     __shared__ float s_in[D];
     __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
@@ -539,6 +540,7 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(void *p, int64_t i, flo
 // One block of d threads per (sequence, head).
 template <int D, typename To>
 __global__ void __launch_bounds__(D) tq_combine_kernel(const __grid_constant__ DecodePlan P, void *out) {
+    tqdev::grid_dep_wait();   // the partials of the decode launches
     const int b = blockIdx.x / P.Hq, j = blockIdx.x % P.Hq;
     const int PF = tq_part_floats(D);
     float mx = -INFINITY;
@@ -660,7 +662,8 @@ cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cud
 
 cudaError_t tq_launch_combine(const DecodePlan &P, void *out, tq_dtype dt, cudaStream_t stream) {
     const unsigned blocks = (unsigned)(P.batch * P.Hq);
-#define TQ_COMB(DD, TT) tq_combine_kernel<DD, TT><<<blocks, DD, 0, stream>>>(P, out)
+#define TQ_COMB(DD, TT) \
+    return tq_launch_dependent(tq_combine_kernel<DD, TT>, dim3((unsigned)blocks), dim3(DD), 0, stream, P, out)
     if (P.d == 128) {
         if (dt == TQ_F32) TQ_COMB(128, float);
         else if (dt == TQ_F16) TQ_COMB(128, __half);

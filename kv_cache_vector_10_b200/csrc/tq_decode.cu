@@ -115,6 +115,11 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     static_assert(D == 64 || D == 128, "head_dim");
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
+    // An append step's new rows are written by the query-preparation kernel:
+    // wait for it before any row is read.  Otherwise only the prepared
+    // queries depend on it (wait below, after the first tiles are requested).
+    if (P.n_append_blocks) tqdev::grid_dep_wait();
+    tqdev::grid_dep_trigger();
     // ---- locate the work item
     int s = 0;
     int64_t item = blockIdx.x;
@@ -170,7 +175,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                         t_begin + (warp + TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
     }
 
-    // ---- per-query lookup tables
+    // ---- per-query lookup tables (from the query-preparation kernel's output)
+    tqdev::grid_dep_wait();
     const float *qp_base = P.qprep + g.qprep_base;
     for (int li = tid; li < 256; li += blockDim.x) {
         const int gslot = li % 16, lo = li / 16;     // fixed low nibble per build lane
@@ -573,7 +579,9 @@ cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vr
         cudaGetLastError();   // do not leave the failure as the thread's sticky last error
         return e;
     }
-    kern<<<(unsigned)items, TQ_DEC_WARPS * 32, smem, stream>>>(P);
+    // starts while the query preparation (or the previous decode launch) runs
+    e = tq_launch_dependent(kern, dim3((unsigned)items), dim3(TQ_DEC_WARPS * 32), smem, stream, P);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/tq.h"
 
 #define TQ_MAX_LEVELS 32
@@ -270,6 +272,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 
 // Instruction descriptor: kind::f16, A and B binary16, K-major, fp32
 // accumulator, M = 128, N = n.
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel in the stream ends;
+// grid_dep_wait blocks until that kernel has completed and its memory is
+// visible (it returns at once for a kernel launched without the attribute),
+// and grid_dep_trigger lets the next such kernel start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Key-row norms.  Binary16 format: n_s and gamma rounded to binary16 (ties
 // to even) in one 32-bit word, n_s in the low half; pack returns false if
 // either rounds to infinity (the row is then stored as a zero row).
@@ -295,6 +305,25 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
 }  // namespace tqdev
 
 // ------------------------------------------------------------ host helpers
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel in the stream is still running; it must call
+// tqdev::grid_dep_wait() before it reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t tq_launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 tq_status tq_check_cuda(cudaError_t e);
 tq_status tq_check_device(const tq_ctx *ctx);
 // Sigma-plane decomposition of the key codebook (odd subsets of the B_K index
