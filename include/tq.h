@@ -231,7 +231,11 @@ int tq_decode_launch_count(const tq_segment *segs, int n_segs, int batch, int n_
  * lookup tables, keeps an online softmax and the value sum in registers,
  * and shares each tile across the query heads of its kv-head group (GQA)
  * and across all sequences of a shared segment; a second kernel merges the
- * partials by log-sum-exp.
+ * partials by log-sum-exp (left out when every sequence has one unsplit
+ * segment: the decode kernel then writes the output).  The decode and merge
+ * kernels are programmatic dependent launches: they may begin while the
+ * kernel before them in the stream ends, and wait for it before reading its
+ * output.
  *  segs      : HOST array of n_segs (<= TQ_MAX_SEGMENTS) segments; every
  *              sequence in [0, batch) must be covered by at least one.
  *  q         : device [batch][n_q_heads][d] in q_dtype.
@@ -321,9 +325,11 @@ tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uin
  *                     tokens [0, n_tokens) of batch slot b are sequence b's.
  *  q, out           : device [batch][n_q_heads][d_o + d_n], outliers first.
  *  workspace        : >= tq_decode_split_workspace_bytes(...), 16-byte aligned.
- * Query head j reads kv head j / (n_q_heads / n_kv_heads).  Launches four
- * kernels: the query's groups as fp32, each group's exact scores, and one
- * softmax-and-value kernel. */
+ * Query head j reads kv head j / (n_q_heads / n_kv_heads).  Launches five
+ * kernels: the query's groups as fp32, each group's exact scores (the
+ * tq_attention_scores kernel), a softmax-and-value kernel over chunks of
+ * tokens, and the log-sum-exp merge of the chunks with each group's
+ * unrotation. */
 size_t tq_decode_split_workspace_bytes(const tq_ctx *ctx_o, const tq_ctx *ctx_n, int batch, int n_q_heads,
                                        int64_t n_tokens);
 tq_status tq_decode_attention_split(tq_ctx *ctx_o, const tq_codes *codes_o, tq_ctx *ctx_n, const tq_codes *codes_n,
