@@ -106,7 +106,7 @@ def arm_config(workload):
 MEASURED_TRAFFIC = {
     ("encode_keys", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 327339776),
     ("encode_values", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 320737792),
-    ("decode", "mha_decode"): ("tq_decode.cu", "f344464501af8ebb494252e10449a289bb4ca771", 151534848),
+    ("decode", "mha_decode"): ("tq_decode.cu", "05c64fbca48ff7d3b112c4b021c5b1213c090796", 151720960),
 }
 
 
