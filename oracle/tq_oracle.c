@@ -22,8 +22,7 @@
  *         MultiHeadKvCache::new (head h uses seed.wrapping_add(h)).
  *
  * Every step below follows those passages.  Where the pages are silent the
- * plainest reading is taken and marked READING; those readings are listed
- * in the design doc:
+ * plainest reading is taken; those readings are:
  *   R1  PRNG: SplitMix64 (Steele, Lea, Flood 2014) seeded with seed+h.
  *       The first d draws give the signs of the rotation (top bit set ->
  *       -1); the next m*d values, taken in Box-Muller pairs, fill the QJL
