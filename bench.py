@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graphs", action="store_true",
+                    help="replay each piece from a captured CUDA graph instead of launching it eagerly")
     return ap.parse_args()
 
 
@@ -302,15 +304,37 @@ class Workload:
         else:
             self._decode(inp)
 
+    def capture(self, inp):
+        """Capture every piece on `inp` as a CUDA graph; later steps on the
+        same input tensors replay them (the library's launches, dependent
+        launches included, are graph-capturable).  Call after one eager step,
+        which builds the head tables and workspaces."""
+        torch = self.torch
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        self.graphs = {}
+        with torch.cuda.stream(s):
+            for name, _, _ in self.pieces:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    self._run_piece(name, inp)
+                self.graphs[name] = g
+        torch.cuda.current_stream().wait_stream(s)
+        self.graph_inp = inp
+
     def step(self, inp, events=None):
         """One step; events: two CUDA events per piece (start, end).  Returns
         the decode output (None for encode-only workloads)."""
+        graphs = getattr(self, "graphs", None) if getattr(self, "graph_inp", None) is inp else None
         for i, (name, _, _) in enumerate(self.pieces):
             if self.flush is not None:
                 self.flush.zero_()            # evict L2 before each piece (outside its events)
             if events:
                 events[2 * i].record()
-            self._run_piece(name, inp)
+            if graphs:
+                graphs[name].replay()
+            else:
+                self._run_piece(name, inp)
             if events:
                 events[2 * i + 1].record()
         return self.out
@@ -521,8 +545,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    for _ in range(max(args.warmup, 3)):
+    for w in range(max(args.warmup, 3)):
         wl.step(inp)
+        if w == 0 and args.graphs:
+            wl.capture(inp)               # later warm-up and timed steps replay the graphs
     torch.cuda.synchronize()
     # timed region: every piece of every step between its own CUDA events on
     # the launching stream; L2 is flushed before each piece, outside them
@@ -604,7 +630,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": arm_config(wl.name),
+            "config": dict(arm_config(wl.name),
+                           launch="each piece replayed from a captured CUDA graph" if args.graphs else "eager"),
             "roofline": roofline, "kernels": kernels, "gpu_launches": wl.launches * args.steps,
             "clocks": clocks, "e2e": e2e}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
