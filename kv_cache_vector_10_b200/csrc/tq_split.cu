@@ -14,7 +14,7 @@
 // exact scoring kernel (tq_scores_kernel); then one block per (sequence,
 // query head, chunk of tokens) combines the scores, takes the chunk's softmax
 // terms and accumulates each group's values in its rotated frame from the
-// packed codes (256-token tiles of probabilities and of both groups' value
+// packed codes (512-token tiles of probabilities and of both groups' value
 // rows staged in shared memory, the next tile's rows copied with cp.async
 // while the current one is accumulated); a last kernel merges the
 // chunks by their maxima and sums (log-sum-exp) and rotates each group back.
@@ -28,7 +28,7 @@ tq_status tq_check_cuda(cudaError_t e);
 
 namespace {
 
-constexpr int SPLIT_TILE = 256;    // tokens per pass: per-token weights and both groups' value rows in smem
+constexpr int SPLIT_TILE = 512;    // tokens per pass: per-token weights and both groups' value rows in smem
 
 struct SplitGroup {
     const uint8_t *vc;        // packed value rows [batch][H_kv][capacity][vrow]
