@@ -47,6 +47,11 @@ def parse():
                     choices=["mha_decode", "gqa_decode", "shared_prefix", "bulk_encode", "single_head",
                              "mha_append", "mha_decode_haar", "mha_split", "mha_decode_f16norms"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-workers", type=int, default=96, help="reference arm: at most this many processes")
+    ap.add_argument("--ref-units", type=int, default=4, help="reference arm: oracle units per process per step")
+    ap.add_argument("--cpu-single", action="store_true", help="CPU baseline single-threaded only")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other workloads in the same run (the `configs` key)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--graphs", action="store_true",
@@ -401,17 +406,33 @@ def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
 
 # ------------------------------------------------------------ CPU oracle arm
 
+def load_workloads():
+    """The seeded input generators, loaded from their file as a module of
+    their own: importing them through the package would run its __init__,
+    which maps libtq.so into a process that only runs the oracle."""
+    import importlib.util
+    name = "tq_workload_generators"
+    if name in sys.modules:
+        return sys.modules[name]
+    spec = importlib.util.spec_from_file_location(name, os.path.join(ROOT, "kv_cache_vector_10_b200", "workloads.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    sys.modules[name] = mod
+    return mod
+
+
 def oracle_unit(wl_name, rank_seed=0):
     """One bounded CPU-oracle unit of the workload: returns (seconds, units, unit_name, sample_desc).
 
-    Units are KV tokens scored (decode workloads) or input bytes (bulk_encode)."""
+    Units are KV tokens scored (decode workloads) or input bytes (bulk_encode).
+    rank_seed shifts the data seed, so parallel workers take different units."""
     import numpy as np
     import torch
 
     import oracle
-    from kv_cache_vector_10_b200 import workloads as W
+    W = load_workloads()
     if wl_name == "bulk_encode":
-        w = W.bulk_encode(device="cpu", layers=1, heads=1, n_tokens=1024)
+        w = W.bulk_encode(device="cpu", layers=1, heads=1, n_tokens=1024, data_seed=4 + rank_seed)
         oc = oracle.Codec(D, 3, M, 42)
         k = w["k"][0, 0].double().numpy()
         v = w["v"][0, 0].double().numpy()
@@ -421,7 +442,7 @@ def oracle_unit(wl_name, rank_seed=0):
         dt = time.perf_counter() - t0
         return dt, 2 * 1024 * D * 2, "bytes", "1 layer x 1 head x 1024 tokens, bits 3, K+V encode"
     if wl_name == "shared_prefix":
-        w = W.shared_prefix(device="cpu", agents=1, prefix_tokens=1024, tail_tokens=256)
+        w = W.shared_prefix(device="cpu", agents=1, prefix_tokens=1024, tail_tokens=256, data_seed=5 + rank_seed)
         pc, tc = oracle.Codec(D, 2, M, 42), oracle.Codec(D, 4, M, 42)
         t0 = time.perf_counter()
         ekp = pc.encode(w["prefix_k"][0, 0].double().numpy(), 0, True)
@@ -434,7 +455,7 @@ def oracle_unit(wl_name, rank_seed=0):
         dt = time.perf_counter() - t0
         return dt, 4 * (1024 + 256), "tokens", "1 agent x 1 kv head (4 q heads), prefix 1024 + tail 256 tokens"
     if wl_name == "mha_split":
-        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=512)
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=512, data_seed=2 + rank_seed)
         order = w["k"][0, 0].pow(2).mean(dim=0).argsort(descending=True)
         k, v, q = (w["k"][0, 0][:, order].double().numpy(), w["v"][0, 0][:, order].double().numpy(),
                    w["q"][0, 0][order].double().numpy())
@@ -446,7 +467,7 @@ def oracle_unit(wl_name, rank_seed=0):
         dt = time.perf_counter() - t0
         return dt, 512, "tokens", "1 kv head x 1 query head x 512 tokens: encode both channel groups + split decode"
     if wl_name == "mha_append":
-        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1025)
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1025, data_seed=2 + rank_seed)
         oc = oracle.Codec(D, w["bits"], M, w["seed"])
         k, v = w["k"][0, 0].double().numpy(), w["v"][0, 0].double().numpy()
         ek, ev = oc.encode(k[:1024], 0, True), oc.encode(v[:1024], 0, False)     # the cached history
@@ -457,13 +478,13 @@ def oracle_unit(wl_name, rank_seed=0):
         dt = time.perf_counter() - t0
         return dt, 1025, "tokens", "1 kv head x 1 query head: append 1 token to 1024 + decode over 1025"
     if wl_name in ("mha_decode", "mha_decode_haar", "mha_decode_f16norms"):
-        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024)
+        w = W.mha_decode(device="cpu", batch=1, heads=1, n_tokens=1024, data_seed=2 + rank_seed)
         G = 1
     elif wl_name == "gqa_decode":
-        w = W.gqa_decode(device="cpu", batch=1, q_heads=4, kv_heads=1, n_tokens=1024)
+        w = W.gqa_decode(device="cpu", batch=1, q_heads=4, kv_heads=1, n_tokens=1024, data_seed=3 + rank_seed)
         G = 4
     else:
-        w = W.single_head(device="cpu")
+        w = W.single_head(device="cpu", data_seed=1 + rank_seed)
         G = 4
     oc = oracle.Codec(D, w["bits"], M, w["seed"], rotation="haar" if wl_name == "mha_decode_haar" else "hadamard",
                       norms="f16" if wl_name == "mha_decode_f16norms" else "f32")
@@ -477,45 +498,194 @@ def oracle_unit(wl_name, rank_seed=0):
     return dt, G * T, "tokens", f"1 kv head x {G} query head(s) x {T} tokens: encode K+V + decode"
 
 
-def cpu_baseline(wl_name, seconds):
+def _oracle_loop(wl_name, seconds, worker):
+    """Run oracle units of the workload for about `seconds` of CPU time
+    (worker w takes data seeds shifted by 1000 w); returns (seconds, units,
+    unit, desc, count)."""
+    try:
+        import torch
+        torch.set_num_threads(1)
+    except Exception:
+        pass
     tot_t, tot_u, n = 0.0, 0, 0
     unit = desc = None
     while tot_t < seconds or n == 0:
-        dt, u, unit, desc = oracle_unit(wl_name)
+        dt, u, unit, desc = oracle_unit(wl_name, rank_seed=1000 * worker + n)
         tot_t += dt
         tot_u += u
         n += 1
-    val = tot_u / tot_t
+    return tot_t, tot_u, unit, desc, n
+
+
+def host_cpu():
+    """(usable cores, CPU model) of this host."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
+def _baseline_entry(val, unit, cores, sample):
     if unit == "bytes":
-        return {"value": val / 1e9, "unit": "GB/s in", "cores": 1, "kind": "oracle",
-                "sample": f"{n} x ({desc}), {tot_t:.1f} s single-threaded fp64 C oracle"}
-    return {"value": val, "unit": "KV tokens scored/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} x ({desc}), {tot_t:.1f} s single-threaded fp64 C oracle"}
+        return {"value": val / 1e9, "unit": "GB/s in", "cores": cores, "kind": "oracle", "sample": sample}
+    return {"value": val, "unit": "KV tokens scored/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+
+def cpu_baseline(wl_name, seconds, all_cores=True, max_workers=96):
+    """The oracle timed on the host: single-threaded, and (all_cores) one
+    process per core over independent (sequence, head) units, each process
+    running its own units for about `seconds`; the all-core value is the sum
+    of the processes' own rates (they run at the same time).  Processes are
+    started with `spawn` (never forked from a process that used the GPU)."""
+    ncores, model = host_cpu()
+    t1, u1, unit, desc, n1 = _oracle_loop(wl_name, seconds, 0)
+    single = _baseline_entry(u1 / t1, unit, 1, f"{n1} x ({desc}), {t1:.1f} s, single-threaded fp64 C oracle")
+    single["cpu_model"] = model
+    single["nproc"] = ncores
+    if not all_cores or ncores <= 1:
+        return single
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    workers = min(ncores, max_workers)
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+        res = list(ex.map(_oracle_loop, [wl_name] * workers, [seconds] * workers, range(1, workers + 1)))
+    rate = sum(u / t for t, u, _, _, _ in res)
+    nall = sum(r[4] for r in res)
+    tall = max(r[0] for r in res)
+    multi = _baseline_entry(rate, unit, workers,
+                            f"{workers} processes x about {tall:.1f} s each, {nall} units of ({desc}) in total, "
+                            f"fp64 C oracle, one process per core over independent (sequence, head) units")
+    multi["cpu_model"] = model
+    multi["nproc"] = ncores
+    multi["single_thread"] = single
+    return multi
+
+
+def _oracle_units(wl_name, n, seed0):
+    """n oracle units of the workload (data seeds seed0, seed0 + 1, ...): (seconds, units, unit, desc);
+    seconds counts the oracle's work only, not the input generation."""
+    try:
+        import torch
+        torch.set_num_threads(1)
+    except Exception:
+        pass
+    tot_t, tot_u = 0.0, 0
+    unit = desc = None
+    for i in range(n):
+        dt, u, unit, desc = oracle_unit(wl_name, rank_seed=seed0 + i)
+        tot_t += dt
+        tot_u += u
+    return tot_t, tot_u, unit, desc
 
 
 def run_reference(args):
+    """The oracle, as it stands, on the host's cores: one process per core
+    (spawned), each step every process runs `--ref-units` oracle units of the
+    workload on its own seeds.  A step's time is the slowest process's oracle
+    time in that step (input generation excluded); value = all units / the
+    sum of the step times.  Rank 0 alone runs it; other ranks exit without
+    work."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    for _ in range(args.warmup):
-        oracle_unit(args.workload)
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    ncores, model = host_cpu()
+    workers = max(1, min(ncores, args.ref_workers))
+    per = max(1, args.ref_units)
     tot_t, tot_u, unit, desc = 0.0, 0, None, None
-    for _ in range(args.steps):
-        dt, u, unit, desc = oracle_unit(args.workload)
-        tot_t += dt
-        tot_u += u
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+        def one_step(i):
+            seeds = [per * (workers * i + w) for w in range(workers)]
+            res = list(ex.map(_oracle_units, [args.workload] * workers, [per] * workers, seeds))
+            return max(r[0] for r in res), sum(r[1] for r in res), res[0][2], res[0][3]
+        for i in range(args.warmup):
+            one_step(i)
+        for i in range(args.steps):
+            dt, u, unit, desc = one_step(args.warmup + i)
+            tot_t += dt
+            tot_u += u
     val = tot_u / tot_t
     unit_name = "GB/s in" if unit == "bytes" else "KV tokens scored/s"
     if unit == "bytes":
         val /= 1e9
+    sample = (f"{args.steps} timed steps; each step {workers} processes x {per} unit(s) of ({desc}), "
+              f"fp64 C oracle, one process per core")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit_name, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(arm_config(args.workload), oracle_sample=desc),
-            "cpu_baseline": {"value": val, "unit": unit_name, "cores": 1, "kind": "oracle",
-                             "sample": f"{args.steps} timed steps, each {desc}"},
+            "cpu_baseline": {"value": val, "unit": unit_name, "cores": workers, "kind": "oracle", "sample": sample,
+                             "nproc": ncores, "cpu_model": model},
             "e2e": {"value": val, "unit": unit_name, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ timing helpers
+
+CONFIG_WORKLOADS = ["mha_decode", "gqa_decode", "bulk_encode", "shared_prefix"]
+
+
+def piece_table(wl, piece_samples, hbm, peak_kind):
+    """Per piece: mean, median and best of its event times, algorithmic bytes,
+    achieved GB/s (from the mean) and the fraction of the HBM peak."""
+    kernels = {}
+    for (name, nbytes, nl), xs in zip(wl.pieces, piece_samples):
+        srt = sorted(xs)
+        ms = sum(xs) / len(xs)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        kernels[name] = {"ms": ms, "ms_median": srt[len(srt) // 2], "ms_best": srt[0], "iterations": len(xs),
+                         "launches": nl, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+                         "frac_of_" + peak_kind + "_hbm": gbs / hbm,
+                         "frac_best_of_" + peak_kind + "_hbm": nbytes / (srt[0] * 1e-3) / 1e9 / hbm,
+                         "traffic": measured_traffic(name, wl.name)}
+        if name.startswith("decode"):
+            kernels[name]["kv_tokens_scored_per_s"] = wl.tokens_scored / (ms * 1e-3)
+    return kernels
+
+
+def time_config(name, dev, steps, warmup):
+    """Time one workload's pieces (L2 flushed before each, CUDA events on the
+    launching stream) over `steps` steps after `warmup`; returns its entry of
+    the `configs` key.  The workload's tensors are released afterwards."""
+    import torch
+    wl = Workload(name, dev, 0)
+    inp = wl.inputs
+    for _ in range(warmup):
+        wl.step(inp)
+    torch.cuda.synchronize()
+    n = len(wl.pieces)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n)] for _ in range(steps)]
+    for i in range(steps):
+        wl.step(inp, evs[i])
+    torch.cuda.synchronize()
+    samples = [[e[2 * p].elapsed_time(e[2 * p + 1]) for e in evs] for p in range(n)]
+    ms_step = sum(sum(x) / steps for x in samples)
+    kernels = piece_table(wl, samples, 1.0, "unit")
+    for k in kernels.values():           # fractions are filled in against the peak by the caller
+        k.pop("frac_of_unit_hbm")
+        k.pop("frac_best_of_unit_hbm")
+    if name == "bulk_encode":
+        value, unit = wl.in_bytes / (ms_step * 1e-3) / 1e9, "GB/s in"
+    else:
+        value, unit = wl.tokens_scored / (ms_step * 1e-3), "KV tokens scored/s"
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    out = {"workload": WORKLOAD_DESC[name], "step": STEP_DESC[name], "value": value, "unit": unit,
+           "ms_per_step": ms_step, "steps": steps, "warmup": warmup, "dominant_kernel": dom, "kernels": kernels,
+           "gpu_launches": wl.launches * steps}
+    del wl, inp
+    torch.cuda.empty_cache()
+    return out
 
 
 # -------------------------------------------------------------------- main
@@ -562,11 +732,21 @@ def main():
         wl.step(inp, evs[i])
     torch.cuda.synchronize()
     barrier()
+    piece_samples = [[e[2 * p].elapsed_time(e[2 * p + 1]) for e in evs] for p in range(npieces)]
+    piece_ms = [sum(x) / args.steps for x in piece_samples]
+    ms_step = max_over_ranks(sum(piece_ms), world, dev)
+
+    # the other workloads, each timed in the same run (one GPU only)
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = {}
+        for other in CONFIG_WORKLOADS:
+            if other == args.workload:
+                continue
+            configs[other] = time_config(other, dev, max(args.steps, 50), max(args.warmup, 5))
     if smi is not None:
         time.sleep(0.25)
         smi.terminate()
-    piece_ms = [sum(e[2 * p].elapsed_time(e[2 * p + 1]) for e in evs) / args.steps for p in range(npieces)]
-    ms_step = max_over_ranks(sum(piece_ms), world, dev)
     clocks = summarize_clocks(rows)
 
     # end to end through host buffers
@@ -615,13 +795,7 @@ def main():
         value, unit = job_throughput(wl.in_bytes, world, ms_step * 1e-3) / 1e9, "GB/s in"
     else:
         value, unit = job_throughput(wl.tokens_scored, world, ms_step * 1e-3), "KV tokens scored/s"
-    kernels = {}
-    for (name, nbytes, nl), ms in zip(wl.pieces, piece_ms):
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        kernels[name] = {"ms": ms, "launches": nl, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
-                         "frac_of_" + peak_kind + "_hbm": gbs / hbm}
-        if name.startswith("decode"):
-            kernels[name]["kv_tokens_scored_per_s"] = wl.tokens_scored / (ms * 1e-3)
+    kernels = piece_table(wl, piece_samples, hbm, peak_kind)
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved_gbs"], "peak": hbm, "unit": "GB/s",
@@ -634,8 +808,15 @@ def main():
                            launch="each piece replayed from a captured CUDA graph" if args.graphs else "eager"),
             "roofline": roofline, "kernels": kernels, "gpu_launches": wl.launches * args.steps,
             "clocks": clocks, "e2e": e2e}
+    if configs is not None:
+        for c in configs.values():
+            c["peak_gbs"] = hbm
+            for k2, v2 in c["kernels"].items():
+                v2["frac_of_" + peak_kind + "_hbm"] = v2["achieved_gbs"] / hbm
+                v2["frac_best_of_" + peak_kind + "_hbm"] = v2["algorithmic_bytes"] / (v2["ms_best"] * 1e-3) / 1e9 / hbm
+        line["configs"] = configs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, all_cores=not args.cpu_single)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -76,8 +76,9 @@ typedef enum tq_status {
 typedef enum tq_dtype { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
 typedef enum tq_which { TQ_KEYS = 0, TQ_VALUES = 1, TQ_BOTH = 2 } tq_which;
 
-/* The random rotation Pi (turboquant-plus-rs README, Architecture: "random
- * rotation (Haar-distributed or fast Walsh-Hadamard)"; Modules: rotation). */
+/* The random rotation Pi (turboquant-plus-rs README, Architecture and
+ * Modules: rotation -- either a Haar-random orthogonal matrix or a fast
+ * Walsh-Hadamard transform with random signs). */
 /* Storage of the two key-row norms (turboquant-plus-rs README,
  * "Compression formats": turbo4 is 4.25 bits per value, which binary16
  * norms give a key row at b = 4, d = m = 128). */
@@ -160,7 +161,10 @@ tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, t
 tq_status tq_create_format(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
                            tq_norm_format key_norms, tq_ctx **out);
 
-/* Release a context and its device tables (synchronizes the device). NULL is a no-op. */
+/* Release a context and its device tables (synchronizes the device). NULL is a no-op.
+ * The counterpart of dropping a bitpolar KvCacheCompressor / MultiHeadKvCache
+ * (bitpolar 0.3.3 src/kv_cache.rs): the context owns its codec state, the
+ * caller owns the caches it filled. */
 void tq_destroy(tq_ctx *ctx);
 
 /* Build and upload the tables of heads 0..n_heads-1 (head h uses seed + h,
@@ -223,7 +227,12 @@ size_t tq_decode_workspace_bytes(const tq_segment *segs, int n_segs, int batch, 
  * the arguments are invalid.  Host-only; no device work. */
 int tq_decode_launch_count(const tq_segment *segs, int n_segs, int batch, int n_q_heads, int n_kv_heads);
 
-/* One decode step: for every sequence b and query head j,
+/* One decode step (bitpolar 0.3.3 src/kv_cache.rs: attention_scores gives the
+ * pre-softmax scores q.K^T/sqrt(d) of the stored keys and decode_values the
+ * stored values; turboquant-plus-rs README, Architecture: the inner product
+ * is estimated from the codes; fib-quant README, C Kernels: compressed
+ * attention logits followed by the softmax).  For every sequence b and
+ * query head j,
  *   out[b][j] = sum_t softmax_t(s_t) v_hat_t
  * over the concatenation of all segments that sequence b attends to, with
  * s_t the score of tq_attention_scores.  Split-K over tokens: each work item
@@ -295,7 +304,10 @@ size_t tq_decode_append_workspace_bytes(const tq_segment *segs, int n_segs, int 
  *    them allocates; call tq_ensure_heads first).
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept for the life of the
+ *    process, per device number: only the device's primary context (the
+ *    one the CUDA runtime uses) is supported, and the address is not looked
+ *    up again after cudaDeviceReset.
  *  - Every call on a device shares the one array and it keeps the last
  *    call's contents; nothing in it needs clearing, because the decode writes
  *    every scratch value it later reads.  Calls that overlap on the GPU
@@ -308,12 +320,16 @@ tq_status tq_decode_attention_static(const tq_segment *segs, int n_segs, const v
 
 /* Synchronize `stream` and read the context's status word: the number of
  * non-finite rows encoded so far, and device error flags (bit 0: a bounded
- * wait inside a kernel gave up; its outputs for that tile are invalid). */
+ * wait inside a kernel gave up; its outputs for that tile are invalid).
+ * bitpolar 0.3.3 src/kv_cache.rs rejects a non-finite input row with
+ * NonFiniteInput before it is stored; on the GPU the rows of one call are
+ * encoded in parallel, so such rows are stored as zero vectors and counted
+ * here instead of failing the call. */
 tq_status tq_get_status(tq_ctx *ctx, void *stream, uint64_t *nonfinite_rows, uint32_t *error_flags);
 
 /* Decode attention over an outlier/normal channel-split cache
- * (turboquant-plus-rs README, Modules: outlier -- "Non-integer bit rates via
- * outlier/normal channel splitting").  A head's channels are split into an
+ * (turboquant-plus-rs README, Modules: outlier -- a fractional bit rate from
+ * coding outlier and normal channels at different widths).  A head's channels are split into an
  * outlier group (the first d_o channels, codec ctx_o) and a normal group (the
  * next d_n channels, codec ctx_n); each group is encoded with tq_encode_kv
  * of its own codec (e.g. 64 channels at b+1 bits and 64 at b: b + 1/2 index

@@ -157,16 +157,21 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         const int e = i / VCOP;
         vlut[i] = make_float2(g.vtab[e & ((1 << BV) - 1)], g.vtab[e >> BV]);
     }
+    // The abort flag is read once per CTA, before any copy is requested: a CTA
+    // of an aborted context requests nothing and waits for nothing.
+    __shared__ int s_abort;
     if (tid == 0) {
         for (int i = 0; i < 2 * TQ_DEC_WARPS; ++i) tqdev::mbar_init(&bars[i], 1);
         tqdev::fence_barrier_init();
+        s_abort = tqdev::status_aborted(g.status) ? 1 : 0;
     }
     __syncthreads();
+    const bool pre_aborted = s_abort != 0;
 
     const int64_t n_chunks = t_end > t_begin ? (t_end - t_begin + TQ_DEC_CHUNK - 1) / TQ_DEC_CHUNK : 0;
     const uint8_t *kbase = g.kc + (int64_t)h * g.capacity * krow;
     const uint8_t *vbase = g.vc + (int64_t)h * g.capacity * vrow;
-    if (lane == 0) {
+    if (lane == 0 && !pre_aborted) {
         if (warp < n_chunks)
             issue_chunk(stage + (warp * 2 + 0) * chunk_bytes, &bars[warp * 2 + 0], kbase, vbase, t_begin + warp * TQ_DEC_CHUNK,
                         g.capacity, krow, vrow);
@@ -252,13 +257,19 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[qq][c] = make_float2(0.f, 0.f);
     }
-    bool aborted = tqdev::status_aborted(g.status);
+    bool aborted = pre_aborted;
     for (int64_t k = 0; !aborted; ++k) {
         const int64_t ci = warp + k * TQ_DEC_WARPS;
         if (ci >= n_chunks) break;
         const int buf = (int)(k & 1);
         if (!tqdev::mbar_wait_bounded(&bars[warp * 2 + buf], (uint32_t)((k >> 1) & 1))) {
             aborted = true;
+            // Both of this warp's buffers may still have a copy in flight (the
+            // one just waited for, and the next chunk's in the other buffer):
+            // give each one more bounded wait before `stage` is reused below.
+            tqdev::mbar_wait_bounded(&bars[warp * 2 + buf], (uint32_t)((k >> 1) & 1));
+            if (ci + TQ_DEC_WARPS < n_chunks)
+                tqdev::mbar_wait_bounded(&bars[warp * 2 + (buf ^ 1)], (uint32_t)(((k + 1) >> 1) & 1));
             break;
         }
         const uint8_t *sK = stage + (warp * 2 + buf) * chunk_bytes;

@@ -624,8 +624,13 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
     tqdev::tc_fence_after();
     const uint32_t tlane = s_tmem + ((uint32_t)(warp * 32) << 16);
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
+    bool q_pending = false;   // thread 0: Q tiles requested, not yet seen
+    int rot_drain = -1;       // phase of a rotation MMA not seen complete
     if constexpr (ROT == 1) {
-        if (tid == 0 && !s_abort) load_q_tiles<D>(sQ, &tmapQ, head, &s_bars[0]);
+        if (tid == 0 && !s_abort) {
+            load_q_tiles<D>(sQ, &tmapQ, head, &s_bars[0]);
+            q_pending = true;
+        }
     }
     // 16-bit inputs: each tile's rows are loaded into registers during the
     // previous tile's quantization
@@ -653,6 +658,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
             __syncthreads();
             if (tid == 0 && !s_abort) {
                 if (tile > 0 || tqdev::mbar_wait_bounded(&s_bars[0], 0)) {
+                    q_pending = false;
                     tqdev::tc_fence_after();
                     issue_dense_rotation<D, Tin>(s_tmem, xHi, xLo, sQ, &s_bars[1]);
                 } else {
@@ -662,6 +668,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
                 }
             }
             const bool done = s_abort ? true : tqdev::mbar_wait_bounded(&s_bars[1], (uint32_t)(tile & 1));
+            if (!done) rot_drain = tile & 1;
             if (__syncthreads_or(!done || s_abort)) {
                 if (tid == 0 && !done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
                 break;
@@ -769,6 +776,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
         }
         if (valid) dst[BV * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2) * inv_scale);
     }
+    if (rot_drain >= 0) tqdev::mbar_wait_bounded(&s_bars[1], (uint32_t)rot_drain);
+    if (q_pending) tqdev::mbar_wait_bounded(&s_bars[0], 0);
     tqdev::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -821,11 +830,19 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     tqdev::tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const uint32_t tlane = tmem_base + ((uint32_t)(warp * 32) << 16);
+    // Copies and MMAs that a timed-out wait left in flight; each gets one more
+    // bounded wait before the CTA frees its TMEM and exits.
+    bool s_pending = false, q_pending = false;   // thread 0: S / Q tiles requested, not yet seen
+    int qjl_drain = -1, rot_drain = -1;          // phase of a QJL / rotation MMA not seen complete
     if (tid == 0 && !*s_abort) {
         tqdev::mbar_expect_tx(&bars[0], (uint32_t)(M * D * 2));
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) tqdev::tma_load_2d(sS + a * M * 128, &tmapS, a * 64, head * M, &bars[0]);
-        if constexpr (ROT == 1) load_q_tiles<D>(sQ, &tmapQ, head, &bars[2]);
+        s_pending = true;
+        if constexpr (ROT == 1) {
+            load_q_tiles<D>(sQ, &tmapQ, head, &bars[2]);
+            q_pending = true;
+        }
     }
     const Tin *src = reinterpret_cast<const Tin *>(p.x) + b * p.sb + (int64_t)head * p.sh;
     uint8_t *aHi = sA, *aLo = sA + A_BYTES;
@@ -860,6 +877,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
             __syncthreads();
             if (tid == 0) {
                 if (tile > 0 || tqdev::mbar_wait_bounded(&bars[2], 0)) {
+                    q_pending = false;
                     tqdev::tc_fence_after();
                     issue_dense_rotation<D, Tin>(tmem_base, aHi, aLo, sQ, &bars[3]);
                 } else {
@@ -872,6 +890,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
                 if (tile + 1 < ntiles) load_row_words<D, Tin>(src + (t + ENC_ROWS) * p.st, t + ENC_ROWS < p.T, raw);
             }
             const bool rdone = tqdev::mbar_wait_bounded(&bars[3], (uint32_t)(tile & 1));
+            if (!rdone) rot_drain = tile & 1;
             if (__syncthreads_or(!rdone || *s_abort)) {
                 if (tid == 0 && !rdone) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
                 if (tid == 0) *s_abort = 1;
@@ -1025,6 +1044,7 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         if (__syncthreads_or(*s_abort)) break;
         if (tid == 0) {
             const bool ok = tile > 0 || tqdev::mbar_wait_bounded(&bars[0], 0);
+            if (ok) s_pending = false;
             if (!ok) {
                 atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
                 *s_abort = 1;
@@ -1059,7 +1079,10 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         if (!done || *s_abort) {
             // this thread skips the epilogue; the flag ends the loop for every
             // thread at the next pre-MMA barrier
-            if (!done) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+            if (!done) {
+                atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+                qjl_drain = tile & 1;
+            }
             *s_abort = 1;
             continue;
         }
@@ -1082,6 +1105,10 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
         }
         n2 = n2_next;
     }
+    if (qjl_drain >= 0) tqdev::mbar_wait_bounded(&bars[1], (uint32_t)qjl_drain);
+    if (rot_drain >= 0) tqdev::mbar_wait_bounded(&bars[3], (uint32_t)rot_drain);
+    if (s_pending) tqdev::mbar_wait_bounded(&bars[0], 0);
+    if (q_pending) tqdev::mbar_wait_bounded(&bars[2], 0);
     tqdev::tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -1,6 +1,6 @@
 // tq_split.cu -- decode attention over an outlier/normal channel-split cache
-// (turboquant-plus-rs README, Modules: outlier -- "Non-integer bit rates via
-// outlier/normal channel splitting").
+// (turboquant-plus-rs README, Modules: outlier -- fractional bits per value
+// obtained by coding outlier and normal channels at different widths).
 //
 // A head's channels are split into an outlier group (channels [0, d_o)) and
 // a normal group (channels [d_o, d_o + d_n)); each group is a codec of its

@@ -7,15 +7,17 @@
 //    and fill the QJL matrix S row-major [m][d], each rounded to binary16
 //    (nearest, ties to even) -- the rounded value is the matrix the codec
 //    uses, which also makes it exact as a tensor-core operand.
-//  * Haar rotations (turboquant-plus-rs README, Modules: rotation --
-//    "Haar-distributed rotation via QR"): Q = the orthogonal factor of the
+//  * Haar rotations (turboquant-plus-rs README, Modules: rotation, which
+//    names a Haar-random rotation built from a QR factorization): Q = the
+//    orthogonal factor of the
 //    QR factorization of a d x d Gaussian matrix G with R's diagonal
 //    positive.  G's entries are Box-Muller pairs continuing head h's stream
 //    after the sign and S draws.  The factorization here is Gram-Schmidt run
 //    twice per column (its R diagonal is a norm, hence positive), in fp64.
 //  * Lloyd-Max codebooks of N(0,1) (turboquant-plus-rs README, Modules:
-//    "codebook -- optimal MSE centroids, closed-form (1-2 bit) and Lloyd's
-//    algorithm (3+ bit)"): the iteration runs on the positive half-line,
+//    codebook -- MSE-optimal centroids, given in closed form at 1 and 2 bits
+//    and found by Lloyd iteration from 3 bits up): the iteration runs on the
+//    positive half-line,
 //    using the codebook's symmetry, to |change| < 1e-15.
 //
 // Compiled by the host C++ compiler (not nvcc) with contraction off so the

@@ -50,8 +50,9 @@
  *       pairs (not rounded) from the head's SplitMix64 stream continued after
  *       the d sign draws and the draws of S.  The rest of the method is
  *       unchanged: z = sqrt(d) Q x / ||x||, reconstruction Q^T (...).
- *   R10 Outlier/normal channel splitting ([TQ] Modules, outlier: "Non-integer
- *       bit rates via outlier/normal channel splitting"): a head's d channels
+ *   R10 Outlier/normal channel splitting ([TQ] Modules, outlier: a
+ *       fractional bit rate from coding outlier and normal channels at
+ *       different widths): a head's d channels
  *       are split into two groups, outliers first (the caller orders the
  *       channels); each group is a codec of its own (its own rotation over the
  *       group's channels, its own bits), so the bits per value are the

@@ -19,6 +19,22 @@ REL = 1e-4           # dequantized vectors, scores, stored norms
 ATTN_ABS = 2e-3      # attention outputs
 
 
+def attn_tolerance(ref: np.ndarray, out_dtype) -> np.ndarray:
+    """Per-element bound on |out - ref| for attention outputs written in
+    `out_dtype`: ATTN_ABS on the value before it is rounded to the output
+    type, plus the rounding itself, at most half an ulp of that type at
+    |ref| + ATTN_ABS (no slack for float32 outputs)."""
+    ref = np.abs(np.asarray(ref, dtype=np.float64)) + ATTN_ABS
+    if out_dtype == torch.float32:
+        return np.full_like(ref, ATTN_ABS)
+    mant = {torch.bfloat16: 8, torch.float16: 11}[out_dtype]
+    _, e = np.frexp(ref)                     # ref in [2^(e-1), 2^e)
+    half_ulp = np.ldexp(1.0, e - 1 - mant)   # ulp 2^(e-1-(mant-1)), halved
+    if out_dtype == torch.float16:
+        half_ulp = np.maximum(half_ulp, 2.0 ** -25)   # binary16 subnormal spacing / 2
+    return ATTN_ABS + half_ulp
+
+
 def unpack_k(rows: np.ndarray, d: int, bk: int, m: int, norms: str = "f32"):
     """rows [N, k_row_bytes] uint8 -> idx [N, d], bits [N, m], ns [N], gamma [N].
     norms "f16": the tail is n_s, gamma as binary16 (one 32-bit word)."""

@@ -1,5 +1,5 @@
-"""The Haar-QR rotation (turboquant-plus-rs README, Modules: rotation --
-"Haar-distributed rotation via QR"), GPU against the oracle.
+"""The Haar-QR rotation (turboquant-plus-rs README, Modules: rotation: a
+Haar-random rotation from a QR factorization), GPU against the oracle.
 
 Same bars as the Walsh-Hadamard path: codes and QJL signs bit-exact outside
 the 1e-5 boundary band, norms / dequantized vectors / scores within 1e-4

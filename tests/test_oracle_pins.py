@@ -60,6 +60,31 @@ def test_head_tables_distribution():
     assert np.array_equal(S1, S0b) and np.array_equal(s1, s0b)   # seed+h wrapping add
 
 
+@pytest.mark.parametrize("d,m,seed,h", [(16, 12, 77, 3), (128, 128, 42, 5), (8, 3, 2 ** 64 - 2, 4)])
+def test_head_tables_draw_layout(d, m, seed, h):
+    """Where each draw of the head's SplitMix64 stream (seed + h, wrapping)
+    lands: draw j < d gives sign j from its top bit (set -> -1); the next
+    draws, two at a time, give S row-major by Box-Muller, u1 = ((a>>11)+1)
+    2^-53 from the first draw of the pair and u2 = (b>>11) 2^-53 from the
+    second, cos to the even entry and sin to the odd one, each entry rounded
+    to binary16 (numpy's IEEE conversion here).  A swapped u1/u2, a swapped
+    cos/sin, another sign bit or a missing rounding fails."""
+    signs, S = oracle.head_tables(d, m, seed, h)
+    n = m * d
+    u = [int(x) for x in oracle.splitmix64_stream((seed + h) % 2 ** 64, d + n + (n % 2))]
+    for j in range(d):
+        assert signs[j] == (-1.0 if u[j] >> 63 else 1.0)
+    flat = S.ravel()
+    for i in range(0, n, 2):
+        a, b = u[d + i], u[d + i + 1]
+        u1 = ((a >> 11) + 1) * 2.0 ** -53
+        u2 = (b >> 11) * 2.0 ** -53
+        rad = math.sqrt(-2.0 * math.log(u1))
+        assert flat[i] == float(np.float16(rad * math.cos(2 * math.pi * u2)))
+        if i + 1 < n:
+            assert flat[i + 1] == float(np.float16(rad * math.sin(2 * math.pi * u2)))
+
+
 # ------------------------------------------------------------------ codebook
 
 def _unit_of_last_digit(text):
