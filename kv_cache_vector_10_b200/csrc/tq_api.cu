@@ -78,6 +78,26 @@ static PFN_encodeTiled get_encode_tiled() {
     return fn;
 }
 
+// 4-D TMA map over caller rows of a 16-bit type, element (b, h, t, j) at
+// base + b sb + h sh + t st + j (strides in elements): dims {d, T, H, batch},
+// box 64 x 128 tokens x 1 x 1, 128-byte swizzle, zero fill past T.  False if
+// the driver rejects the layout (the caller then uses another kernel).
+bool tq_rows_map_4d(CUtensorMap *map, bool bf16, const void *base, int d, int64_t T, int H, int batch, int64_t sb,
+                    int64_t sh, int64_t st) {
+    PFN_encodeTiled enc = get_encode_tiled();
+    if (!enc || T <= 0 || T > 0xFFFFFFFFll) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {(cuuint64_t)st * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+    for (int i = 0; i < 3; ++i)
+        if (strides[i] == 0 || strides[i] % 16 || strides[i] >= (1ull << 40)) return false;
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                     const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 extern "C" {
 
 const char *tq_status_string(tq_status s) {
@@ -170,7 +190,27 @@ void tq_destroy(tq_ctx *ctx) {
     cudaFree(ctx->d_book);
     cudaFree(ctx->d_Q32);
     cudaFree(ctx->d_Qh);
+    cudaFree(ctx->d_HD16);
+    cudaFree(ctx->d_HDbf);
     delete ctx;
+}
+
+// 2-D TMA map over [rows][d] 16-bit entries: box 64 x box_rows, 128-byte swizzle.
+static tq_status encode_rows_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, int d, int64_t rows,
+                                 int box_rows) {
+    PFN_encodeTiled enc = get_encode_tiled();
+    if (!enc) return TQ_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(map, dt, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_cuda_msg, sizeof(g_cuda_msg), "cuTensorMapEncodeTiled failed: %d", (int)r);
+        return TQ_ERR_CUDA;
+    }
+    return TQ_OK;
 }
 
 tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
@@ -249,11 +289,36 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
             }
         }
     }
+    // The Walsh-Hadamard rotation with the head's signs as a +-1 matrix,
+    // B[n][k] = (-1)^popcount(n & k) D[k], in both 16-bit types.
+    uint16_t *nHD16 = nullptr, *nHDbf = nullptr;
+    CUtensorMap hdmap16, hdmapbf;
+    std::memset(&hdmap16, 0, sizeof(hdmap16));
+    std::memset(&hdmapbf, 0, sizeof(hdmapbf));
+    if (st == TQ_OK && ctx->rotation == TQ_ROT_HADAMARD) {
+        const size_t dd = (size_t)d * d;
+        std::vector<uint16_t> h16((size_t)n_heads * dd), hbf((size_t)n_heads * dd);
+        for (int h = 0; h < n_heads; ++h)
+            for (int n = 0; n < d; ++n)
+                for (int k = 0; k < d; ++k) {
+                    const bool neg = (__builtin_popcount((unsigned)(n & k)) & 1) ^ ((signs[(size_t)h * (d / 32) + k / 32] >> (k % 32)) & 1);
+                    h16[(size_t)h * dd + (size_t)n * d + k] = neg ? 0xBC00u : 0x3C00u;   // binary16 -1 / +1
+                    hbf[(size_t)h * dd + (size_t)n * d + k] = neg ? 0xBF80u : 0x3F80u;   // bfloat16 -1 / +1
+                }
+        st = tq_check_cuda(cudaMalloc(&nHD16, h16.size() * 2));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMalloc(&nHDbf, hbf.size() * 2));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nHD16, h16.data(), h16.size() * 2, cudaMemcpyHostToDevice));
+        if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nHDbf, hbf.data(), hbf.size() * 2, cudaMemcpyHostToDevice));
+        if (st == TQ_OK) st = encode_rows_map(&hdmap16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, nHD16, d, (int64_t)n_heads * d, d);
+        if (st == TQ_OK) st = encode_rows_map(&hdmapbf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nHDbf, d, (int64_t)n_heads * d, d);
+    }
     if (st != TQ_OK) {
         cudaFree(nsig);
         cudaFree(nS);
         cudaFree(nQ32);
         cudaFree(nQh);
+        cudaFree(nHD16);
+        cudaFree(nHDbf);
         return st;
     }
     cudaDeviceSynchronize();   // no kernel may still read the old tables
@@ -261,12 +326,18 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
     cudaFree(ctx->d_S);
     cudaFree(ctx->d_Q32);
     cudaFree(ctx->d_Qh);
+    cudaFree(ctx->d_HD16);
+    cudaFree(ctx->d_HDbf);
     ctx->d_signs = nsig;
     ctx->d_S = nS;
     ctx->tmap_S = map;
     ctx->d_Q32 = nQ32;
     ctx->d_Qh = nQh;
     ctx->tmap_Q = qmap;
+    ctx->d_HD16 = nHD16;
+    ctx->d_HDbf = nHDbf;
+    ctx->tmap_HD16 = hdmap16;
+    ctx->tmap_HDbf = hdmapbf;
     ctx->heads_built = n_heads;
     return TQ_OK;
 }

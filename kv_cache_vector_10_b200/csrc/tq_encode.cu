@@ -42,6 +42,8 @@
 // overflows fp32 (|x| beyond ~1.5e18) are counted as non-finite; rows where
 // it falls below the smallest normal float (|x| below ~1e-20) are encoded as
 // zero rows (the exact search steps need normal-range boundaries).
+#include <algorithm>
+#include <cstdlib>
 #include <type_traits>
 
 #include "tq_internal.cuh"
@@ -1117,6 +1119,577 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     }
 }
 
+// ===================================================== TMA-fed encoders
+// For binary16 / bfloat16 rows and the Walsh-Hadamard rotation.  One
+// persistent CTA per SM takes a contiguous range of 128-row tiles (each tile
+// holds rows of one (batch, head)), so the head-dependent operands change
+// only a few times per CTA.
+//
+// The last warp is the producer: one lane requests every tile's rows with
+// 4-D TMA loads into a ring of shared-memory stages and issues the
+// tensor-core work as soon as its inputs are ready (it polls the barriers,
+// never blocking on one of them):
+//   * the rotation U = X B^T with B[n][k] = H[n][k] D[k] (+-1, exact in the
+//     16-bit input type), accumulated in fp32 in TMEM -- the Walsh-Hadamard
+//     transform of the signed row as a dense product: exact products, fp32
+//     sums (the rounding order differs from the butterflies, within float
+//     rounding);
+//   * keys: the QJL projection P = E S^T of the residual operand E written
+//     by a compute group (binary16 hi + lo, two passes, fp32 in TMEM).
+// The other warps form NG groups of four; group g takes tiles g, g + NG, ...
+// of the CTA's range, one thread per row (the TMEM lane of warp w is 32 (w % 4)
+// + lane): it reads the row's rotation from its group's TMEM columns in
+// 32-coordinate chunks, takes |u|^2, quantizes chunk by chunk and stores the
+// packed row.  Keys also stage the signed centroids in TMEM, write the
+// residual operand (one shared buffer, taken in tile order), and store the
+// sign plane once the QJL projection of their tile is done.  The groups run
+// independently of each other, so while one waits for the tensor cores the
+// others issue.
+struct PipeParams {
+    uint8_t *out;           // packed rows of this side
+    int64_t capacity, token_offset, T;
+    int H;
+    int row_bytes;
+    int M;                  // keys: projections
+    int64_t tiles_per_bh, n_tiles;
+    uint32_t s_bytes;       // keys: bytes of head's S tile, (d/64) * m * 128
+    unsigned long long *status;
+    float mag[16];          // positive-half centroid magnitudes
+    float pb[16];           // positive boundaries
+    float cl[8];            // keys: centroid magnitude as a multilinear form in the search bits
+    int norm_f16;
+};
+
+template <int D, bool KEYS>
+struct PipeLayout {
+    static constexpr int NG = KEYS ? 2 : 3;              // compute groups (4 warps each)
+    static constexpr int THREADS = 32 * (4 * NG + 1);    // + the producer warp
+    static constexpr int XBOX = ENC_ROWS * 128;          // one 64-column box of a tile (16 KB)
+    static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
+    static constexpr int NS = KEYS ? 2 : 4;              // stages of the row ring
+    static constexpr int OFF_HD = NS * XSTAGE;           // rotation operand [d/64][d][128 B]
+    static constexpr int OFF_A = OFF_HD + D * D * 2;     // keys: residual operand hi, lo
+    static constexpr int OFF_S = OFF_A + (KEYS ? 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
+    static constexpr int FIXED = 1024 + OFF_S;           // dynamic bytes before S (with alignment slack)
+};
+
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(tqdev::smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait (bounded) by every lane of a warp; true if all of them saw the phase.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase) {
+    const bool ok = tqdev::mbar_wait_bounded(bar, phase);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D, int B, typename Tin, bool KEYS>
+__global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
+    tq_encode_pipe_kernel(const __grid_constant__ PipeParams p, const __grid_constant__ CUtensorMap tmapX,
+                          const __grid_constant__ CUtensorMap tmapHD, const __grid_constant__ CUtensorMap tmapS) {
+    using L = PipeLayout<D, KEYS>;
+    constexpr int NS = L::NS;
+    constexpr int NG = L::NG;
+    constexpr int HB = (1 << B) / 2;             // magnitude cells of the positive half
+    constexpr int NC = D / 32;                   // 32-coordinate chunks per row (= words per key index plane)
+    constexpr int PWARP = 4 * NG;                // the producer warp
+    constexpr bool BF = std::is_same<Tin, __nv_bfloat16>::value;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sX = sm;
+    uint8_t *sHD = sm + L::OFF_HD;
+    uint8_t *sA = sm + L::OFF_A;
+    uint8_t *sS = sm + L::OFF_S;
+    __shared__ __align__(8) uint64_t bar_xfull[NS], bar_xfree[NS], bar_rot[NG], bar_ufree[NG], bar_qjl[NG];
+    __shared__ __align__(8) uint64_t bar_afull, bar_afree, bar_hd, bar_s;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ float s_mag2[16];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t tile_begin = (int64_t)blockIdx.x * p.n_tiles / gridDim.x;
+    const int64_t tile_end = ((int64_t)blockIdx.x + 1) * p.n_tiles / gridDim.x;
+    const int ntile = (int)(tile_end - tile_begin);
+    const int M = KEYS ? p.M : 0;
+    // TMEM: group g's rotation U at g * GSTRIDE, keys' signed centroids C and
+    // then the projections P (C is consumed before the QJL MMA writes P) right after
+    const uint32_t GSTRIDE = KEYS ? (uint32_t)(D + (M > D ? M : D)) : (uint32_t)D;
+    const uint32_t tmem_cols = tmem_cols_for((int)(NG * GSTRIDE));
+
+    if (tid == 0) {
+        for (int i = 0; i < NS; ++i) {
+            tqdev::mbar_init(&bar_xfull[i], 1);
+            tqdev::mbar_init(&bar_xfree[i], 1);
+        }
+        for (int i = 0; i < NG; ++i) {
+            tqdev::mbar_init(&bar_rot[i], 1);
+            tqdev::mbar_init(&bar_ufree[i], 128);
+            tqdev::mbar_init(&bar_qjl[i], 1);
+        }
+        tqdev::mbar_init(&bar_afull, 128);
+        tqdev::mbar_init(&bar_afree, 1);
+        tqdev::mbar_init(&bar_hd, 1);
+        tqdev::mbar_init(&bar_s, 1);
+        s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
+        tqdev::fence_barrier_init();
+    }
+    if (tid < 16) s_mag2[tid] = tid < HB ? p.mag[tid] * p.mag[tid] : 0.f;
+    if (warp == 0) tqdev::tmem_alloc(&s_tmem, tmem_cols);
+    tqdev::tc_fence_before();
+    __syncthreads();
+    tqdev::tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const bool run = !s_abort && ntile > 0;
+
+    if (warp == PWARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && run) {
+            auto head_of = [&](int li) { return (int)(((tile_begin + li) / p.tiles_per_bh) % p.H); };
+            auto issue_x = [&](int li) {
+                const int64_t tile = tile_begin + li, bh = tile / p.tiles_per_bh;
+                const int t0 = (int)((tile % p.tiles_per_bh) * ENC_ROWS);
+                const int h = (int)(bh % p.H), b = (int)(bh / p.H);
+                const int s = li % NS;
+                tqdev::mbar_expect_tx(&bar_xfull[s], (uint32_t)L::XSTAGE);
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a)
+                    tqdev::tma_load_4d(sX + s * L::XSTAGE + a * L::XBOX, &tmapX, a * 64, t0, h, b, &bar_xfull[s]);
+            };
+            const uint32_t idesc_rot = BF ? tqdev::idesc_bf16_f32(D) : tqdev::idesc_f16_f32(D);
+            const uint32_t idesc_qjl = tqdev::idesc_f16_f32(KEYS ? M : 16);
+            int next_rot = 0, next_qjl = 0, next_x = 0, xfree_seen = 0;
+            int hd_head = -1, s_head = -1;               // head of the operand loaded / being loaded
+            bool hd_busy = false, s_busy = false;        // a load in flight
+            uint32_t hd_ph = 0, s_ph = 0;
+            bool ok = true;
+            uint64_t last = tqdev::globaltimer_ns();
+            for (; next_x < NS && next_x < ntile; ++next_x) issue_x(next_x);
+            while (next_rot < ntile || (KEYS && next_qjl < ntile)) {
+                bool progress = false;
+                // ---- rotation of tile next_rot into its group's U
+                if (next_rot < ntile) {
+                    const int li = next_rot, g = li % NG, h = head_of(li);
+                    if (h != hd_head && !hd_busy) {
+                        // the previous rotation (old operand) must be complete
+                        if (li == 0 || mbar_test(&bar_xfree[(li - 1) % NS], (uint32_t)(((li - 1) / NS) & 1))) {
+                            tqdev::mbar_expect_tx(&bar_hd, (uint32_t)(D * D * 2));
+#pragma unroll
+                            for (int a = 0; a < D / 64; ++a)
+                                tqdev::tma_load_2d(sHD + a * D * 128, &tmapHD, a * 64, h * D, &bar_hd);
+                            hd_busy = true;
+                            hd_head = h;
+                            progress = true;
+                        }
+                    }
+                    if (hd_busy && mbar_test(&bar_hd, hd_ph)) {
+                        hd_ph ^= 1;
+                        hd_busy = false;
+                        progress = true;
+                    }
+                    if (h == hd_head && !hd_busy && mbar_test(&bar_xfull[li % NS], (uint32_t)((li / NS) & 1)) &&
+                        (li < NG || mbar_test(&bar_ufree[g], (uint32_t)(((li - NG) / NG) & 1)))) {
+                        tqdev::tc_fence_after();
+                        const uint32_t abase = tqdev::smem_u32(sX + (li % NS) * L::XSTAGE);
+                        const uint32_t bbase = tqdev::smem_u32(sHD);
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t a_addr = abase + (ks / 4) * L::XBOX + (ks % 4) * 32;
+                            const uint32_t b_addr = bbase + (ks / 4) * (D * 128) + (ks % 4) * 32;
+                            tqdev::mma_f16_ss(tmem + (uint32_t)g * GSTRIDE, tqdev::smem_desc_sw128(a_addr),
+                                              tqdev::smem_desc_sw128(b_addr), idesc_rot, ks != 0);
+                        }
+                        tqdev::mma_commit(&bar_rot[g]);
+                        tqdev::mma_commit(&bar_xfree[li % NS]);
+                        ++next_rot;
+                        progress = true;
+                    }
+                }
+                // ---- QJL projection of tile next_qjl (keys)
+                if (KEYS && next_qjl < next_rot) {
+                    const int j = next_qjl, h = head_of(j);
+                    if (h != s_head && !s_busy) {
+                        // the previous projection (old S) must be complete
+                        if (j == 0 || mbar_test(&bar_afree, (uint32_t)((j - 1) & 1))) {
+                            tqdev::mbar_expect_tx(&bar_s, p.s_bytes);
+#pragma unroll
+                            for (int a = 0; a < D / 64; ++a)
+                                tqdev::tma_load_2d(sS + a * M * 128, &tmapS, a * 64, h * M, &bar_s);
+                            s_busy = true;
+                            s_head = h;
+                            progress = true;
+                        }
+                    }
+                    if (s_busy && mbar_test(&bar_s, s_ph)) {
+                        s_ph ^= 1;
+                        s_busy = false;
+                        progress = true;
+                    }
+                    if (h == s_head && !s_busy && mbar_test(&bar_afull, (uint32_t)(j & 1))) {
+                        tqdev::tc_fence_after();
+                        const uint32_t col = (uint32_t)(j % NG) * GSTRIDE + (uint32_t)D;
+#pragma unroll
+                        for (int pass = 0; pass < 2; ++pass) {
+                            const uint32_t abase = tqdev::smem_u32(sA + pass * L::XSTAGE);
+                            const uint32_t bbase = tqdev::smem_u32(sS);
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t a_addr = abase + (ks / 4) * L::XBOX + (ks % 4) * 32;
+                                const uint32_t b_addr = bbase + (ks / 4) * (M * 128) + (ks % 4) * 32;
+                                tqdev::mma_f16_ss(tmem + col, tqdev::smem_desc_sw128(a_addr),
+                                                  tqdev::smem_desc_sw128(b_addr), idesc_qjl, (pass | ks) != 0);
+                            }
+                        }
+                        tqdev::mma_commit(&bar_qjl[j % NG]);
+                        tqdev::mma_commit(&bar_afree);
+                        ++next_qjl;
+                        progress = true;
+                    }
+                }
+                // ---- refill the ring: tile next_x goes where tile next_x - NS was
+                if (next_x < ntile && next_x - NS < next_rot &&
+                    mbar_test(&bar_xfree[next_x % NS], (uint32_t)(((next_x - NS) / NS) & 1))) {
+                    issue_x(next_x);
+                    ++next_x;
+                    xfree_seen = next_x - NS;
+                    progress = true;
+                }
+                if (progress) {
+                    last = tqdev::globaltimer_ns();
+                } else if (tqdev::globaltimer_ns() - last > 200000000ull || tqdev::status_aborted(p.status)) {
+                    ok = false;
+                    break;
+                } else {
+                    __nanosleep(40);                                   // leave the issue slots to the compute warps
+                }
+            }
+            if (!ok) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+            // Drain: every copy and MMA issued is seen complete (bounded) before
+            // the CTA frees its TMEM and shared memory.
+            for (int li = next_rot; li < next_x; ++li)                 // rows requested, never rotated
+                tqdev::mbar_wait_bounded(&bar_xfull[li % NS], (uint32_t)((li / NS) & 1));
+            for (int li = xfree_seen; li < next_rot; ++li)             // rotations not seen through xfree
+                tqdev::mbar_wait_bounded(&bar_xfree[li % NS], (uint32_t)((li / NS) & 1));
+            if (next_qjl > 0) tqdev::mbar_wait_bounded(&bar_afree, (uint32_t)((next_qjl - 1) & 1));
+            if (hd_busy) tqdev::mbar_wait_bounded(&bar_hd, hd_ph);
+            if (s_busy) tqdev::mbar_wait_bounded(&bar_s, s_ph);
+        }
+    } else if (run) {
+        // ------------------------------------------------------------ compute
+        const int g = warp >> 2;                                // group
+        const int row = ((warp & 3) << 5) | lane;               // tile row = TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)g * GSTRIDE;
+        const uint32_t tU = tl, tC = tl + (uint32_t)D;          // keys: C, then P, at tC
+        bool failed = false;
+        for (int li = g, k = 0; li < ntile && !failed; li += NG, ++k) {
+            const int64_t tile = tile_begin + li, bh = tile / p.tiles_per_bh;
+            const int64_t t = (tile % p.tiles_per_bh) * ENC_ROWS + row;
+            const bool valid = t < p.T;
+            uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
+            if (!warp_wait(&bar_rot[g], (uint32_t)(k & 1))) {
+                failed = true;
+                break;
+            }
+            tqdev::tc_fence_after();
+            // ---- |u|^2 over the row
+            float2 n2p = make_float2(0.f, 0.f);
+#pragma unroll 1
+            for (int c = 0; c < NC; ++c) {
+                float u[32];
+                tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) n2p = fma2(make_float2(u[i], u[i + 1]), make_float2(u[i], u[i + 1]), n2p);
+            }
+            const float n2 = n2p.x + n2p.y;
+            const bool nonfinite = !(n2 <= 3.0e38f);
+            const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
+            if (valid && nonfinite) atomicAdd(&p.status[0], 1ull);
+            const float n = sqrtf(n2 * (1.f / D));
+            float c2 = 0.f;
+            if constexpr (!KEYS) {
+                // ---- values: quantize chunk by chunk, B-bit fields
+                constexpr uint32_t FMASK = (1u << B) - 1u;
+                if constexpr (HB <= 8) {
+                    float rb[8];
+                    row_bounds<HB>(n, p.pb, rb);
+                    int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                    const float magic = 8388608.0f + (float)HB;
+#pragma unroll 1
+                    for (int c = 0; c < NC; ++c) {
+                        float u[32];
+                        tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
+                        uint32_t f[B], S[3] = {0u, 0u, 0u};
+#pragma unroll
+                        for (int w = 0; w < B; ++w) f[w] = 0u;
+#pragma unroll
+                        for (int j = 15; j >= 0; --j) {
+                            const float2 A = make_float2(fabsf(u[2 * j]), fabsf(u[2 * j + 1]));
+                            float2 T[3], dd[3];
+                            search2<HB>(A, rb, T, dd);
+                            float2 K = add2(T[0], dup2(magic));
+                            if constexpr (HB >= 4) K = fma2(T[1], dup2(2.f), K);
+                            if constexpr (HB >= 8) K = fma2(T[2], dup2(4.f), K);
+#pragma unroll
+                            for (int hh = 1; hh >= 0; --hh) {
+                                const int i = 2 * j + hh;
+                                const uint32_t kb = __float_as_uint(hh ? K.y : K.x);
+                                const uint32_t sg = (uint32_t)((int32_t)__float_as_uint(u[i]) >> 31);
+                                const uint32_t idx = (kb ^ sg) & FMASK;
+                                const int bit = B * i;
+                                f[bit / 32] |= idx << (bit % 32);
+                                if ((bit % 32) + B > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
+#pragma unroll
+                                for (int l = 0; l < Levels<HB>::L; ++l) S[l] = push_sign(S[l], hh ? dd[l].y : dd[l].x);
+                            }
+                        }
+                        count_cells<HB>(S, cnt);
+                        if (valid) {
+#pragma unroll
+                            for (int w = 0; w < B; ++w) dst[B * c + w] = degenerate ? degenerate_field_word<B>(B * c + w) : f[w];
+                        }
+                    }
+                    int rest = D;
+#pragma unroll
+                    for (int kc = 1; kc < HB; ++kc) {
+                        rest -= cnt[kc];
+                        c2 = fmaf((float)cnt[kc], s_mag2[kc], c2);
+                    }
+                    c2 = fmaf((float)rest, s_mag2[0], c2);
+                } else {
+                    float nb[16];
+#pragma unroll
+                    for (int kc = 0; kc < HB - 1; ++kc) nb[kc] = n * p.pb[kc];
+#pragma unroll 1
+                    for (int c = 0; c < NC; ++c) {
+                        float u[32];
+                        tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
+                        uint32_t f[B];
+#pragma unroll
+                        for (int w = 0; w < B; ++w) f[w] = 0u;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const uint32_t cell = mag_index<HB>(fabsf(u[i]), nb);
+                            const uint32_t idx = u[i] < 0.f ? (uint32_t)(HB - 1) - cell : (uint32_t)HB + cell;
+                            c2 += s_mag2[cell];
+                            const int bit = B * i;
+                            f[bit / 32] |= idx << (bit % 32);
+                            if ((bit % 32) + B > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int w = 0; w < B; ++w) dst[B * c + w] = degenerate ? degenerate_field_word<B>(B * c + w) : f[w];
+                        }
+                    }
+                }
+                tqdev::tc_fence_before();
+                tqdev::mbar_arrive(&bar_ufree[g]);                    // U read for the last time
+                if (valid) dst[B * NC] = __float_as_uint(degenerate ? 0.f : n * sqrtf((float)D / c2));
+            } else {
+                // ---- keys: index planes, signed centroids to TMEM C, sum C^2, sum |u| C
+                float rb[8];
+                row_bounds<HB>(n, p.pb, rb);
+                int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                float2 ucp = make_float2(0.f, 0.f);
+#pragma unroll 1
+                for (int c = 0; c < NC; ++c) {
+                    float u[32];
+                    tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
+                    uint32_t S[3] = {0u, 0u, 0u}, Sn = 0u;
+#pragma unroll
+                    for (int j = 15; j >= 0; --j) {
+                        const float2 A = make_float2(fabsf(u[2 * j]), fabsf(u[2 * j + 1]));
+                        float2 T[3], dd[3];
+                        search2<HB>(A, rb, T, dd);
+                        float2 cm;
+                        if constexpr (HB == 1) {
+                            cm = dup2(p.cl[0]);
+                        } else if constexpr (HB == 2) {
+                            cm = fma2(T[0], dup2(p.cl[0]), dup2(p.cl[1]));
+                        } else if constexpr (HB == 4) {
+                            const float2 lo = fma2(T[1], dup2(p.cl[0]), dup2(p.cl[1]));
+                            const float2 df = fma2(T[1], dup2(p.cl[2]), dup2(p.cl[3]));
+                            cm = fma2(T[0], df, lo);
+                        } else {
+                            const float2 lo = fma2(T[1], fma2(T[2], dup2(p.cl[0]), dup2(p.cl[1])),
+                                                   fma2(T[2], dup2(p.cl[2]), dup2(p.cl[3])));
+                            const float2 df = fma2(T[1], fma2(T[2], dup2(p.cl[4]), dup2(p.cl[5])),
+                                                   fma2(T[2], dup2(p.cl[6]), dup2(p.cl[7])));
+                            cm = fma2(T[0], df, lo);
+                        }
+                        ucp = fma2(A, cm, ucp);
+#pragma unroll
+                        for (int hh = 1; hh >= 0; --hh) {
+#pragma unroll
+                            for (int l = 0; l < Levels<HB>::L; ++l) S[l] = push_sign(S[l], hh ? dd[l].y : dd[l].x);
+                            Sn = push_sign(Sn, u[2 * j + hh]);
+                        }
+                        u[2 * j] = copysignf(cm.x, u[2 * j]);
+                        u[2 * j + 1] = copysignf(cm.y, u[2 * j + 1]);
+                    }
+                    tqdev::tmem_st_32x32b_x32(tC + 32 * c, u);   // signed centroids
+                    count_cells<HB>(S, cnt);
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < B - 1; ++q)
+                            dst[q * NC + c] = degenerate ? (((HB >> q) & 1) ? ~0u : 0u) : (~S[q] ^ Sn);
+                        dst[(B - 1) * NC + c] = degenerate ? ~0u : ~Sn;
+                    }
+                }
+                tqdev::tmem_wait_st();
+                {
+                    int rest = D;
+#pragma unroll
+                    for (int kc = 1; kc < HB; ++kc) {
+                        rest -= cnt[kc];
+                        c2 = fmaf((float)cnt[kc], s_mag2[kc], c2);
+                    }
+                    c2 = fmaf((float)rest, s_mag2[0], c2);
+                }
+                const float uc = ucp.x + ucp.y;
+                const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
+                // |e|^2 from the sums, only to scale the MMA operand
+                float e2a = n2 - 2.f * ns * uc + ns * ns * c2;
+                e2a = fmaxf(e2a, 1e-10f * n2);
+                const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
+                // ---- residual operand (the shared buffer is taken in tile order)
+                if (li > 0 && !warp_wait(&bar_afree, (uint32_t)((li - 1) & 1))) {
+                    failed = true;
+                    break;
+                }
+                float2 e2p = make_float2(0.f, 0.f);
+#pragma unroll 1
+                for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float uu[16], cv[16];
+                        tqdev::tmem_ld_32x32b_x16_nowait(tU + 32 * c + 16 * half, uu);
+                        tqdev::tmem_ld_32x32b_x16_nowait(tC + 32 * c + 16 * half, cv);
+                        tqdev::tmem_wait_ld();
+#pragma unroll
+                        for (int jh = 0; jh < 2; ++jh) {
+                            uint32_t hw[4], lw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 8 * jh + 2 * e;
+                                const float2 E = fma2(dup2(-ns), make_float2(cv[i], cv[i + 1]), make_float2(uu[i], uu[i + 1]));
+                                e2p = fma2(E, E, e2p);
+                                const float2 a = mul2(E, dup2(sc));
+                                const __half2 hh = __floats2half2_rn(a.x, a.y);
+                                const float2 l = sub2(a, __half22float2(hh));
+                                const __half2 ll = __floats2half2_rn(l.x, l.y);
+                                hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                                lw[e] = *reinterpret_cast<const uint32_t *>(&ll);
+                            }
+                            const int kk = 4 * c + 2 * half + jh;             // 16-byte unit of the row
+                            const int off = (kk / 8) * L::XBOX + row * 128 + (((kk % 8) ^ (row & 7)) << 4);
+                            *reinterpret_cast<uint4 *>(sA + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                            *reinterpret_cast<uint4 *>(sA + L::XSTAGE + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                        }
+                    }
+                }
+                tqdev::tc_fence_before();
+                tqdev::mbar_arrive(&bar_ufree[g]);                    // U read for the last time
+                tqdev::fence_proxy_async_smem();
+                tqdev::mbar_arrive(&bar_afull);                       // residual operand written
+                const float e2 = e2p.x + e2p.y;
+                bool zero_row = degenerate;
+                const int tail = B * NC + M / 32;
+                const float gv = degenerate ? 0.f : sqrtf(e2 * (1.f / D));
+                if (p.norm_f16) {
+                    uint32_t w;
+                    if (!tqdev::pack_norms_f16(ns, gv, w)) {
+                        // binary16 overflow: the zero row, counted with the non-finite rows
+                        zero_row = true;
+                        w = 0u;
+                        if (valid) {
+                            atomicAdd(&p.status[0], 1ull);
+#pragma unroll 1
+                            for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                                for (int q = 0; q < B - 1; ++q) dst[q * NC + c] = ((HB >> q) & 1) ? ~0u : 0u;
+                                dst[(B - 1) * NC + c] = ~0u;
+                            }
+                        }
+                    }
+                    if (valid) dst[tail] = w;
+                } else if (valid) {
+                    dst[tail] = __float_as_uint(ns);
+                    dst[tail + 1] = __float_as_uint(gv);
+                }
+                // ---- sign plane from this tile's projections
+                if (!warp_wait(&bar_qjl[g], (uint32_t)(k & 1))) {
+                    failed = true;
+                    break;
+                }
+                tqdev::tc_fence_after();
+                uint32_t *sdst = dst + B * NC;
+#pragma unroll 1
+                for (int c = 0; c < M / 32; ++c) {
+                    uint32_t neg = 0u;
+#pragma unroll
+                    for (int half = 1; half >= 0; --half) {
+                        float pv[16];
+                        tqdev::tmem_ld_32x32b_x16_nowait(tC + 32 * c + 16 * half, pv);
+                        tqdev::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 7; j >= 0; --j) {
+                            const float2 q = add2(make_float2(pv[2 * j], pv[2 * j + 1]), dup2(0.f));
+                            neg = push_sign(neg, q.y);
+                            neg = push_sign(neg, q.x);
+                        }
+                    }
+                    if (valid) sdst[c] = zero_row ? ~0u : ~neg;
+                }
+                tqdev::tc_fence_before();
+            }
+        }
+        if (failed && lane == 0) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
+    }
+    tqdev::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tqdev::tc_fence_after();
+        tqdev::tmem_dealloc(tmem, tmem_cols);
+    }
+}
+
+template <int D, typename Tin, bool KEYS>
+cudaError_t launch_pipe(int B, const PipeParams &p, const CUtensorMap &mx, const CUtensorMap &mhd,
+                        const CUtensorMap &ms, int grid, cudaStream_t s) {
+    using L = PipeLayout<D, KEYS>;
+    cudaError_t e = cudaSuccess;
+    auto go = [&](auto kern) {
+        size_t smem = (size_t)L::FIXED + (KEYS ? p.s_bytes : 0);
+        // one CTA per SM: a second one could wait in tcgen05.alloc until the
+        // first exits (the grid is one CTA per SM anyway)
+        if (smem < 120 * 1024) smem = 120 * 1024;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        kern<<<grid, L::THREADS, smem, s>>>(p, mx, mhd, ms);
+        e = cudaGetLastError();
+    };
+    switch (B) {
+        case 1: if constexpr (KEYS) go(tq_encode_pipe_kernel<D, 1, Tin, KEYS>); else return cudaErrorInvalidValue; break;
+        case 2: go(tq_encode_pipe_kernel<D, 2, Tin, KEYS>); break;
+        case 3: go(tq_encode_pipe_kernel<D, 3, Tin, KEYS>); break;
+        case 4: go(tq_encode_pipe_kernel<D, 4, Tin, KEYS>); break;
+        case 5: if constexpr (!KEYS) go(tq_encode_pipe_kernel<D, 5, Tin, KEYS>); else return cudaErrorInvalidValue; break;
+        default: return cudaErrorInvalidValue;
+    }
+    return e;
+}
+
 template <int D, typename Tin, int ROT>
 cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &mapS, const CUtensorMap &mapQ, int64_t grid,
                      cudaStream_t s) {
@@ -1189,10 +1762,126 @@ cudaError_t launch_side(const tq_ctx *ctx, bool keys, const EncodeParams &p, int
 
 }  // namespace
 
+// The key centroid magnitude C_k of cell k = sum_L T_L 2^L written as the
+// multilinear form the key kernels evaluate in the search bits T_L
+// (cb: the 2 HB centroids, ascending; cl: the form's 8 coefficients).
+static void key_centroid_form(const float *cb, int HB, float *cl) {
+    double m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int i = 0; i < HB && i < 8; ++i) m[i] = cb[HB + i];
+    double c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (HB == 1) {
+        c[0] = m[0];
+    } else if (HB == 2) {
+        c[0] = m[1] - m[0];
+        c[1] = m[0];
+    } else if (HB == 4) {
+        c[0] = m[2] - m[0];
+        c[1] = m[0];
+        c[2] = (m[3] - m[2]) - (m[1] - m[0]);
+        c[3] = m[1] - m[0];
+    } else if (HB == 8) {
+        const double d0 = m[1] - m[0], d2 = m[3] - m[2], d4 = m[5] - m[4], d6 = m[7] - m[6];
+        c[0] = m[6] - m[4] - m[2] + m[0];
+        c[1] = m[2] - m[0];
+        c[2] = m[4] - m[0];
+        c[3] = m[0];
+        c[4] = d6 - d4 - d2 + d0;
+        c[5] = d2 - d0;
+        c[6] = d4 - d0;
+        c[7] = d0;
+    }
+    for (int i = 0; i < 8; ++i) cl[i] = (float)c[i];
+}
+
+// Which encoder serves 16-bit Walsh-Hadamard rows: 0 = the TMA-fed
+// persistent kernels where they apply (default), 1 = the per-thread
+// Walsh-Hadamard kernels always.  Read once from TQ_ENCODE_PATH.
+static int tq_encode_path() {
+    static const int v = [] {
+        const char *e = getenv("TQ_ENCODE_PATH");
+        return (e && e[0] == '1') ? 1 : 0;
+    }();
+    return v;
+}
+
+bool tq_rows_map_4d(CUtensorMap *map, bool bf16, const void *base, int d, int64_t T, int H, int batch, int64_t sb,
+                    int64_t sh, int64_t st);
+
+// The TMA-fed encoder of one side, when it serves the call: 16-bit rows,
+// the Walsh-Hadamard rotation, d in {64, 128}, and its shared memory and
+// TMEM columns fit.  Returns false (nothing launched) otherwise.
+static bool pipe_side(tq_ctx *ctx, bool keys, const void *x, tq_dtype dtype, int batch, int H, int64_t T, int64_t sb,
+                      int64_t sh, int64_t st, const tq_codes *codes, int64_t token_offset, cudaStream_t stream,
+                      int n_sms, cudaError_t *err) {
+    if (dtype == TQ_F32 || ctx->rotation != TQ_ROT_HADAMARD || (ctx->d != 64 && ctx->d != 128)) return false;
+    if (!ctx->d_HD16 || !ctx->d_HDbf) return false;
+    const int d = ctx->d, M = ctx->m;
+    if (keys) {
+        if (2 * (d + std::max(d, M)) > 512) return false;   // two groups' TMEM columns
+        const size_t smem = (d == 128 ? PipeLayout<128, true>::FIXED : PipeLayout<64, true>::FIXED) + (size_t)(d / 64) * M * 128;
+        if (smem > 227 * 1024) return false;
+    }
+    if (T > 0x7FFFFFFF - ENC_ROWS) return false;
+    CUtensorMap mx;
+    if (!tq_rows_map_4d(&mx, dtype == TQ_BF16, x, d, T, H, batch, sb, sh, st)) return false;
+    PipeParams p{};
+    p.out = static_cast<uint8_t *>(keys ? codes->k : codes->v);
+    p.capacity = codes->capacity;
+    p.token_offset = token_offset;
+    p.T = T;
+    p.H = H;
+    p.row_bytes = (int)tq_row_bytes(ctx, keys ? TQ_KEYS : TQ_VALUES);
+    p.M = M;
+    p.tiles_per_bh = (T + ENC_ROWS - 1) / ENC_ROWS;
+    p.n_tiles = p.tiles_per_bh * (int64_t)batch * H;
+    p.s_bytes = (uint32_t)((d / 64) * M * 128);
+    p.status = ctx->d_status;
+    p.norm_f16 = ctx->norm_f16;
+    const int Bq = keys ? ctx->BK : ctx->BV;
+    const float *cb = keys ? ctx->ck : ctx->cv;
+    const float *bd = keys ? ctx->bk : ctx->bv;
+    const int HBq = (1 << Bq) / 2;
+    for (int i = 0; i < HBq; ++i) p.mag[i] = cb[HBq + i];
+    for (int i = 0; i + 1 < HBq; ++i) p.pb[i] = bd[HBq + i];
+    if (keys) key_centroid_form(cb, HBq, p.cl);
+    const int grid = (int)std::min<int64_t>(p.n_tiles, n_sms > 0 ? n_sms : 148);
+    const CUtensorMap &mhd = dtype == TQ_BF16 ? ctx->tmap_HDbf : ctx->tmap_HD16;
+    cudaError_t e;
+    if (d == 128) {
+        e = dtype == TQ_BF16 ? (keys ? launch_pipe<128, __nv_bfloat16, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                                     : launch_pipe<128, __nv_bfloat16, false>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream))
+                             : (keys ? launch_pipe<128, __half, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                                     : launch_pipe<128, __half, false>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream));
+    } else {
+        e = dtype == TQ_BF16 ? (keys ? launch_pipe<64, __nv_bfloat16, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                                     : launch_pipe<64, __nv_bfloat16, false>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream))
+                             : (keys ? launch_pipe<64, __half, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                                     : launch_pipe<64, __half, false>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream));
+    }
+    *err = e;
+    return true;
+}
+
 tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype dtype, int batch, int H,
                            int64_t T, int64_t sb, int64_t sh, int64_t st, const tq_codes *codes,
                            int64_t token_offset, cudaStream_t stream, int n_sms) {
-    (void)n_sms;
+    if (tq_encode_path() != 1) {
+        bool done_k = !k, done_v = !v;
+        for (int side = 0; side < 2; ++side) {
+            const bool keys = side == 0;
+            const void *x = keys ? k : v;
+            if (!x) continue;
+            cudaError_t e = cudaSuccess;
+            if (pipe_side(ctx, keys, x, dtype, batch, H, T, sb, sh, st, codes, token_offset, stream, n_sms, &e)) {
+                tq_status s = tq_check_cuda(e);
+                if (s != TQ_OK) return s;
+                (keys ? done_k : done_v) = true;
+            }
+        }
+        if (done_k && done_v) return TQ_OK;
+        if (done_k) k = nullptr;
+        if (done_v) v = nullptr;
+    }
     const int64_t blocks_per_bh = (T + ENC_TILES * ENC_ROWS - 1) / (ENC_TILES * ENC_ROWS);
     const int64_t grid = blocks_per_bh * (int64_t)batch * H;
     if (grid == 0) return TQ_OK;
@@ -1223,35 +1912,7 @@ tq_status tq_launch_encode(tq_ctx *ctx, const void *k, const void *v, tq_dtype d
         const int HB = (1 << B) / 2;
         for (int i = 0; i < HB; ++i) p.mag[i] = cb[HB + i];
         for (int i = 0; i + 1 < HB; ++i) p.pb[i] = bd[HB + i];
-        if (keys) {
-            // cell k = sum_L T_L 2^L; the magnitude C_k written as the
-            // multilinear form the key kernel evaluates in the bits T_L
-            double m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            for (int i = 0; i < HB && i < 8; ++i) m[i] = cb[HB + i];
-            double c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (HB == 1) {
-                c[0] = m[0];
-            } else if (HB == 2) {
-                c[0] = m[1] - m[0];
-                c[1] = m[0];
-            } else if (HB == 4) {
-                c[0] = m[2] - m[0];
-                c[1] = m[0];
-                c[2] = (m[3] - m[2]) - (m[1] - m[0]);
-                c[3] = m[1] - m[0];
-            } else if (HB == 8) {
-                const double d0 = m[1] - m[0], d2 = m[3] - m[2], d4 = m[5] - m[4], d6 = m[7] - m[6];
-                c[0] = m[6] - m[4] - m[2] + m[0];
-                c[1] = m[2] - m[0];
-                c[2] = m[4] - m[0];
-                c[3] = m[0];
-                c[4] = d6 - d4 - d2 + d0;
-                c[5] = d2 - d0;
-                c[6] = d4 - d0;
-                c[7] = d0;
-            }
-            for (int i = 0; i < 8; ++i) p.cl[i] = (float)c[i];
-        }
+        if (keys) key_centroid_form(cb, HB, p.cl);
         cudaError_t e;
         switch (dtype) {
             case TQ_F32: e = launch_side<float>(ctx, keys, p, grid, stream); break;

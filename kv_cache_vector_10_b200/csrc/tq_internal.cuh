@@ -40,6 +40,12 @@ struct tq_ctx {
     float *d_Q32;
     __half *d_Qh;
     CUtensorMap tmap_Q;
+    // Walsh-Hadamard rotation as a tensor-core operand: B[h][n][k] = H[n][k] D_h[k]
+    // (+-1, exact in both 16-bit types), binary16 and bfloat16 copies
+    // [heads][d][d], with TMA maps (inner d, outer heads*d rows, box 64 x d,
+    // 128-byte swizzle).  Built for TQ_ROT_HADAMARD contexts.
+    uint16_t *d_HD16, *d_HDbf;
+    CUtensorMap tmap_HD16, tmap_HDbf;
 };
 
 // Positive halves of the codebooks: magnitudes of the centroids and the
@@ -127,6 +133,21 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+// 4-D tiled bulk tensor load (no multicast), completion on an mbarrier.
+__device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Named barrier `id` over `nthreads` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0).
@@ -226,6 +247,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8_nowait(uint32_t taddr, float (
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Each thread of the warp reads 16 consecutive 32-bit columns of its lane (no wait).
+__device__ __forceinline__ void tmem_ld_32x32b_x16_nowait(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -300,6 +334,10 @@ __device__ __forceinline__ float2 key_norms(const uint32_t *tail, bool f16) {
 
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+// The same with A and B in bfloat16.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
+    return idesc_f16_f32(n) | (1u << 7) | (1u << 10);
 }
 
 }  // namespace tqdev
