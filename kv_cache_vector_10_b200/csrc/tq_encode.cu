@@ -1145,6 +1145,42 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
 // sign plane once the QJL projection of their tile is done.  The groups run
 // independently of each other, so while one waits for the tensor cores the
 // others issue.
+// B-bit index fields of 32 coordinates (coordinate j at bit B j of f[0..B),
+// little-endian) from the B index planes (bit j of P[q] = bit q of index j),
+// for B in {2, 3, 4}; spread[x] holds bit i of the byte x at bit B i.
+template <int B>
+__device__ __forceinline__ void fields_from_planes(const uint32_t (&P)[B], const uint32_t *spread, uint32_t (&f)[B]) {
+    if constexpr (B == 2 || B == 4) {
+        // a byte of the planes covers 8 coordinates = 8 B bits
+        constexpr int PARTS = B == 2 ? 2 : 1;   // plane bytes per output word
+#pragma unroll
+        for (int w = 0; w < B; ++w) {
+            uint32_t acc = 0u;
+#pragma unroll
+            for (int part = 0; part < PARTS; ++part) {
+                const int byte = (B == 4) ? w : 2 * w + part;
+                uint32_t g = 0u;
+#pragma unroll
+                for (int q = 0; q < B; ++q) g |= spread[(P[q] >> (8 * byte)) & 0xFFu] << q;
+                acc |= (B == 4) ? g : g << (16 * part);
+            }
+            f[w] = acc;
+        }
+    } else if constexpr (B == 3) {
+        // 8 coordinates = 24 bits; the four 24-bit groups straddle the words
+        uint32_t g[4];
+#pragma unroll
+        for (int byte = 0; byte < 4; ++byte) {
+            g[byte] = 0u;
+#pragma unroll
+            for (int q = 0; q < 3; ++q) g[byte] |= spread[(P[q] >> (8 * byte)) & 0xFFu] << q;
+        }
+        f[0] = g[0] | (g[1] << 24);
+        f[1] = (g[1] >> 8) | (g[2] << 16);
+        f[2] = (g[2] >> 16) | (g[3] << 8);
+    }
+}
+
 struct PipeParams {
     uint8_t *out;           // packed rows of this side
     int64_t capacity, token_offset, T;
@@ -1214,8 +1250,17 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_mag2[16];
+    __shared__ uint32_t s_spread[KEYS ? 1 : 256];   // values: bit i of a byte -> bit B i
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if constexpr (!KEYS) {
+        for (int i = tid; i < 256; i += blockDim.x) {
+            uint32_t v = 0u;
+            if (B <= 4)
+                for (int bit = 0; bit < 8; ++bit) v |= ((uint32_t)(i >> bit) & 1u) << (B * bit);
+            s_spread[i] = v;
+        }
+    }
     const int64_t tile_begin = (int64_t)blockIdx.x * p.n_tiles / gridDim.x;
     const int64_t tile_end = ((int64_t)blockIdx.x + 1) * p.n_tiles / gridDim.x;
     const int ntile = (int)(tile_end - tile_begin);
@@ -1399,14 +1444,21 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                 break;
             }
             tqdev::tc_fence_after();
-            // ---- |u|^2 over the row
+            // ---- |u|^2 over the row (the next chunk's load in flight meanwhile)
             float2 n2p = make_float2(0.f, 0.f);
-#pragma unroll 1
-            for (int c = 0; c < NC; ++c) {
-                float u[32];
-                tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
+            {
+                float ua[32], ub[32];
+                tqdev::tmem_ld_32x32b_x32(tU, ua);
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) n2p = fma2(make_float2(u[i], u[i + 1]), make_float2(u[i], u[i + 1]), n2p);
+                for (int c = 0; c < NC; ++c) {
+                    float(&cur)[32] = (c & 1) ? ub : ua;
+                    float(&nxt)[32] = (c & 1) ? ua : ub;
+                    if (c + 1 < NC) tqdev::tmem_ld_32x32b_x32_nowait(tU + 32 * (c + 1), nxt);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2)
+                        n2p = fma2(make_float2(cur[i], cur[i + 1]), make_float2(cur[i], cur[i + 1]), n2p);
+                    if (c + 1 < NC) tqdev::tmem_wait_ld();
+                }
             }
             const float n2 = n2p.x + n2p.y;
             const bool nonfinite = !(n2 <= 3.0e38f);
@@ -1418,39 +1470,40 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                 // ---- values: quantize chunk by chunk, B-bit fields
                 constexpr uint32_t FMASK = (1u << B) - 1u;
                 if constexpr (HB <= 8) {
+                    // The search's level words give the cell bits of all 32
+                    // coordinates (bit j of S[l] set: level l's test failed),
+                    // so the B index planes are word operations; the fields
+                    // are the planes' bits interleaved, byte by byte through
+                    // the spread table (bit i of a byte to bit B i).
                     float rb[8];
                     row_bounds<HB>(n, p.pb, rb);
                     int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                    const float magic = 8388608.0f + (float)HB;
 #pragma unroll 1
                     for (int c = 0; c < NC; ++c) {
                         float u[32];
                         tqdev::tmem_ld_32x32b_x32(tU + 32 * c, u);
-                        uint32_t f[B], S[3] = {0u, 0u, 0u};
-#pragma unroll
-                        for (int w = 0; w < B; ++w) f[w] = 0u;
+                        uint32_t S[3] = {0u, 0u, 0u}, Sn = 0u;
 #pragma unroll
                         for (int j = 15; j >= 0; --j) {
                             const float2 A = make_float2(fabsf(u[2 * j]), fabsf(u[2 * j + 1]));
                             float2 T[3], dd[3];
                             search2<HB>(A, rb, T, dd);
-                            float2 K = add2(T[0], dup2(magic));
-                            if constexpr (HB >= 4) K = fma2(T[1], dup2(2.f), K);
-                            if constexpr (HB >= 8) K = fma2(T[2], dup2(4.f), K);
 #pragma unroll
                             for (int hh = 1; hh >= 0; --hh) {
-                                const int i = 2 * j + hh;
-                                const uint32_t kb = __float_as_uint(hh ? K.y : K.x);
-                                const uint32_t sg = (uint32_t)((int32_t)__float_as_uint(u[i]) >> 31);
-                                const uint32_t idx = (kb ^ sg) & FMASK;
-                                const int bit = B * i;
-                                f[bit / 32] |= idx << (bit % 32);
-                                if ((bit % 32) + B > 32) f[bit / 32 + 1] |= idx >> (32 - bit % 32);
 #pragma unroll
                                 for (int l = 0; l < Levels<HB>::L; ++l) S[l] = push_sign(S[l], hh ? dd[l].y : dd[l].x);
+                                Sn = push_sign(Sn, u[2 * j + hh]);
                             }
                         }
                         count_cells<HB>(S, cnt);
+                        // index plane q: ascending index = top bit non-negative,
+                        // low bits the cell, complemented for negative values
+                        uint32_t P[B];
+#pragma unroll
+                        for (int q = 0; q < B - 1; ++q) P[q] = ~S[q] ^ Sn;
+                        P[B - 1] = ~Sn;
+                        uint32_t f[B];
+                        fields_from_planes<B>(P, s_spread, f);
                         if (valid) {
 #pragma unroll
                             for (int w = 0; w < B; ++w) dst[B * c + w] = degenerate ? degenerate_field_word<B>(B * c + w) : f[w];
@@ -1639,12 +1692,10 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                         float pv[16];
                         tqdev::tmem_ld_32x32b_x16_nowait(tC + 32 * c + 16 * half, pv);
                         tqdev::tmem_wait_ld();
+                        // bit i = [p_i >= 0] from the sign bit; an exact zero (of
+                        // either sign) lies inside the decision band of p = 0
 #pragma unroll
-                        for (int j = 7; j >= 0; --j) {
-                            const float2 q = add2(make_float2(pv[2 * j], pv[2 * j + 1]), dup2(0.f));
-                            neg = push_sign(neg, q.y);
-                            neg = push_sign(neg, q.x);
-                        }
+                        for (int j = 15; j >= 0; --j) neg = push_sign(neg, pv[j]);
                     }
                     if (valid) sdst[c] = zero_row ? ~0u : ~neg;
                 }
