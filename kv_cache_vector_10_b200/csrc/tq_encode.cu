@@ -1196,9 +1196,11 @@ struct PipeParams {
     int norm_f16;
 };
 
-template <int D, bool KEYS>
+template <int D, bool KEYS, int B>
 struct PipeLayout {
-    static constexpr int NG = KEYS ? 2 : 3;              // compute groups (4 warps each)
+    // compute groups of 4 warps: keys hold U and C/P (2 x 128 TMEM columns)
+    // per group; 4-bit values need more registers than four groups leave
+    static constexpr int NG = KEYS ? 2 : (B == 4 ? 3 : 4);
     static constexpr int THREADS = 32 * (4 * NG + 1);    // + the producer warp
     static constexpr int XBOX = ENC_ROWS * 128;          // one 64-column box of a tile (16 KB)
     static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
@@ -1229,10 +1231,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase) {
 }
 
 template <int D, int B, typename Tin, bool KEYS>
-__global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
+__global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
     tq_encode_pipe_kernel(const __grid_constant__ PipeParams p, const __grid_constant__ CUtensorMap tmapX,
                           const __grid_constant__ CUtensorMap tmapHD, const __grid_constant__ CUtensorMap tmapS) {
-    using L = PipeLayout<D, KEYS>;
+    using L = PipeLayout<D, KEYS, B>;
     constexpr int NS = L::NS;
     constexpr int NG = L::NG;
     constexpr int HB = (1 << B) / 2;             // magnitude cells of the positive half
@@ -1264,6 +1266,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
     const int64_t tile_begin = (int64_t)blockIdx.x * p.n_tiles / gridDim.x;
     const int64_t tile_end = ((int64_t)blockIdx.x + 1) * p.n_tiles / gridDim.x;
     const int ntile = (int)(tile_end - tile_begin);
+    const uint32_t tpb = (uint32_t)p.tiles_per_bh;
     const int M = KEYS ? p.M : 0;
     // TMEM: group g's rotation U at g * GSTRIDE, keys' signed centroids C and
     // then the projections P (C is consumed before the QJL MMA writes P) right after
@@ -1298,10 +1301,12 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
     if (warp == PWARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0 && run) {
-            auto head_of = [&](int li) { return (int)(((tile_begin + li) / p.tiles_per_bh) % p.H); };
+            // tile indices fit in 32 bits (the launcher checks), so the
+            // divisions are 32-bit ones
+            auto head_of = [&](int li) { return (int)(((uint32_t)(tile_begin + li) / tpb) % (uint32_t)p.H); };
             auto issue_x = [&](int li) {
-                const int64_t tile = tile_begin + li, bh = tile / p.tiles_per_bh;
-                const int t0 = (int)((tile % p.tiles_per_bh) * ENC_ROWS);
+                const uint32_t tile = (uint32_t)(tile_begin + li), bh = tile / tpb;
+                const int t0 = (int)((tile - bh * tpb) * ENC_ROWS);
                 const int h = (int)(bh % p.H), b = (int)(bh / p.H);
                 const int s = li % NS;
                 tqdev::mbar_expect_tx(&bar_xfull[s], (uint32_t)L::XSTAGE);
@@ -1316,7 +1321,8 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
             bool hd_busy = false, s_busy = false;        // a load in flight
             uint32_t hd_ph = 0, s_ph = 0;
             bool ok = true;
-            uint64_t last = tqdev::globaltimer_ns();
+            uint64_t last = 0;
+            uint32_t idle = 0;
             for (; next_x < NS && next_x < ntile; ++next_x) issue_x(next_x);
             while (next_rot < ntile || (KEYS && next_qjl < ntile)) {
                 bool progress = false;
@@ -1407,13 +1413,17 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                     xfree_seen = next_x - NS;
                     progress = true;
                 }
+                // poll shared-memory barriers only; the wall clock is read every
+                // 256 idle rounds (the abort flag was read at the CTA's start)
                 if (progress) {
-                    last = tqdev::globaltimer_ns();
-                } else if (tqdev::globaltimer_ns() - last > 200000000ull || tqdev::status_aborted(p.status)) {
-                    ok = false;
-                    break;
-                } else {
-                    __nanosleep(40);                                   // leave the issue slots to the compute warps
+                    idle = 0;
+                } else if ((++idle & 255) == 0) {
+                    const uint64_t now = tqdev::globaltimer_ns();
+                    if (idle == 256) last = now;
+                    else if (now - last > 200000000ull) {
+                        ok = false;
+                        break;
+                    }
                 }
             }
             if (!ok) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
@@ -1434,9 +1444,37 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)g * GSTRIDE;
         const uint32_t tU = tl, tC = tl + (uint32_t)D;          // keys: C, then P, at tC
         bool failed = false;
-        for (int li = g, k = 0; li < ntile && !failed; li += NG, ++k) {
-            const int64_t tile = tile_begin + li, bh = tile / p.tiles_per_bh;
-            const int64_t t = (tile % p.tiles_per_bh) * ENC_ROWS + row;
+        // keys: the sign plane of the group's previous tile is stored after this
+        // tile's |u|^2 pass, so its QJL projection overlaps that pass
+        uint32_t *prev_dst = nullptr;
+        bool prev_valid = false, prev_zero = false;
+        auto sign_epilogue = [&](int kprev) -> bool {
+            if (!warp_wait(&bar_qjl[g], (uint32_t)(kprev & 1))) return false;
+            tqdev::tc_fence_after();
+            uint32_t *sdst = prev_dst + B * NC;
+#pragma unroll 1
+            for (int c = 0; c < M / 32; ++c) {
+                uint32_t neg = 0u;
+#pragma unroll
+                for (int half = 1; half >= 0; --half) {
+                    float pv[16];
+                    tqdev::tmem_ld_32x32b_x16_nowait(tC + 32 * c + 16 * half, pv);
+                    tqdev::tmem_wait_ld();
+                    // bit i = [p_i >= 0] from the sign bit; an exact zero (of
+                    // either sign) lies inside the decision band of p = 0
+#pragma unroll
+                    for (int j = 15; j >= 0; --j) neg = push_sign(neg, pv[j]);
+                }
+                if (prev_valid) sdst[c] = prev_zero ? ~0u : ~neg;
+            }
+            tqdev::tc_fence_before();
+            return true;
+        };
+        int k = 0;
+        for (int li = g; li < ntile && !failed; li += NG, ++k) {
+            const uint32_t tile = (uint32_t)(tile_begin + li), bh32 = tile / tpb;
+            const int64_t bh = bh32;
+            const int64_t t = (int64_t)(tile - bh32 * tpb) * ENC_ROWS + row;
             const bool valid = t < p.T;
             uint32_t *dst = reinterpret_cast<uint32_t *>(p.out + (bh * p.capacity + p.token_offset + t) * p.row_bytes);
             if (!warp_wait(&bar_rot[g], (uint32_t)(k & 1))) {
@@ -1458,6 +1496,12 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                     for (int i = 0; i < 32; i += 2)
                         n2p = fma2(make_float2(cur[i], cur[i + 1]), make_float2(cur[i], cur[i + 1]), n2p);
                     if (c + 1 < NC) tqdev::tmem_wait_ld();
+                }
+            }
+            if constexpr (KEYS) {
+                if (k > 0 && !sign_epilogue(k - 1)) {
+                    failed = true;
+                    break;
                 }
             }
             const float n2 = n2p.x + n2p.y;
@@ -1677,30 +1721,13 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
                     dst[tail] = __float_as_uint(ns);
                     dst[tail + 1] = __float_as_uint(gv);
                 }
-                // ---- sign plane from this tile's projections
-                if (!warp_wait(&bar_qjl[g], (uint32_t)(k & 1))) {
-                    failed = true;
-                    break;
-                }
-                tqdev::tc_fence_after();
-                uint32_t *sdst = dst + B * NC;
-#pragma unroll 1
-                for (int c = 0; c < M / 32; ++c) {
-                    uint32_t neg = 0u;
-#pragma unroll
-                    for (int half = 1; half >= 0; --half) {
-                        float pv[16];
-                        tqdev::tmem_ld_32x32b_x16_nowait(tC + 32 * c + 16 * half, pv);
-                        tqdev::tmem_wait_ld();
-                        // bit i = [p_i >= 0] from the sign bit; an exact zero (of
-                        // either sign) lies inside the decision band of p = 0
-#pragma unroll
-                        for (int j = 15; j >= 0; --j) neg = push_sign(neg, pv[j]);
-                    }
-                    if (valid) sdst[c] = zero_row ? ~0u : ~neg;
-                }
-                tqdev::tc_fence_before();
+                prev_dst = dst;
+                prev_valid = valid;
+                prev_zero = zero_row;
             }
+        }
+        if constexpr (KEYS) {
+            if (!failed && k > 0 && !sign_epilogue(k - 1)) failed = true;   // the group's last tile
         }
         if (failed && lane == 0) atomicOr(reinterpret_cast<unsigned int *>(&p.status[1]), TQ_FLAG_WAIT_TIMEOUT);
     }
@@ -1715,9 +1742,9 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS>::THREADS, 1)
 template <int D, typename Tin, bool KEYS>
 cudaError_t launch_pipe(int B, const PipeParams &p, const CUtensorMap &mx, const CUtensorMap &mhd,
                         const CUtensorMap &ms, int grid, cudaStream_t s) {
-    using L = PipeLayout<D, KEYS>;
+    using L = PipeLayout<D, KEYS, 2>;   // the byte layout does not depend on B
     cudaError_t e = cudaSuccess;
-    auto go = [&](auto kern) {
+    auto go = [&](auto kern, int threads) {
         size_t smem = (size_t)L::FIXED + (KEYS ? p.s_bytes : 0);
         // one CTA per SM: a second one could wait in tcgen05.alloc until the
         // first exits (the grid is one CTA per SM anyway)
@@ -1727,15 +1754,15 @@ cudaError_t launch_pipe(int B, const PipeParams &p, const CUtensorMap &mx, const
             cudaGetLastError();
             return;
         }
-        kern<<<grid, L::THREADS, smem, s>>>(p, mx, mhd, ms);
+        kern<<<grid, threads, smem, s>>>(p, mx, mhd, ms);
         e = cudaGetLastError();
     };
     switch (B) {
-        case 1: if constexpr (KEYS) go(tq_encode_pipe_kernel<D, 1, Tin, KEYS>); else return cudaErrorInvalidValue; break;
-        case 2: go(tq_encode_pipe_kernel<D, 2, Tin, KEYS>); break;
-        case 3: go(tq_encode_pipe_kernel<D, 3, Tin, KEYS>); break;
-        case 4: go(tq_encode_pipe_kernel<D, 4, Tin, KEYS>); break;
-        case 5: if constexpr (!KEYS) go(tq_encode_pipe_kernel<D, 5, Tin, KEYS>); else return cudaErrorInvalidValue; break;
+        case 1: if constexpr (KEYS) go(tq_encode_pipe_kernel<D, 1, Tin, KEYS>, PipeLayout<D, KEYS, 1>::THREADS); else return cudaErrorInvalidValue; break;
+        case 2: go(tq_encode_pipe_kernel<D, 2, Tin, KEYS>, PipeLayout<D, KEYS, 2>::THREADS); break;
+        case 3: go(tq_encode_pipe_kernel<D, 3, Tin, KEYS>, PipeLayout<D, KEYS, 3>::THREADS); break;
+        case 4: go(tq_encode_pipe_kernel<D, 4, Tin, KEYS>, PipeLayout<D, KEYS, 4>::THREADS); break;
+        case 5: if constexpr (!KEYS) go(tq_encode_pipe_kernel<D, 5, Tin, KEYS>, PipeLayout<D, KEYS, 5>::THREADS); else return cudaErrorInvalidValue; break;
         default: return cudaErrorInvalidValue;
     }
     return e;
@@ -1869,7 +1896,7 @@ static bool pipe_side(tq_ctx *ctx, bool keys, const void *x, tq_dtype dtype, int
     const int d = ctx->d, M = ctx->m;
     if (keys) {
         if (2 * (d + std::max(d, M)) > 512) return false;   // two groups' TMEM columns
-        const size_t smem = (d == 128 ? PipeLayout<128, true>::FIXED : PipeLayout<64, true>::FIXED) + (size_t)(d / 64) * M * 128;
+        const size_t smem = (d == 128 ? PipeLayout<128, true, 2>::FIXED : PipeLayout<64, true, 2>::FIXED) + (size_t)(d / 64) * M * 128;
         if (smem > 227 * 1024) return false;
     }
     if (T > 0x7FFFFFFF - ENC_ROWS) return false;
@@ -1885,6 +1912,7 @@ static bool pipe_side(tq_ctx *ctx, bool keys, const void *x, tq_dtype dtype, int
     p.M = M;
     p.tiles_per_bh = (T + ENC_ROWS - 1) / ENC_ROWS;
     p.n_tiles = p.tiles_per_bh * (int64_t)batch * H;
+    if (p.n_tiles > 0x7FFFFFFF) return false;   // the kernel's tile indices are 32-bit
     p.s_bytes = (uint32_t)((d / 64) * M * 128);
     p.status = ctx->d_status;
     p.norm_f16 = ctx->norm_f16;
