@@ -105,15 +105,24 @@ def arm_config(workload):
     return {"workload": WORKLOAD_DESC[workload], "step": STEP_DESC[workload], "l2": L2_DESC}
 
 
-# DRAM traffic of a piece's main kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum of one launch, one ncu capture, caches flushed before
-# the launch), keyed by (piece, workload), with the SHA-1 of the source file
-# holding that kernel when the counters were taken: once the source changes
-# the entry no longer applies (traffic: null).  Summaries: profiles/.
+# DRAM traffic of a piece: dram__bytes_read.sum + dram__bytes_write.sum summed
+# over the piece's launches of one step (one ncu capture, caches flushed before
+# the piece, the median step of those captured), keyed by (piece, workload),
+# with the SHA-1 of the source files holding those kernels when the counters
+# were taken: once one of them changes the entry no longer applies (traffic:
+# null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 327339776),
-    ("encode_values", "mha_decode"): ("tq_encode.cu", "0092e96e8d41ba04ed05e9e764e258c52dff545c", 320737792),
-    ("decode", "mha_decode"): ("tq_decode.cu", "05c64fbca48ff7d3b112c4b021c5b1213c090796", 151720960),
+    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 329518080),
+    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 320385280),
+    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 148876800),
+    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 297863936),
+    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 292844288),
+    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 80967168),
+    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 628645376),
+    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 616377600),
+    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 43086080),
+    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 42775552),
+    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 24092416),
 }
 
 
@@ -122,13 +131,15 @@ def measured_traffic(piece, workload):
     ent = MEASURED_TRAFFIC.get((piece, workload))
     if not ent:
         return None
-    src, sha, nbytes = ent
+    files, sha, nbytes = ent
+    h = hashlib.sha1()
     try:
-        with open(os.path.join(ROOT, "kv_cache_vector_10_b200", "csrc", src), "rb") as f:
-            cur = hashlib.sha1(f.read()).hexdigest()
+        for src in files:
+            with open(os.path.join(ROOT, "kv_cache_vector_10_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
     except OSError:
         return None
-    return nbytes if cur == sha else None
+    return nbytes if h.hexdigest() == sha else None
 
 
 def row_bytes(bits, norms="f32"):

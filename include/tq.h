@@ -59,10 +59,12 @@ typedef enum tq_status {
     TQ_OK = 0,
     TQ_ERR_NULL = 1,          /* a required pointer is NULL */
     TQ_ERR_ZERO_DIM = 2,      /* head_dim == 0 (bitpolar ZeroDimension) */
-    TQ_ERR_DIM = 3,           /* head_dim not 64 or 128 (bitpolar OddDimension, generalized) */
+    TQ_ERR_DIM = 3,           /* head_dim not 64, 128 or 256, or 256 with the Haar rotation
+                                 (bitpolar OddDimension, generalized) */
     TQ_ERR_BITS = 4,          /* bits not in 2..5 (bitpolar InvalidBitWidth) */
     TQ_ERR_ZERO_PROJ = 5,     /* projections == 0 (bitpolar ZeroProjections) */
-    TQ_ERR_PROJ = 6,          /* projections not a multiple of 32 in [32, 256] */
+    TQ_ERR_PROJ = 6,          /* projections not a multiple of 32 in [32, 256] ([32, 192] at
+                                 head_dim 256) */
     TQ_ERR_EMPTY = 7,         /* zero heads or zero batch (bitpolar EmptyInput) */
     TQ_ERR_DIM_MISMATCH = 8,  /* shapes disagree: H_q % H_kv, tokens beyond capacity,
                                  capacity not a multiple of 16 (bitpolar DimensionMismatch) */
@@ -131,9 +133,11 @@ typedef struct tq_segment {
  * total TurboQuant width b (keys: b-1 PolarQuant bits + 1 QJL bit; values: b
  * MSE bits; turboquant-plus-rs "Architecture").  Builds the Lloyd-Max
  * codebooks on the host and uploads them.  Head tables are built by
- * tq_ensure_heads (or on first use).  head_dim in {64, 128}; bits in 2..5;
- * projections a multiple of 32 in [32, 256].  On success *out owns device
- * memory released by tq_destroy.  Synchronous. */
+ * tq_ensure_heads (or on first use).  head_dim in {64, 128, 256}; bits in
+ * 2..5; projections a multiple of 32 in [32, 256], at most 192 when head_dim
+ * is 256 (the key encoder's S tile and residual operand share 227 KB of
+ * shared memory).  On success *out owns device memory released by
+ * tq_destroy.  Synchronous. */
 tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_ctx **out);
 
 /* tq_create with a choice of rotation.  TQ_ROT_HADAMARD is tq_create.
@@ -144,7 +148,9 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
  * rows are rotated on the tensor cores (sqrt(d) Q as binary16 hi + lo
  * against the row scaled by a power of two into binary16 range: binary16
  * and bfloat16 rows exactly, float32 rows as hi + lo), queries and outputs
- * with fp32 Q.  Packed formats and every other call are unchanged.  In this
+ * with fp32 Q.  Not available at head_dim 256 (TQ_ERR_DIM: the two binary16
+ * pieces of sqrt(d) Q alone fill 256 KB, above the 227 KB of shared memory a
+ * CTA can hold).  Packed formats and every other call are unchanged.  In this
  * mode a row whose largest |x_j| is below 2^-100 is encoded as a zero row.
  * Returns TQ_ERR_DIM for an unknown rotation. */
 tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,

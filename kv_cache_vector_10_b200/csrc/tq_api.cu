@@ -141,10 +141,15 @@ tq_status tq_create_format(int head_dim, int bits, int projections, uint64_t see
     }
     *out = nullptr;
     if (head_dim == 0) return TQ_ERR_ZERO_DIM;
-    if (head_dim != 64 && head_dim != 128) return TQ_ERR_DIM;
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256) return TQ_ERR_DIM;
+    // d = 256: the Haar operands (2 x d x d binary16) do not fit in shared memory
+    if (head_dim == 256 && rotation == TQ_ROT_HAAR) return TQ_ERR_DIM;
     if (bits < 2 || bits > 5) return TQ_ERR_BITS;
     if (projections == 0) return TQ_ERR_ZERO_PROJ;
     if (projections < 32 || projections > 256 || projections % 32) return TQ_ERR_PROJ;
+    // d = 256: the key encoder's S tile and residual operand take
+    // (d/64) (128 m + 32 K) bytes of shared memory, within 227 KB for m <= 192
+    if (head_dim == 256 && projections > 192) return TQ_ERR_PROJ;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
     cudaDeviceProp prop;
@@ -295,7 +300,7 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
     CUtensorMap hdmap16, hdmapbf;
     std::memset(&hdmap16, 0, sizeof(hdmap16));
     std::memset(&hdmapbf, 0, sizeof(hdmapbf));
-    if (st == TQ_OK && ctx->rotation == TQ_ROT_HADAMARD) {
+    if (st == TQ_OK && ctx->rotation == TQ_ROT_HADAMARD && d <= 128) {   // the TMA-fed encoders' d
         const size_t dd = (size_t)d * d;
         std::vector<uint16_t> h16((size_t)n_heads * dd), hbf((size_t)n_heads * dd);
         for (int h = 0; h < n_heads; ++h)

@@ -334,7 +334,12 @@ __device__ __forceinline__ float load_dt(const void *p, int64_t i, int dt) {
     return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
 }
 
-// Sum over the block (AUX_THREADS threads); every thread gets the total.
+// Threads of a query-preparation block: one per coordinate for the append
+// step (at least AUX_THREADS).
+__host__ __device__ constexpr int qprep_threads(int d) { return d > AUX_THREADS ? d : AUX_THREADS; }
+
+// Sum over the block (NT threads); every thread gets the total.
+template <int NT>
 __device__ __forceinline__ float block_sum(float v, float *s_red) {
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -343,7 +348,7 @@ __device__ __forceinline__ float block_sum(float v, float *s_red) {
     __syncthreads();
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < AUX_THREADS / 32; ++w) t += s_red[w];
+    for (int w = 0; w < NT / 32; ++w) t += s_red[w];
     return t;
 }
 
@@ -353,7 +358,7 @@ __device__ __forceinline__ float block_sum(float v, float *s_red) {
 // u = H (D x); n = |x|; cell = #{positive boundaries <= |u| / n}; index
 // 2^(B-1) + cell, mirrored for u < 0; n_s = n / |C[idx]/sqrt(d)|; keys add
 // the QJL signs of S (u - n_s C[idx]) and gamma = |u - n_s C[idx]| / sqrt(d).
-// One block of AUX_THREADS threads, coordinate j on thread j.
+// One block of qprep_threads(D) threads, coordinate j on thread j.
 template <int D>
 __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, const SegDesc &g, int h, int64_t t,
                            float *s_u, float *s_e, float *s_red, uint8_t *s_idx) {
@@ -392,7 +397,7 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
         }
         u = tid < D ? s_u[tid] : 0.f;
     }
-    const float n2 = block_sum(u * u, s_red);
+    const float n2 = block_sum<qprep_threads(D)>(u * u, s_red);
     const bool nonfinite = !(n2 <= 3.0e38f);
     const bool degenerate = nonfinite || !(n2 >= 1.17549435e-38f);
     if (tid == 0 && nonfinite) atomicAdd(&g.status[0], 1ull);
@@ -400,7 +405,7 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
     int cell = 0;
     for (int k = 0; k + 1 < HB; ++k) cell += fabsf(u) >= n * pb[k] ? 1 : 0;
     const float cm = mag[cell];
-    const float c2 = block_sum(tid < D ? cm * cm : 0.f, s_red);
+    const float c2 = block_sum<qprep_threads(D)>(tid < D ? cm * cm : 0.f, s_red);
     const float ns = degenerate ? 0.f : n * sqrtf((float)D / c2);
     const uint32_t idx = degenerate ? (uint32_t)HB : u < 0.f ? (uint32_t)(HB - 1 - cell) : (uint32_t)(HB + cell);
     const int64_t rowb = key ? g.krow : g.vrow;
@@ -409,7 +414,7 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
     if (key) {
         const float e = tid < D && !degenerate ? u - ns * (u < 0.f ? -cm : cm) : 0.f;
         if (tid < D) s_e[tid] = e;
-        const float e2 = block_sum(e * e, s_red);   // its barriers publish s_e
+        const float e2 = block_sum<qprep_threads(D)>(e * e, s_red);   // its barriers publish s_e
         const float gv = degenerate ? 0.f : sqrtf(e2 * (1.f / D));
         // binary16 norms: a row whose norms overflow is the zero row, counted
         // with the non-finite rows (ns and e2 are block-wide, so is this)
@@ -480,12 +485,12 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
 // query [q_rot | S q_rot].  Blocks after those: one per (appending segment,
 // kv head), the append step's new key and value rows.
 template <int D, typename Tq>
-__global__ void __launch_bounds__(AUX_THREADS) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
+__global__ void __launch_bounds__(qprep_threads(D)) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
     tqdev::grid_dep_trigger();   // the decode CTAs may start their set-up now
     __shared__ float s_in[D];
     __shared__ __align__(16) float s_qr[D];
     __shared__ float s_sq[256];
-    __shared__ float s_red[AUX_THREADS / 32];
+    __shared__ float s_red[qprep_threads(D) / 32];
     __shared__ uint8_t s_idx[D];
     int s = 0;
     int64_t blk = blockIdx.x;
@@ -603,7 +608,7 @@ tq_status tq_launch_scores(tq_ctx *ctx, const tq_codes *codes, const float *q, i
     const int64_t per_block = (int64_t)SCORE_THREADS * SCORE_TPT;
     dim3 grid((unsigned)((T + per_block - 1) / per_block), (unsigned)Hq, (unsigned)codes->batch);
     const size_t tab = (size_t)(ctx->d / 8 + ctx->m / 8) * 256 * sizeof(float);
-    auto kern = ctx->d == 128 ? tq_scores_kernel<128> : tq_scores_kernel<64>;
+    auto kern = ctx->d == 256 ? tq_scores_kernel<256> : ctx->d == 128 ? tq_scores_kernel<128> : tq_scores_kernel<64>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tab);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -637,7 +642,10 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
     dim3 grid((unsigned)((T + AUX_THREADS - 1) / AUX_THREADS), (unsigned)codes->n_kv_heads, (unsigned)codes->batch);
     const size_t smem = k_hat ? (size_t)ctx->m * ctx->d * 2 : 0;
     cudaError_t e;
-    if (ctx->d == 128) {
+    if (ctx->d == 256) {
+        e = cudaFuncSetAttribute(tq_dequant_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) tq_dequant_kernel<256><<<grid, AUX_THREADS, smem, stream>>>(p);
+    } else if (ctx->d == 128) {
         e = cudaFuncSetAttribute(tq_dequant_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess) tq_dequant_kernel<128><<<grid, AUX_THREADS, smem, stream>>>(p);
     } else {
@@ -655,8 +663,12 @@ cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cud
     int64_t blocks = P.n_append_blocks;
     for (int s = 0; s < P.n_segs; ++s) blocks += (int64_t)P.seg[s].n_seqs * P.Hq;
     if (blocks == 0) return cudaSuccess;
-#define TQ_QPREP(DD, TT) tq_qprep_kernel<DD, TT><<<(unsigned)blocks, AUX_THREADS, 0, stream>>>(P, q)
-    if (P.d == 128) {
+#define TQ_QPREP(DD, TT) tq_qprep_kernel<DD, TT><<<(unsigned)blocks, qprep_threads(DD), 0, stream>>>(P, q)
+    if (P.d == 256) {
+        if (dt == TQ_F32) TQ_QPREP(256, float);
+        else if (dt == TQ_F16) TQ_QPREP(256, __half);
+        else TQ_QPREP(256, __nv_bfloat16);
+    } else if (P.d == 128) {
         if (dt == TQ_F32) TQ_QPREP(128, float);
         else if (dt == TQ_F16) TQ_QPREP(128, __half);
         else TQ_QPREP(128, __nv_bfloat16);
@@ -673,7 +685,11 @@ cudaError_t tq_launch_combine(const DecodePlan &P, void *out, tq_dtype dt, cudaS
     const unsigned blocks = (unsigned)(P.batch * P.Hq);
 #define TQ_COMB(DD, TT) \
     return tq_launch_dependent(tq_combine_kernel<DD, TT>, dim3((unsigned)blocks), dim3(DD), 0, stream, P, out)
-    if (P.d == 128) {
+    if (P.d == 256) {
+        if (dt == TQ_F32) TQ_COMB(256, float);
+        else if (dt == TQ_F16) TQ_COMB(256, __half);
+        else TQ_COMB(256, __nv_bfloat16);
+    } else if (P.d == 128) {
         if (dt == TQ_F32) TQ_COMB(128, float);
         else if (dt == TQ_F16) TQ_COMB(128, __half);
         else TQ_COMB(128, __nv_bfloat16);

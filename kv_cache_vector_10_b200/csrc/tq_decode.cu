@@ -103,8 +103,9 @@ __device__ __forceinline__ void store_out_dt(void *p, int64_t i, float v, int dt
 
 // MT = number of QJL projections when known at compile time (128), else 0;
 // KF = key norms as binary16 (1) or fp32 (0) when MT > 0 (else read from the
-// segment).
-template <int D, int BK, int BV, int QC, int MT, int KF>
+// segment); NBUF = staging buffers per warp (2, or 1 where two do not fit in
+// shared memory: head_dim 256 at the larger bit widths).
+template <int D, int BK, int BV, int QC, int MT, int KF, int NBUF>
 __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const __grid_constant__ DecodePlan P) {
     using VT = typename Vec<QC>::T;
     constexpr int NGK = D / 8;                    // byte groups of an index plane = value slots
@@ -112,7 +113,9 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     constexpr int NP = n_sigma_planes(BK);
     constexpr int VPB = 2 * BV;                   // bits of a value pair
     constexpr int VCOP = vpair_copies<BV>();
-    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(D == 64 || D == 128 || D == 256, "head_dim");
+    static_assert(NBUF == 1 || NBUF == 2, "staging depth");
+    constexpr int VR = D > 128 ? D / 128 : 1;      // value rounds: 128 coordinates per warp-half each
     extern __shared__ __align__(128) uint8_t smem_raw[];
 
     // An append step's new rows are written by the query-preparation kernel:
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     VT *luts = lutq + lut_entries<QC>(RK);
     float2 *vlut = reinterpret_cast<float2 *>(luts + lut_entries<QC>(RS));
     uint64_t *bars = reinterpret_cast<uint64_t *>(vlut + vpair_entries<BV>() * VCOP);
-    uint8_t *stage = reinterpret_cast<uint8_t *>(bars + 2 * TQ_DEC_WARPS);
+    uint8_t *stage = reinterpret_cast<uint8_t *>(bars + NBUF * TQ_DEC_WARPS);
     const int chunk_bytes = TQ_DEC_CHUNK * (krow + vrow);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     // of an aborted context requests nothing and waits for nothing.
     __shared__ int s_abort;
     if (tid == 0) {
-        for (int i = 0; i < 2 * TQ_DEC_WARPS; ++i) tqdev::mbar_init(&bars[i], 1);
+        for (int i = 0; i < NBUF * TQ_DEC_WARPS; ++i) tqdev::mbar_init(&bars[i], 1);
         tqdev::fence_barrier_init();
         s_abort = tqdev::status_aborted(g.status) ? 1 : 0;
     }
@@ -172,12 +175,11 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const uint8_t *kbase = g.kc + (int64_t)h * g.capacity * krow;
     const uint8_t *vbase = g.vc + (int64_t)h * g.capacity * vrow;
     if (lane == 0 && !pre_aborted) {
-        if (warp < n_chunks)
-            issue_chunk(stage + (warp * 2 + 0) * chunk_bytes, &bars[warp * 2 + 0], kbase, vbase, t_begin + warp * TQ_DEC_CHUNK,
-                        g.capacity, krow, vrow);
-        if (warp + TQ_DEC_WARPS < n_chunks)
-            issue_chunk(stage + (warp * 2 + 1) * chunk_bytes, &bars[warp * 2 + 1], kbase, vbase,
-                        t_begin + (warp + TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
+#pragma unroll
+        for (int b = 0; b < NBUF; ++b)
+            if (warp + b * TQ_DEC_WARPS < n_chunks)
+                issue_chunk(stage + (warp * NBUF + b) * chunk_bytes, &bars[warp * NBUF + b], kbase, vbase,
+                            t_begin + (warp + b * TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
     }
 
     // ---- per-query lookup tables (from the query-preparation kernel's output)
@@ -242,37 +244,36 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int off_ns = off_sign + M / 8;
     const bool kf16 = MT > 0 ? KF != 0 : g.kf16 != 0;
     const int voff_ns = BV * D / 8;
-    // value bits of this lane's 8 coordinates: [8*BV*slot, 8*BV*slot + 8*BV)
-    const int vbit = 8 * BV * slot;
-    const int vw0 = vbit / 32, vsh = vbit % 32;
+    // value bits of this lane's 8 coordinates of round r (coordinates
+    // 128 r + 8 slot .. + 7): [8*BV*(16 r + slot), + 8*BV)
     const bool vslot = slot < NGK;
     const int vcopy = VCOP > 1 ? slot : 0;
 
     float m_run[QC], l_lane[QC];
-    float2 o[QC][4];   // coordinates 8*slot + 2p, +1 (tokens of parity `half`)
+    float2 o[QC][4 * VR];   // coordinates 128 r + 8*slot + 2p, +1 at [4 r + p] (tokens of parity `half`)
 #pragma unroll
     for (int qq = 0; qq < QC; ++qq) {
         m_run[qq] = -INFINITY;
         l_lane[qq] = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[qq][c] = make_float2(0.f, 0.f);
+        for (int c = 0; c < 4 * VR; ++c) o[qq][c] = make_float2(0.f, 0.f);
     }
     bool aborted = pre_aborted;
     for (int64_t k = 0; !aborted; ++k) {
         const int64_t ci = warp + k * TQ_DEC_WARPS;
         if (ci >= n_chunks) break;
-        const int buf = (int)(k & 1);
-        if (!tqdev::mbar_wait_bounded(&bars[warp * 2 + buf], (uint32_t)((k >> 1) & 1))) {
+        const int buf = (int)(k % NBUF);
+        if (!tqdev::mbar_wait_bounded(&bars[warp * NBUF + buf], (uint32_t)((k / NBUF) & 1))) {
             aborted = true;
-            // Both of this warp's buffers may still have a copy in flight (the
-            // one just waited for, and the next chunk's in the other buffer):
-            // give each one more bounded wait before `stage` is reused below.
-            tqdev::mbar_wait_bounded(&bars[warp * 2 + buf], (uint32_t)((k >> 1) & 1));
-            if (ci + TQ_DEC_WARPS < n_chunks)
-                tqdev::mbar_wait_bounded(&bars[warp * 2 + (buf ^ 1)], (uint32_t)(((k + 1) >> 1) & 1));
+            // Each of this warp's buffers may still have a copy in flight (the
+            // one just waited for, and with two buffers the next chunk's in the
+            // other): give each one more bounded wait before `stage` is reused.
+            tqdev::mbar_wait_bounded(&bars[warp * NBUF + buf], (uint32_t)((k / NBUF) & 1));
+            if (NBUF == 2 && ci + TQ_DEC_WARPS < n_chunks)
+                tqdev::mbar_wait_bounded(&bars[warp * NBUF + (buf ^ 1)], (uint32_t)(((k + 1) / NBUF) & 1));
             break;
         }
-        const uint8_t *sK = stage + (warp * 2 + buf) * chunk_bytes;
+        const uint8_t *sK = stage + (warp * NBUF + buf) * chunk_bytes;
         const uint8_t *sV = sK + TQ_DEC_CHUNK * krow;
         const int64_t t0 = t_begin + ci * TQ_DEC_CHUNK;
 
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             l_lane[qq] = fmaf(l_lane[qq], corr, pr);
             const float2 c2 = make_float2(corr, corr);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) o[qq][c] = __fmul2_rn(o[qq][c], c2);
+            for (int c = 0; c < 4 * VR; ++c) o[qq][c] = __fmul2_rn(o[qq][c], c2);
             m_run[qq] = mn;
             w_tok[qq] = valid ? pr * nsv : 0.f;
         }
@@ -364,32 +365,37 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                 wq[qq] = make_float2(wv, wv);
             }
             if (vslot) {
-                uint32_t raw;
-                if constexpr (BV == 4) raw = vr[vw0];
-                else raw = __funnelshift_r(vr[vw0], vr[vw0 + 1], vsh);
-                uint32_t raw_hi = 0;
-                if constexpr (BV == 5) raw_hi = __funnelshift_r(vr[vw0 + 1], vr[vw0 + 2], vsh);
 #pragma unroll
-                for (int pp = 0; pp < 4; ++pp) {
-                    uint32_t e;
-                    if constexpr (BV == 5) {
-                        const int sh = VPB * pp;
-                        e = (sh >= 32 ? raw_hi >> (sh - 32) : (sh + VPB > 32 ? (raw >> sh) | (raw_hi << (32 - sh)) : raw >> sh)) &
-                            ((1u << VPB) - 1);
-                    } else {
-                        e = (raw >> (VPB * pp)) & ((1u << VPB) - 1);
+                for (int r = 0; r < VR; ++r) {
+                    const int vbit = 8 * BV * (16 * r + slot);
+                    const int vw0 = vbit / 32, vsh = vbit % 32;
+                    uint32_t raw;
+                    if constexpr (BV == 4) raw = vr[vw0];
+                    else raw = __funnelshift_r(vr[vw0], vr[vw0 + 1], vsh);
+                    uint32_t raw_hi = 0;
+                    if constexpr (BV == 5) raw_hi = __funnelshift_r(vr[vw0 + 1], vr[vw0 + 2], vsh);
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) {
+                        uint32_t e;
+                        if constexpr (BV == 5) {
+                            const int sh = VPB * pp;
+                            e = (sh >= 32 ? raw_hi >> (sh - 32) : (sh + VPB > 32 ? (raw >> sh) | (raw_hi << (32 - sh)) : raw >> sh)) &
+                                ((1u << VPB) - 1);
+                        } else {
+                            e = (raw >> (VPB * pp)) & ((1u << VPB) - 1);
+                        }
+                        const float2 cv = vlut[e * VCOP + vcopy];
+#pragma unroll
+                        for (int qq = 0; qq < QC; ++qq) o[qq][4 * r + pp] = __ffma2_rn(wq[qq], cv, o[qq][4 * r + pp]);
                     }
-                    const float2 cv = vlut[e * VCOP + vcopy];
-#pragma unroll
-                    for (int qq = 0; qq < QC; ++qq) o[qq][pp] = __ffma2_rn(wq[qq], cv, o[qq][pp]);
                 }
             }
         }
         __syncwarp();
-        if (lane == 0 && ci + 2 * TQ_DEC_WARPS < n_chunks) {
+        if (lane == 0 && ci + NBUF * TQ_DEC_WARPS < n_chunks) {
             tqdev::fence_proxy_async_smem();
-            issue_chunk(stage + (warp * 2 + buf) * chunk_bytes, &bars[warp * 2 + buf], kbase, vbase,
-                        t_begin + (ci + 2 * TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
+            issue_chunk(stage + (warp * NBUF + buf) * chunk_bytes, &bars[warp * NBUF + buf], kbase, vbase,
+                        t_begin + (ci + NBUF * TQ_DEC_WARPS) * TQ_DEC_CHUNK, g.capacity, krow, vrow);
         }
     }
     if (aborted && lane == 0) atomicOr(reinterpret_cast<unsigned int *>(g.status + 1), TQ_FLAG_WAIT_TIMEOUT);
@@ -408,13 +414,14 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             row[1] = aborted ? 0.f : lt;
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 4 * VR; ++c) {
             float2 v = o[qq][c];
             v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
             v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
             if (half == 0 && vslot) {
-                row[2 + 8 * slot + 2 * c] = aborted ? 0.f : v.x;
-                row[2 + 8 * slot + 2 * c + 1] = aborted ? 0.f : v.y;
+                const int j = 128 * (c / 4) + 8 * slot + 2 * (c % 4);
+                row[2 + j] = aborted ? 0.f : v.x;
+                row[2 + j + 1] = aborted ? 0.f : v.y;
             }
         }
     }
@@ -516,18 +523,26 @@ struct SegPlan {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Shared memory of one decode CTA (must match tq_decode_kernel's carve-up).
-size_t decode_smem_bytes(int d, int bv, int qc, int krow, int vrow, int M) {
+// Shared memory of one decode CTA with nbuf staging buffers per warp (must
+// match tq_decode_kernel's carve-up).
+size_t decode_smem_bytes(int d, int bv, int qc, int krow, int vrow, int M, int nbuf) {
     const int RK = (d / 8 + 15) / 16, RS = (M / 8 + 15) / 16;
     const size_t vt = qc == 1 ? 4 : qc == 2 ? 8 : 16;
     const size_t lut = (size_t)(RK + RS) * 256 * 16 * (qc == 1 ? 2 : 1) * vt;
     const size_t vpair = (size_t)(1 << (2 * bv)) * (bv <= 4 ? 16 : 1) * 8;
-    const size_t stage = (size_t)TQ_DEC_WARPS * 2 * TQ_DEC_CHUNK * (krow + vrow);
+    const size_t stage = (size_t)TQ_DEC_WARPS * nbuf * TQ_DEC_CHUNK * (krow + vrow);
     const size_t merge = ((size_t)TQ_DEC_WARPS * qc * (d + 2) + qc * d + 2 * qc) * 4;
-    return lut + vpair + 2 * TQ_DEC_WARPS * 8 + std::max(stage, merge);
+    return lut + vpair + (size_t)nbuf * TQ_DEC_WARPS * 8 + std::max(stage, merge);
 }
 
 constexpr size_t kMaxDynSmem = 232448;   // 227 KB per block on sm_100
+
+// Staging buffers per warp: two where they fit, else one (0: none fits).
+int decode_nbuf(int d, int bv, int qc, int krow, int vrow, int M) {
+    if (decode_smem_bytes(d, bv, qc, krow, vrow, M, 2) <= kMaxDynSmem) return 2;
+    if (decode_smem_bytes(d, bv, qc, krow, vrow, M, 1) <= kMaxDynSmem) return 1;
+    return 0;
+}
 
 void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sms, std::vector<SegPlan> &out) {
     const int G = Hq / Hkv;
@@ -539,7 +554,7 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
         const tq_ctx *c = segs[s].ctx;
         const int krow = (int)tq_row_bytes(c, TQ_KEYS), vrow = (int)tq_row_bytes(c, TQ_VALUES);
         p.qc = nq >= 4 ? 4 : nq >= 2 ? 2 : 1;
-        while (p.qc > 1 && decode_smem_bytes(c->d, c->BV, p.qc, krow, vrow, c->m) > kMaxDynSmem) p.qc /= 2;
+        while (p.qc > 1 && decode_nbuf(c->d, c->BV, p.qc, krow, vrow, c->m) == 0) p.qc /= 2;
         p.n_qchunks = (nq + p.qc - 1) / p.qc;
         work += segs[s].n_tokens * (int64_t)Hkv * p.n_qchunks;
     }
@@ -579,12 +594,17 @@ void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sm
 
 template <int D, int BK, int BV, int QC>
 cudaError_t launch_decode_t(const DecodePlan &P, int64_t items, int krow, int vrow, int M, cudaStream_t stream) {
-    const size_t smem = decode_smem_bytes(D, BV, QC, krow, vrow, M);
+    const int nbuf = decode_nbuf(D, BV, QC, krow, vrow, M);
+    if (nbuf == 0) return cudaErrorInvalidValue;
+    const size_t smem = decode_smem_bytes(D, BV, QC, krow, vrow, M, nbuf);
     // the launch's segments share one key-row length, hence one norm format
     const bool kf16 = krow == BK * D / 8 + M / 8 + 4;
-    auto kern = M != 128 ? tq_decode_kernel<D, BK, BV, QC, 0, 0>
-                : kf16   ? tq_decode_kernel<D, BK, BV, QC, 128, 1>
-                         : tq_decode_kernel<D, BK, BV, QC, 128, 0>;
+    auto kern = nbuf == 2 ? (M != 128 ? tq_decode_kernel<D, BK, BV, QC, 0, 0, 2>
+                             : kf16   ? tq_decode_kernel<D, BK, BV, QC, 128, 1, 2>
+                                      : tq_decode_kernel<D, BK, BV, QC, 128, 0, 2>)
+                          : (M != 128 ? tq_decode_kernel<D, BK, BV, QC, 0, 0, 1>
+                             : kf16   ? tq_decode_kernel<D, BK, BV, QC, 128, 1, 1>
+                                      : tq_decode_kernel<D, BK, BV, QC, 128, 0, 1>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
         cudaGetLastError();   // do not leave the failure as the thread's sticky last error
@@ -782,8 +802,9 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         for (int s = 0; s < n_segs; ++s)
             if (!done[s] && same(s)) done[s] = 1;
         if (items == 0) continue;
-        e = P.d == 128 ? launch_decode_dim<128>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
-                       : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);
+        e = P.d == 256   ? launch_decode_dim<256>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
+            : P.d == 128 ? launch_decode_dim<128>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
+                         : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);
         if (e != cudaSuccess) return tq_check_cuda(e);
     }
     if (P.direct) return TQ_OK;   // the decode kernel wrote the output

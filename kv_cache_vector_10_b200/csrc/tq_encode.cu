@@ -635,8 +635,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_v_kernel(const __grid_cons
         }
     }
     // 16-bit inputs: each tile's rows are loaded into registers during the
-    // previous tile's quantization
-    constexpr bool PF = sizeof(Tin) == 2;
+    // previous tile's quantization (d <= 128: a d = 256 row is 128 registers)
+    constexpr bool PF = sizeof(Tin) == 2 && D <= 128;
     RowWords<D> raw;
     if constexpr (PF) {
         if (tb0 < p.T) load_row_words<D, Tin>(src + (tb0 + tid) * p.st, tb0 + tid < p.T, raw);
@@ -799,15 +799,17 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     constexpr int A_BYTES = (D / 64) * ATOM;   // one residual pass
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // misc region [0, 1024): sign masks, squared centroid magnitudes, barriers
-    uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);                 // <= 512 B
-    float *s_mag2 = reinterpret_cast<float *>(smem + 512);                  // [16]
+    // misc region [0, MISC): sign masks (up to MISC / 2 bytes), squared
+    // centroid magnitudes, barriers
+    constexpr int MISC = D > 128 ? 2048 : 1024;
+    uint32_t *s_mask = reinterpret_cast<uint32_t *>(smem);
+    float *s_mag2 = reinterpret_cast<float *>(smem + MISC / 2);             // [16]
     // [0] S loaded, [1] QJL MMA done, [2] Q loaded, [3] rotation MMA done (dense rotation)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 768);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + MISC / 2 + 256);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 4);
     int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
     const int M = p.M;
-    uint8_t *sS = smem + 1024;                                              // [D/64][M rows][128 B]
+    uint8_t *sS = smem + MISC;                                              // [D/64][M rows][128 B]
     uint8_t *sA = sS + (D / 64) * M * 128;                                   // [pass][D/64][128 rows][128 B]
     uint8_t *sQ = sA + 2 * A_BYTES;                                          // dense rotation: [2][D/64][D][128 B]
     const int tid = threadIdx.x, warp = tid / 32;
@@ -852,8 +854,8 @@ __global__ void __launch_bounds__(ENC_ROWS) tq_encode_k_kernel(const __grid_cons
     int ntiles = 0;
     while (ntiles < ENC_TILES && tb0 + (int64_t)ntiles * ENC_ROWS < p.T) ++ntiles;
     // A, B of the first tile; later tiles' rotations overlap the previous MMA,
-    // and (16-bit inputs) their rows are loaded into registers a tile ahead
-    constexpr bool PF = sizeof(Tin) == 2;
+    // and (16-bit inputs, d <= 128) their rows are loaded into registers a tile ahead
+    constexpr bool PF = sizeof(Tin) == 2 && D <= 128;
     RowWords<D> raw;
     float n2 = 0.f;
     if (ntiles > 0 && !*s_abort) {
@@ -1773,7 +1775,7 @@ cudaError_t launch_k(int bits, const EncodeParams &p, const CUtensorMap &mapS, c
                      cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     auto go = [&](auto kern) {
-        size_t smem = 2048 + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
+        size_t smem = (D > 128 ? 3072 : 2048) + (size_t)(D / 64) * p.M * 128 + 2 * (size_t)(D / 64) * ENC_ROWS * 128;
         if (ROT == 1) smem += 2 * (size_t)(D / 64) * D * 128;   // sqrt(d) Q, hi + lo
         // a CTA holding all 512 TMEM columns (d + m > 256) gets an SM to itself
         if (D + p.M > 256 && smem < 120 * 1024) smem = 120 * 1024;
@@ -1833,6 +1835,13 @@ cudaError_t launch_dim(const tq_ctx *ctx, bool keys, const EncodeParams &p, int6
 
 template <typename Tin>
 cudaError_t launch_side(const tq_ctx *ctx, bool keys, const EncodeParams &p, int64_t grid, cudaStream_t s) {
+    if (ctx->d == 256) {
+        // Walsh-Hadamard only: the Haar operands (2 x d x d binary16) do not
+        // fit in shared memory at d = 256 (tq_create_ex rejects that pair)
+        if (ctx->rotation != TQ_ROT_HADAMARD) return cudaErrorInvalidValue;
+        return keys ? launch_k<256, Tin, 0>(ctx->bits, p, ctx->tmap_S, ctx->tmap_Q, grid, s)
+                    : launch_v<256, Tin, 0>(ctx->bits, p, ctx->tmap_Q, grid, s);
+    }
     if (ctx->d == 128) return launch_dim<128, Tin>(ctx, keys, p, grid, s);
     if (ctx->d == 64) return launch_dim<64, Tin>(ctx, keys, p, grid, s);
     return cudaErrorInvalidValue;

@@ -43,12 +43,18 @@ def test_create_validates_arguments_on_host():
     cases = [((0, 3, 128, 42), "TQ_ERR_ZERO_DIM"), ((96, 3, 128, 42), "TQ_ERR_DIM"),
              ((130, 3, 128, 42), "TQ_ERR_DIM"), ((128, 1, 128, 42), "TQ_ERR_BITS"),
              ((128, 6, 128, 42), "TQ_ERR_BITS"), ((128, 3, 0, 42), "TQ_ERR_ZERO_PROJ"),
-             ((128, 3, 48, 42), "TQ_ERR_PROJ"), ((128, 3, 512, 42), "TQ_ERR_PROJ")]
+             ((128, 3, 48, 42), "TQ_ERR_PROJ"), ((128, 3, 512, 42), "TQ_ERR_PROJ"),
+             ((512, 3, 128, 42), "TQ_ERR_DIM"), ((256, 3, 224, 42), "TQ_ERR_PROJ"),
+             ((256, 3, 256, 42), "TQ_ERR_PROJ")]
     for args, want in cases:
         code = lib.tq_create(*args, ctypes.byref(out))
         assert lib.tq_status_string(code).decode() == want, (args, code)
         assert out.value is None
     assert lib.tq_create(128, 3, 128, 42, None) != 0
+    # head_dim 256 runs the Walsh-Hadamard rotation only (the Haar operands
+    # do not fit in a CTA's shared memory)
+    code = lib.tq_create_ex(256, 3, 128, 42, tq.TQ_ROT_HAAR, ctypes.byref(out))
+    assert lib.tq_status_string(code).decode() == "TQ_ERR_DIM" and out.value is None
 
 
 def test_null_and_empty_arguments():
