@@ -20,7 +20,7 @@ OBJ_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libtq.so")
 ROOT = os.path.dirname(HERE)
 
-CU_SOURCES = ["tq_api.cu", "tq_encode.cu", "tq_decode.cu", "tq_aux.cu", "tq_static.cu", "tq_selftest.cu", "tq_split.cu"]
+CU_SOURCES = ["tq_api.cu", "tq_encode.cu", "tq_decode.cu", "tq_decode_mma.cu", "tq_aux.cu", "tq_static.cu", "tq_selftest.cu", "tq_split.cu"]
 CPP_SOURCES = ["tq_tables.cpp"]
 HEADERS = ["tq_internal.cuh", "tq_decode.cuh"]
 

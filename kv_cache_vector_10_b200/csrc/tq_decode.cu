@@ -22,6 +22,9 @@
 // Every query of a kv-head group (GQA) and every sequence of a shared
 // segment reads the same staged tile.
 #include <algorithm>
+#include <climits>
+#include <cstdlib>
+#include <cstring>
 #include <cmath>
 #include <vector>
 
@@ -516,10 +519,21 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
 
 // ------------------------------------------------------------------ planning
 struct SegPlan {
-    int qc;
+    int qc;                    // queries per CTA (TQ_MMA_QUERIES: the tensor-core decode)
     int n_qchunks, n_splits, split_len;
     int64_t part_floats, qprep_floats;
 };
+
+// Queries per kv head (sequences x query heads of a group) from which a
+// segment is decoded on the tensor cores, where its format fits them.
+// TQ_DECODE_PATH=lut keeps every segment on the lookup-table decode and
+// TQ_DECODE_PATH=mma sends every segment that fits to the tensor cores.
+int mma_min_queries() {
+    const char *e = getenv("TQ_DECODE_PATH");
+    if (e && strcmp(e, "lut") == 0) return 1 << 30;
+    if (e && strcmp(e, "mma") == 0) return 1;
+    return 16;
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -546,47 +560,57 @@ int decode_nbuf(int d, int bv, int qc, int krow, int vrow, int M) {
 
 void plan_segments(const tq_segment *segs, int n_segs, int Hq, int Hkv, int n_sms, std::vector<SegPlan> &out) {
     const int G = Hq / Hkv;
+    const int qmin = mma_min_queries();
     out.resize(n_segs);
-    int64_t work = 0;
     for (int s = 0; s < n_segs; ++s) {
         const int nq = segs[s].n_seqs * G;
         SegPlan &p = out[s];
         const tq_ctx *c = segs[s].ctx;
         const int krow = (int)tq_row_bytes(c, TQ_KEYS), vrow = (int)tq_row_bytes(c, TQ_VALUES);
-        p.qc = nq >= 4 ? 4 : nq >= 2 ? 2 : 1;
-        while (p.qc > 1 && decode_nbuf(c->d, c->BV, p.qc, krow, vrow, c->m) == 0) p.qc /= 2;
+        if (nq >= qmin && c->rotation != TQ_ROT_HAAR && tq_decode_mma_fits(c->d, c->m, c->BK, c->BV, krow, vrow)) {
+            p.qc = TQ_MMA_QUERIES;
+        } else {
+            p.qc = nq >= 4 ? 4 : nq >= 2 ? 2 : 1;
+            while (p.qc > 1 && decode_nbuf(c->d, c->BV, p.qc, krow, vrow, c->m) == 0) p.qc /= 2;
+        }
         p.n_qchunks = (nq + p.qc - 1) / p.qc;
-        work += segs[s].n_tokens * (int64_t)Hkv * p.n_qchunks;
     }
-    // Split length: one value for all segments, chosen to minimise the
+    // Split lengths, one per decode kind, each chosen to minimise the
     // estimated time = waves x (tokens per CTA + fixed per-CTA cost), so the
     // last wave is not mostly empty.  One decode CTA per SM is resident.
-    (void)work;
-    const int64_t kFixedTokens = 256;   // per-CTA set-up (tables, merge) in token-equivalents
-    int64_t Tmax = 0;
-    for (int s = 0; s < n_segs; ++s) Tmax = std::max<int64_t>(Tmax, segs[s].n_tokens);
-    int64_t bestL = TQ_DEC_SPLIT_UNIT;
-    double best = 1e300;
-    for (int64_t L = TQ_DEC_SPLIT_UNIT; ; L += TQ_DEC_SPLIT_UNIT) {
-        int64_t items = 0;
+    auto choose = [&](bool mma, int64_t unit, int64_t fixed) {
+        int64_t Tmax = 0;
         for (int s = 0; s < n_segs; ++s)
-            items += (int64_t)Hkv * out[s].n_qchunks * std::max<int64_t>(1, (segs[s].n_tokens + L - 1) / L);
-        const int64_t waves = (items + n_sms - 1) / std::max(n_sms, 1);
-        const double t = (double)waves * (double)(std::min(L, std::max<int64_t>(Tmax, 1)) + kFixedTokens);
-        if (t < best - 1e-9) {
-            best = t;
-            bestL = L;
+            if ((out[s].qc == TQ_MMA_QUERIES) == mma) Tmax = std::max<int64_t>(Tmax, segs[s].n_tokens);
+        int64_t bestL = unit;
+        double best = 1e300;
+        for (int64_t L = unit;; L += unit) {
+            int64_t items = 0;
+            for (int s = 0; s < n_segs; ++s)
+                if ((out[s].qc == TQ_MMA_QUERIES) == mma)
+                    items += (int64_t)Hkv * out[s].n_qchunks * std::max<int64_t>(1, (segs[s].n_tokens + L - 1) / L);
+            const int64_t waves = (items + n_sms - 1) / std::max(n_sms, 1);
+            const double t = (double)waves * (double)(std::min(L, std::max<int64_t>(Tmax, 1)) + fixed);
+            if (t < best - 1e-9) {
+                best = t;
+                bestL = L;
+            }
+            if (L >= Tmax) break;
         }
-        if (L >= Tmax) break;
-    }
+        return bestL;
+    };
+    // lookup-table decode: per-CTA set-up (tables, merge) ~ 256 tokens;
+    // tensor-core decode: 64-token tiles, set-up and output ~ 3 tiles
+    const int64_t L_lut = choose(false, TQ_DEC_SPLIT_UNIT, 256);
+    const int64_t L_mma = choose(true, 64, 192);
     const int d = segs[0].ctx->d;
     for (int s = 0; s < n_segs; ++s) {
         SegPlan &p = out[s];
         const int64_t T = segs[s].n_tokens;
-        const int64_t ns = std::max<int64_t>(1, (T + bestL - 1) / bestL);
-        const int64_t sl = bestL;
+        const int64_t L = p.qc == TQ_MMA_QUERIES ? L_mma : L_lut;
+        const int64_t ns = std::max<int64_t>(1, (T + L - 1) / L);
         p.n_splits = (int)ns;
-        p.split_len = (int)sl;
+        p.split_len = (int)L;
         p.part_floats = (int64_t)ns * segs[s].n_seqs * Hq * tq_part_floats(d);
         p.qprep_floats = (int64_t)segs[s].n_seqs * Hq * (d + segs[s].ctx->m);
     }
@@ -767,6 +791,7 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         for (int i = 0; i < d.n_planes; ++i) d.plane_sets[i] = sigma_set(c->BK, i);
         sigma_alphas(c, d.alpha);
         for (int i = 0; i < 32; ++i) d.vtab[i] = i < c->LV ? c->cv[i] : 0.f;
+        for (int i = 0; i < 16; ++i) d.ktab[i] = i < (1 << c->BK) ? c->ck[i] : 0.f;
         qoff += pl[s].qprep_floats;
         poff += pl[s].part_floats;
     }
@@ -802,6 +827,11 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
         for (int s = 0; s < n_segs; ++s)
             if (!done[s] && same(s)) done[s] = 1;
         if (items == 0) continue;
+        if (qc == TQ_MMA_QUERIES) {
+            e = tq_launch_decode_mma(Pg, items, P.d, m, bk, P.seg[s0].krow, P.seg[s0].vrow, stream);
+            if (e != cudaSuccess) return tq_check_cuda(e);
+            continue;
+        }
         e = P.d == 256   ? launch_decode_dim<256>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
             : P.d == 128 ? launch_decode_dim<128>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream)
                          : launch_decode_dim<64>(bk + 1, qc, Pg, items, P.seg[s0].krow, P.seg[s0].vrow, m, stream);

@@ -32,6 +32,7 @@ struct SegDesc {
     uint32_t plane_sets[8];    // bit mask of index planes XOR-ed into sigma-plane s
     float alpha[8];            // Walsh coefficient of sigma-plane s
     float vtab[32];            // value centroids, indexed by code
+    float ktab[16];            // key centroids, indexed by code (tensor-core decode)
 };
 
 struct DecodePlan {
@@ -62,6 +63,13 @@ struct TqAppend {
     tq_dtype dtype;
     const uint8_t *flags;      // [n_segs]: 1 = the segment receives the new rows
 };
+
+// Tensor-core decode (tq_decode_mma.cu): whether a segment's format fits it,
+// and one launch over the items of the plan's segments with bk = `bk`.
+bool tq_decode_mma_fits(int d, int m, int bk, int bv, int krow, int vrow);
+cudaError_t tq_launch_decode_mma(const DecodePlan &P, int64_t items, int d, int m, int bk, int krow, int vrow,
+                                 cudaStream_t stream);
+#define TQ_MMA_QUERIES 128    // queries per tensor-core decode CTA
 
 // Floats per partial slot.
 __host__ __device__ constexpr int tq_part_floats(int d) { return d + 4; }
