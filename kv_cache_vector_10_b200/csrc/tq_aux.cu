@@ -481,21 +481,26 @@ __device__ void append_row(bool key, const void *src, int64_t src_off, int dt, c
     __syncthreads();
 }
 
-// Blocks [0, query blocks): one per (segment, seq_local, head), the prepared
-// query [q_rot | S q_rot].  Blocks after those: one per (appending segment,
-// kv head), the append step's new key and value rows.
+// Query heads per pass of a query-preparation block.
+constexpr int QP_GROUP = 4;
+
+// Blocks [0, query blocks): one per (segment, seq_local, kv head), the
+// prepared queries [q_rot | S q_rot] of the G query heads of the group, in
+// passes of up to QP_GROUP heads.  Thread i's row of S (projection i) is
+// requested before the first rotation and serves every head of the group.
+// Blocks after those: one per (appending segment, kv head), the append
+// step's new key and value rows.
 template <int D, typename Tq>
 __global__ void __launch_bounds__(qprep_threads(D)) tq_qprep_kernel(const __grid_constant__ DecodePlan P, const void *q) {
     tqdev::grid_dep_trigger();   // the decode CTAs may start their set-up now
-    __shared__ float s_in[D];
-    __shared__ __align__(16) float s_qr[D];
-    __shared__ float s_sq[256];
+    __shared__ __align__(16) float s_in[QP_GROUP][D];   // raw queries (Haar), append scratch
+    __shared__ __align__(16) float s_qr[QP_GROUP][D];
     __shared__ float s_red[qprep_threads(D) / 32];
     __shared__ uint8_t s_idx[D];
     int s = 0;
     int64_t blk = blockIdx.x;
     for (; s < P.n_segs; ++s) {
-        const int64_t n = (int64_t)P.seg[s].n_seqs * P.Hq;
+        const int64_t n = (int64_t)P.seg[s].n_seqs * P.Hkv;
         if (blk < n) break;
         blk -= n;
     }
@@ -510,21 +515,135 @@ __global__ void __launch_bounds__(qprep_threads(D)) tq_qprep_kernel(const __grid
         const SegDesc &g = P.seg[s];
         const int h = (int)blk;
         const int64_t src = ((int64_t)g.first_seq * P.Hkv + h) * D;
-        append_row<D>(true, P.k_new, src, P.kv_dtype, g, h, g.T - 1, s_in, s_qr, s_red, s_idx);
-        append_row<D>(false, P.v_new, src, P.kv_dtype, g, h, g.T - 1, s_in, s_qr, s_red, s_idx);
+        append_row<D>(true, P.k_new, src, P.kv_dtype, g, h, g.T - 1, s_in[0], s_qr[0], s_red, s_idx);
+        append_row<D>(false, P.v_new, src, P.kv_dtype, g, h, g.T - 1, s_in[0], s_qr[0], s_red, s_idx);
         return;
     }
     const SegDesc &g = P.seg[s];
-    const int seq_local = (int)(blk / P.Hq), j = (int)(blk % P.Hq);
+    const int seq_local = (int)(blk / P.Hkv), h = (int)(blk % P.Hkv);
     const int seq = g.first_seq + seq_local;
-    const int h = j / P.G;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) s_in[i] = load_as_float<Tq>(q, ((int64_t)seq * P.Hq + j) * D + i);
-    __syncthreads();
-    prep_query<D>(s_in, g.signs + (int64_t)h * (D / 32), g.S + (int64_t)h * g.m * D, g.m, s_qr, s_sq,
-                  g.Q ? g.Q + (int64_t)h * D * D : nullptr);
-    float *dst = P.qprep + g.qprep_base + ((int64_t)seq_local * P.Hq + j) * (D + g.m);
-    for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = s_qr[i];
-    for (int i = threadIdx.x; i < g.m; i += blockDim.x) dst[D + i] = s_sq[i];
+    const int M = g.m, G = P.G;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const __half *Sh = g.S + (int64_t)h * M * D;
+    const float *Qh = g.Q ? g.Q + (int64_t)h * D * D : nullptr;
+    // this thread's row of S, kept for every pass (head_dim <= 128)
+    constexpr bool KEEP = D <= 128;
+    uint4 wkeep[KEEP ? D / 8 : 1];
+    if (KEEP && tid < M) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(Sh + (int64_t)tid * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) wkeep[c] = __ldg(row + c);
+    }
+    for (int g0 = 0; g0 < G; g0 += QP_GROUP) {
+        const int ng = min(QP_GROUP, G - g0);
+        const int64_t qrow0 = (int64_t)seq * P.Hq + h * G + g0;   // first query row of the pass
+        if (Qh) {
+            // Haar rotation: q_rot = Q q, one output coordinate per thread
+            for (int e = tid; e < ng * D; e += blockDim.x) s_in[e / D][e % D] = load_as_float<Tq>(q, qrow0 * D + e);
+            __syncthreads();
+            for (int i = tid; i < D; i += blockDim.x) {
+                const float4 *row = reinterpret_cast<const float4 *>(Qh + (int64_t)i * D);
+                float a0[QP_GROUP], a1[QP_GROUP];
+#pragma unroll
+                for (int k = 0; k < QP_GROUP; ++k) a0[k] = a1[k] = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < D / 4; ++c) {
+                    const float4 w = __ldg(row + c);
+#pragma unroll
+                    for (int k = 0; k < QP_GROUP; ++k) {
+                        if (k < ng) {
+                            a0[k] = fmaf(w.x, s_in[k][4 * c], a0[k]);
+                            a1[k] = fmaf(w.y, s_in[k][4 * c + 1], a1[k]);
+                            a0[k] = fmaf(w.z, s_in[k][4 * c + 2], a0[k]);
+                            a1[k] = fmaf(w.w, s_in[k][4 * c + 3], a1[k]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < QP_GROUP; ++k)
+                    if (k < ng) s_qr[k][i] = a0[k] + a1[k];
+            }
+        } else if (warp < ng) {
+            // Walsh-Hadamard: warp k rotates head g0 + k (lane l holds
+            // coordinates l + 32 i: the stages of stride >= 32 in registers,
+            // the others across lanes by shuffles)
+            constexpr int V = D / 32;
+            const uint32_t *sg = g.signs + (int64_t)h * (D / 32);
+            float x[V];
+#pragma unroll
+            for (int k = 0; k < V; ++k) {
+                const int j = lane + 32 * k;
+                const float v = load_as_float<Tq>(q, (qrow0 + warp) * D + j);
+                x[k] = ((sg[j / 32] >> (j % 32)) & 1) ? -v : v;
+            }
+#pragma unroll
+            for (int len = 1; len < V; len <<= 1)
+#pragma unroll
+                for (int k = 0; k < V; k += 2 * len)
+#pragma unroll
+                    for (int kk = k; kk < k + len; ++kk) {
+                        const float a = x[kk], b = x[kk + len];
+                        x[kk] = a + b;
+                        x[kk + len] = a - b;
+                    }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const bool upper = (lane & o) != 0;
+#pragma unroll
+                for (int k = 0; k < V; ++k) {
+                    const float y = __shfl_xor_sync(0xffffffffu, x[k], o);
+                    x[k] = upper ? y - x[k] : x[k] + y;
+                }
+            }
+            const float sc = rsqrtf((float)D);
+#pragma unroll
+            for (int k = 0; k < V; ++k) s_qr[warp][lane + 32 * k] = x[k] * sc;
+        }
+        __syncthreads();
+        float *dst0 = P.qprep + g.qprep_base + ((int64_t)seq_local * P.Hq + h * G + g0) * (D + M);
+        // S q_rot: projection i of every head of the pass from one row of S
+        for (int i = tid; i < M; i += blockDim.x) {
+            uint4 w[D / 8];
+            if (KEEP && i == tid) {
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) w[c] = wkeep[KEEP ? c : 0];
+            } else {
+                const uint4 *row = reinterpret_cast<const uint4 *>(Sh + (int64_t)i * D);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) w[c] = __ldg(row + c);
+            }
+            float acc0[QP_GROUP], acc1[QP_GROUP];
+#pragma unroll
+            for (int k = 0; k < QP_GROUP; ++k) acc0[k] = acc1[k] = 0.f;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].x));
+                const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].y));
+                const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].z));
+                const float2 f3 = __half22float2(*reinterpret_cast<const __half2 *>(&w[c].w));
+#pragma unroll
+                for (int k = 0; k < QP_GROUP; ++k) {
+                    if (k < ng) {
+                        const float4 qa = reinterpret_cast<const float4 *>(s_qr[k])[2 * c];
+                        const float4 qb = reinterpret_cast<const float4 *>(s_qr[k])[2 * c + 1];
+                        acc0[k] = fmaf(f0.x, qa.x, acc0[k]);
+                        acc1[k] = fmaf(f0.y, qa.y, acc1[k]);
+                        acc0[k] = fmaf(f1.x, qa.z, acc0[k]);
+                        acc1[k] = fmaf(f1.y, qa.w, acc1[k]);
+                        acc0[k] = fmaf(f2.x, qb.x, acc0[k]);
+                        acc1[k] = fmaf(f2.y, qb.y, acc1[k]);
+                        acc0[k] = fmaf(f3.x, qb.z, acc0[k]);
+                        acc1[k] = fmaf(f3.y, qb.w, acc1[k]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < QP_GROUP; ++k)
+                if (k < ng) dst0[(int64_t)k * (D + M) + D + i] = acc0[k] + acc1[k];
+        }
+        for (int e = tid; e < ng * D; e += blockDim.x) dst0[(int64_t)(e / D) * (D + M) + e % D] = s_qr[e / D][e % D];
+        __syncthreads();
+    }
 }
 
 template <typename To>
@@ -661,7 +780,7 @@ tq_status tq_launch_dequant(tq_ctx *ctx, const tq_codes *codes, int64_t T, float
 
 cudaError_t tq_launch_qprep(const DecodePlan &P, const void *q, tq_dtype dt, cudaStream_t stream) {
     int64_t blocks = P.n_append_blocks;
-    for (int s = 0; s < P.n_segs; ++s) blocks += (int64_t)P.seg[s].n_seqs * P.Hq;
+    for (int s = 0; s < P.n_segs; ++s) blocks += (int64_t)P.seg[s].n_seqs * P.Hkv;
     if (blocks == 0) return cudaSuccess;
 #define TQ_QPREP(DD, TT) tq_qprep_kernel<DD, TT><<<(unsigned)blocks, qprep_threads(DD), 0, stream>>>(P, q)
     if (P.d == 256) {

@@ -803,10 +803,13 @@ tq_status tq_launch_decode(const tq_segment *segs, int n_segs, const void *q, tq
     cudaError_t e = tq_launch_qprep(P, q, q_dtype, stream);
     if (e != cudaSuccess) return tq_check_cuda(e);
     // one launch per (bits, queries per CTA, row format) group: the CTA's
-    // shared memory is sized by the group's row lengths
+    // shared memory is sized by the group's row lengths.  Lookup-table groups
+    // go first: a tensor-core launch after them fills the SMs they leave
+    // idle and those that finish first.
     std::vector<int> done(n_segs, 0);
+    for (int pass = 0; pass < 2; ++pass)
     for (int s0 = 0; s0 < n_segs; ++s0) {
-        if (done[s0]) continue;
+        if (done[s0] || (pl[s0].qc == TQ_MMA_QUERIES) != (pass == 1)) continue;
         const int bk = P.seg[s0].bk, qc = pl[s0].qc, m = P.seg[s0].m, kr = P.seg[s0].krow;
         auto same = [&](int s) {
             return P.seg[s].bk == bk && pl[s].qc == qc && P.seg[s].m == m && P.seg[s].krow == kr;

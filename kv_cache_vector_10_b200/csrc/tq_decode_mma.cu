@@ -123,14 +123,11 @@ __device__ __forceinline__ void wht32(float (&x)[32]) {
     }
 }
 
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, float (&v)[8]) {
-    uint32_t r[8];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7])
-                 : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tqdev::smem_u32(smem)), "l"(gmem),
+                 "r"(src_bytes)
+                 : "memory");
 }
 
 // One output element in the caller's type.
@@ -513,35 +510,19 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) tq_decode_mma_kernel(const __g
             // coalesced in the operand buffers: row rr, 16-byte chunk k at
             // chunk k ^ (rr % 8)
             constexpr int QCH = (D + MP) / 4;
-            constexpr int KPL = (QCH + 31) / 32;
             uint8_t *stg = sm + L::OFF_K;
-#pragma unroll
-            for (int b8 = 0; b8 < MMA_Q / SM_WARPS; b8 += 4) {
-                float4 buf[4][KPL];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int rr = warp + SM_WARPS * (b8 + u);
-                    const int q2 = qchunk * MMA_Q + rr;
-                    const float4 *src = q2 < nq ? reinterpret_cast<const float4 *>(
-                                                      P.qprep + g.qprep_base +
-                                                      ((int64_t)(q2 / P.G) * P.Hq + h * P.G + q2 % P.G) * (D + MP))
-                                                : nullptr;
-#pragma unroll
-                    for (int kk = 0; kk < KPL; ++kk) {
-                        const int k = lane + 32 * kk;
-                        buf[u][kk] = (src && k < QCH) ? src[k] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int rr = warp + SM_WARPS * (b8 + u);
-#pragma unroll
-                    for (int kk = 0; kk < KPL; ++kk) {
-                        const int k = lane + 32 * kk;
-                        if (k < QCH) *reinterpret_cast<float4 *>(stg + rr * QCH * 16 + ((k ^ (rr & 7)) << 4)) = buf[u][kk];
-                    }
-                }
+            const float *qp0 = P.qprep + g.qprep_base;
+#pragma unroll 1
+            for (int rr = warp; rr < MMA_Q; rr += SM_WARPS) {
+                const int q2 = qchunk * MMA_Q + rr;
+                const bool ok = q2 < nq;
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    ok ? qp0 + ((int64_t)(q2 / P.G) * P.Hq + h * P.G + q2 % P.G) * (D + MP) : qp0);
+                for (int k = lane; k < QCH; k += 32)
+                    cp_async16(stg + rr * QCH * 16 + ((k ^ (rr & 7)) << 4), src + (ok ? k : 0), ok ? 16u : 0u);
             }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
             tqdev::named_sync(1, 32 * SM_WARPS);
             // ---- bfloat16 hi + lo into TMEM (column c: elements 2c, 2c + 1):
             // half 0 writes q_rot, half 1 writes S q_rot
@@ -677,78 +658,81 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) tq_decode_mma_kernel(const __g
             }
             if (!failed && !bar_wait_warp(&bars.p_free, (uint32_t)((nt - 1) & 1))) failed = true;
         }
-        // ---- the row's sum of weights, then rotate back (out = D H O / d)
+        // ---- the row's sum of weights, then rotate back: out = D H O / d with
+        // H_d = H_2 x H_{d/2}: each half transforms its d/2 columns in
+        // registers, and the halves' last stage meets in shared memory
+        constexpr int HC = D / 2;   // output columns per half
         lx[half * 128 + r] = l_part;
         const bool paired = pair_sync();
         const float l_run = lx[r] + lx[128 + r];
         const bool have = run && !failed && paired;
+        float o[HC];
         if (have) {
-            // H_32 on this half's 32-column chunks (TMEM as scratch)
             tqdev::tc_fence_after();
-#pragma unroll 1
-            for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
-                float o[32];
-                tqdev::tmem_ld_32x32b_x32(tl + L::COL_O + 32 * c, o);
-                wht32(o);
-                tqdev::tmem_st_32x32b_x32(tl + L::COL_O + 32 * c, o);
+#pragma unroll
+            for (int c = 0; c < HC / 32; ++c) {
+                float t32[32];
+                tqdev::tmem_ld_32x32b_x32(tl + L::COL_O + HC * half + 32 * c, t32);
+                wht32(t32);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[32 * c + k] = t32[k];
             }
-            tqdev::tmem_wait_st();
-            tqdev::tc_fence_before();
+#pragma unroll
+            for (int len = 32; len < HC; len <<= 1)
+#pragma unroll
+                for (int k = 0; k < HC; ++k) {
+                    if (k & len) continue;
+                    const float x0 = o[k], x1 = o[k + len];
+                    o[k] = x0 + x1;
+                    o[k + len] = x0 - x1;
+                }
+        } else {
+#pragma unroll
+            for (int k = 0; k < HC; ++k) o[k] = 0.f;
         }
-        const bool both = pair_sync() && have;   // both halves' chunks transformed
-        const float inv_d = 1.f / (float)D;
-        const uint32_t *sgn = g.signs + (int64_t)h * (D / 32);
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-        const int64_t obase = ((int64_t)(g.first_seq + seq_local) * P.Hq + jh) * D;
-        float *ost = reinterpret_cast<float *>(sm + L::OFF_K);   // output staging: row r, 16-byte chunk k at k ^ (r % 8)
-        if (both) tqdev::tc_fence_after();
-#pragma unroll 1
-        for (int rb = 2 * half; rb < 2 * half + 2; ++rb) {
-            // the butterflies across the 32-column chunks (H_d = H_{d/32} x H_32)
-            float v[D / 32][8];
-            if (both) {
+        // exchange buffers [half][row][HC] and the output staging [row][d],
+        // both with 16-byte chunk c of row r at chunk c ^ (r % 8)
+        float *xo = reinterpret_cast<float *>(sm + L::OFF_K);
+        float *ost = xo + 2 * 128 * HC;
+        {
+            float *mine = xo + (half * 128 + r) * HC;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) tmem_ld_x8(tl + L::COL_O + 32 * c + 8 * rb, v[c]);
-                tqdev::tmem_wait_ld();
-            } else {
+            for (int c = 0; c < HC / 4; ++c)
+                *reinterpret_cast<float4 *>(mine + ((c ^ (r & 7)) << 2)) =
+                    make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        const bool both = pair_sync() && have;
+        const float *other = xo + ((half ^ 1) * 128 + r) * HC;
+        const float sc = both ? 1.f / (float)D : 0.f;
+        uint32_t sgn[HC / 32];   // sign words of this half's output columns
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
+        for (int c = 0; c < HC / 32; ++c) sgn[c] = __ldg(g.signs + (int64_t)h * (D / 32) + (HC / 32) * half + c);
+        // half 0: a + b (output columns [0, d/2)); half 1: a - b, a being half 0's
+        const float sa = half == 0 ? 1.f : -1.f;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) v[c][k] = 0.f;
+        for (int c = 0; c < HC / 4; ++c) {
+            const float4 p4 = *reinterpret_cast<const float4 *>(other + ((c ^ (r & 7)) << 2));
+            o[4 * c] = (p4.x + sa * o[4 * c]) * sc;
+            o[4 * c + 1] = (p4.y + sa * o[4 * c + 1]) * sc;
+            o[4 * c + 2] = (p4.z + sa * o[4 * c + 2]) * sc;
+            o[4 * c + 3] = (p4.w + sa * o[4 * c + 3]) * sc;
+        }
+#pragma unroll
+        for (int k = 0; k < HC; ++k)
+            if ((sgn[k >> 5] >> (k & 31)) & 1u) o[k] = -o[k];
+        if (P.direct) {
+            if (qvalid) {
+                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                const int64_t obase = ((int64_t)(g.first_seq + seq_local) * P.Hq + jh) * D + HC * half;
+#pragma unroll
+                for (int k = 0; k < HC; ++k) store_out_elem(P.out, obase + k, o[k] * inv_l, P.out_dtype);
             }
+        } else {
 #pragma unroll
-            for (int len = 1; len < D / 32; len <<= 1)
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    if (c & len) continue;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float x0 = v[c][k], x1 = v[c + len][k];
-                        v[c][k] = x0 + x1;
-                        v[c + len][k] = x0 - x1;
-                    }
-                }
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                const uint32_t sw = sgn[c];
-                float o8[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float x = v[c][k] * inv_d;
-                    o8[k] = ((sw >> (8 * rb + k)) & 1u) ? -x : x;
-                }
-                const int j0 = 32 * c + 8 * rb;
-                if (P.direct) {
-                    if (qvalid)
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) store_out_elem(P.out, obase + j0 + k, o8[k] * inv_l, P.out_dtype);
-                } else {
-                    const int k0 = j0 / 4;
-                    *reinterpret_cast<float4 *>(ost + r * D + (((k0) ^ (r & 7)) << 2)) =
-                        make_float4(o8[0], o8[1], o8[2], o8[3]);
-                    *reinterpret_cast<float4 *>(ost + r * D + (((k0 + 1) ^ (r & 7)) << 2)) =
-                        make_float4(o8[4], o8[5], o8[6], o8[7]);
-                }
+            for (int c = 0; c < HC / 4; ++c) {
+                const int k = (HC * half) / 4 + c;   // 16-byte chunk of the output row
+                *reinterpret_cast<float4 *>(ost + r * D + ((k ^ (r & 7)) << 2)) =
+                    make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
             }
         }
         if (half == 0) {
@@ -759,17 +743,22 @@ __global__ void __launch_bounds__(MMA_THREADS, 1) tq_decode_mma_kernel(const __g
             // coalesced partials: one warp per row, [m, l, 0, 0 | o]
             tqdev::named_sync(1, 32 * SM_WARPS);
             constexpr int OCH = D / 4;   // 16-byte chunks of a row's output
+            const int rows = min(MMA_Q, nq - qchunk * MMA_Q);
+            int sl = (qchunk * MMA_Q + warp) / P.G, gq = (qchunk * MMA_Q + warp) % P.G;
 #pragma unroll 1
-            for (int rr = warp; rr < MMA_Q; rr += SM_WARPS) {
-                const int q2 = qchunk * MMA_Q + rr;
-                if (q2 >= nq) break;
-                const int sl = q2 / P.G, j2 = h * P.G + q2 % P.G;
-                float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + sl) * P.Hq + j2) * tq_part_floats(D);
+            for (int rr = warp; rr < rows; rr += SM_WARPS) {
+                float *dst = P.part + (g.part_base + ((int64_t)split * g.n_seqs + sl) * P.Hq + h * P.G + gq) * tq_part_floats(D);
                 if (lane < OCH) {
                     const float4 x = *reinterpret_cast<const float4 *>(ost + rr * D + ((lane ^ (rr & 7)) << 2));
                     reinterpret_cast<float4 *>(dst + 4)[lane] = x;
                 }
                 if (lane == 0) reinterpret_cast<float4 *>(dst)[0] = make_float4(mlr[2 * rr], mlr[2 * rr + 1], 0.f, 0.f);
+                // next row of this warp: query index + SM_WARPS
+                gq += SM_WARPS;
+                while (gq >= P.G) {
+                    gq -= P.G;
+                    ++sl;
+                }
             }
         }
     }
