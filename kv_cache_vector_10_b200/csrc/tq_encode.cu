@@ -1206,10 +1206,10 @@ struct PipeLayout {
     static constexpr int THREADS = 32 * (4 * NG + 1);    // + the producer warp
     static constexpr int XBOX = ENC_ROWS * 128;          // one 64-column box of a tile (16 KB)
     static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
-    static constexpr int NS = KEYS ? 2 : 4;              // stages of the row ring
+    static constexpr int NS = KEYS ? 1 : 4;              // stages of the row ring
     static constexpr int OFF_HD = NS * XSTAGE;           // rotation operand [d/64][d][128 B]
-    static constexpr int OFF_A = OFF_HD + D * D * 2;     // keys: residual operand hi, lo
-    static constexpr int OFF_S = OFF_A + (KEYS ? 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
+    static constexpr int OFF_A = OFF_HD + D * D * 2;     // keys: residual operand hi, lo of each group
+    static constexpr int OFF_S = OFF_A + (KEYS ? NG * 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
     static constexpr int FIXED = 1024 + OFF_S;           // dynamic bytes before S (with alignment slack)
 };
 
@@ -1250,7 +1250,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
     uint8_t *sA = sm + L::OFF_A;
     uint8_t *sS = sm + L::OFF_S;
     __shared__ __align__(8) uint64_t bar_xfull[NS], bar_xfree[NS], bar_rot[NG], bar_ufree[NG], bar_qjl[NG];
-    __shared__ __align__(8) uint64_t bar_afull, bar_afree, bar_hd, bar_s;
+    __shared__ __align__(8) uint64_t bar_afull[NG], bar_afree[NG], bar_hd, bar_s;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_mag2[16];
@@ -1285,8 +1285,10 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
             tqdev::mbar_init(&bar_ufree[i], 128);
             tqdev::mbar_init(&bar_qjl[i], 1);
         }
-        tqdev::mbar_init(&bar_afull, 128);
-        tqdev::mbar_init(&bar_afree, 1);
+        for (int i = 0; i < NG; ++i) {
+            tqdev::mbar_init(&bar_afull[i], 128);
+            tqdev::mbar_init(&bar_afree[i], 1);
+        }
         tqdev::mbar_init(&bar_hd, 1);
         tqdev::mbar_init(&bar_s, 1);
         s_abort = tqdev::status_aborted(p.status) ? 1 : 0;
@@ -1371,7 +1373,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                     const int j = next_qjl, h = head_of(j);
                     if (h != s_head && !s_busy) {
                         // the previous projection (old S) must be complete
-                        if (j == 0 || mbar_test(&bar_afree, (uint32_t)((j - 1) & 1))) {
+                        if (j == 0 || mbar_test(&bar_afree[(j - 1) % NG], (uint32_t)(((j - 1) / NG) & 1))) {
                             tqdev::mbar_expect_tx(&bar_s, p.s_bytes);
 #pragma unroll
                             for (int a = 0; a < D / 64; ++a)
@@ -1386,12 +1388,12 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                         s_busy = false;
                         progress = true;
                     }
-                    if (h == s_head && !s_busy && mbar_test(&bar_afull, (uint32_t)(j & 1))) {
+                    if (h == s_head && !s_busy && mbar_test(&bar_afull[j % NG], (uint32_t)((j / NG) & 1))) {
                         tqdev::tc_fence_after();
                         const uint32_t col = (uint32_t)(j % NG) * GSTRIDE + (uint32_t)D;
 #pragma unroll
                         for (int pass = 0; pass < 2; ++pass) {
-                            const uint32_t abase = tqdev::smem_u32(sA + pass * L::XSTAGE);
+                            const uint32_t abase = tqdev::smem_u32(sA + ((j % NG) * 2 + pass) * L::XSTAGE);
                             const uint32_t bbase = tqdev::smem_u32(sS);
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
@@ -1402,7 +1404,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                             }
                         }
                         tqdev::mma_commit(&bar_qjl[j % NG]);
-                        tqdev::mma_commit(&bar_afree);
+                        tqdev::mma_commit(&bar_afree[j % NG]);
                         ++next_qjl;
                         progress = true;
                     }
@@ -1435,7 +1437,8 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                 tqdev::mbar_wait_bounded(&bar_xfull[li % NS], (uint32_t)((li / NS) & 1));
             for (int li = xfree_seen; li < next_rot; ++li)             // rotations not seen through xfree
                 tqdev::mbar_wait_bounded(&bar_xfree[li % NS], (uint32_t)((li / NS) & 1));
-            if (next_qjl > 0) tqdev::mbar_wait_bounded(&bar_afree, (uint32_t)((next_qjl - 1) & 1));
+            for (int j = next_qjl - NG < 0 ? 0 : next_qjl - NG; j < next_qjl; ++j)
+                tqdev::mbar_wait_bounded(&bar_afree[j % NG], (uint32_t)((j / NG) & 1));
             if (hd_busy) tqdev::mbar_wait_bounded(&bar_hd, hd_ph);
             if (s_busy) tqdev::mbar_wait_bounded(&bar_s, s_ph);
         }
@@ -1445,6 +1448,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
         const int row = ((warp & 3) << 5) | lane;               // tile row = TMEM lane
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)g * GSTRIDE;
         const uint32_t tU = tl, tC = tl + (uint32_t)D;          // keys: C, then P, at tC
+        uint8_t *sAg = sA + g * 2 * L::XSTAGE;                  // keys: this group's residual operand
         bool failed = false;
         // keys: the sign plane of the group's previous tile is stored after this
         // tile's |u|^2 pass, so its QJL projection overlaps that pass
@@ -1658,8 +1662,8 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                 float e2a = n2 - 2.f * ns * uc + ns * ns * c2;
                 e2a = fmaxf(e2a, 1e-10f * n2);
                 const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
-                // ---- residual operand (the shared buffer is taken in tile order)
-                if (li > 0 && !warp_wait(&bar_afree, (uint32_t)((li - 1) & 1))) {
+                // ---- residual operand (the group's buffer, free once its previous projection is done)
+                if (k > 0 && !warp_wait(&bar_afree[g], (uint32_t)((k - 1) & 1))) {
                     failed = true;
                     break;
                 }
@@ -1689,15 +1693,15 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                             }
                             const int kk = 4 * c + 2 * half + jh;             // 16-byte unit of the row
                             const int off = (kk / 8) * L::XBOX + row * 128 + (((kk % 8) ^ (row & 7)) << 4);
-                            *reinterpret_cast<uint4 *>(sA + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                            *reinterpret_cast<uint4 *>(sA + L::XSTAGE + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                            *reinterpret_cast<uint4 *>(sAg + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                            *reinterpret_cast<uint4 *>(sAg + L::XSTAGE + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                         }
                     }
                 }
                 tqdev::tc_fence_before();
                 tqdev::mbar_arrive(&bar_ufree[g]);                    // U read for the last time
                 tqdev::fence_proxy_async_smem();
-                tqdev::mbar_arrive(&bar_afull);                       // residual operand written
+                tqdev::mbar_arrive(&bar_afull[g]);                    // residual operand written
                 const float e2 = e2p.x + e2p.y;
                 bool zero_row = degenerate;
                 const int tail = B * NC + M / 32;
