@@ -106,23 +106,27 @@ def arm_config(workload):
 
 
 # DRAM traffic of a piece: dram__bytes_read.sum + dram__bytes_write.sum summed
-# over the piece's launches of one step (one ncu capture, caches flushed before
-# the piece, the median step of those captured), keyed by (piece, workload),
+# over the piece's launches of one step (one ncu capture of every launch, caches
+# flushed before each kernel, averaged over the captured steps), keyed by (piece, workload),
 # with the SHA-1 of the source files holding those kernels when the counters
 # were taken: once one of them changes the entry no longer applies (traffic:
 # null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 329518080),
-    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 320385280),
-    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 148876800),
-    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 297863936),
-    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 292844288),
-    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 80967168),
-    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 628645376),
-    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 616377600),
-    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 43086080),
-    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "bcbcc0bb71110488468ab838f5a53bbf58fe3061", 42775552),
-    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b76068c23bb09a3026c1745cb18d7f737bd9f505", 24092416),
+    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 330416320),
+    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 320637184),
+    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 148961152),
+    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 298767808),
+    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 292875968),
+    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 80961920),
+    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 629057664),
+    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 616405760),
+    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 43085184),
+    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 42539072),
+    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 27370752),
+    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 149602368),
+    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 446450560),
+    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 437225984),
+    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b4267ffe37d4375c1f3ad2780e25487d8149eccf", 152443712),
 }
 
 
