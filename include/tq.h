@@ -247,10 +247,17 @@ int tq_decode_launch_count(const tq_segment *segs, int n_segs, int batch, int n_
  * and shares each tile across the query heads of its kv-head group (GQA)
  * and across all sequences of a shared segment; a second kernel merges the
  * partials by log-sum-exp (left out when every sequence has one unsplit
- * segment: the decode kernel then writes the output).  The decode and merge
- * kernels are programmatic dependent launches: they may begin while the
- * kernel before them in the stream ends, and wait for it before reading its
- * output.
+ * segment: the decode kernel then writes the output).  A segment read by 16
+ * or more queries per kv head (sequences x query heads of a group), with d
+ * and m in {64, 128} and the Walsh-Hadamard rotation, is decoded on the
+ * tensor cores instead: the queries are the rows of the score and value
+ * MMAs, with q_rot, S q_rot, the centroids and the softmax weights split
+ * into bfloat16 hi + lo parts (about 2^-16 relative error per product).
+ * The environment variable TQ_DECODE_PATH, read at each call, overrides the
+ * choice: "lut" keeps every segment on the lookup tables, "mma" sends every
+ * segment that fits to the tensor cores.  The decode and merge kernels are
+ * programmatic dependent launches: they may begin while the kernel before
+ * them in the stream ends, and wait for it before reading its output.
  *  segs      : HOST array of n_segs (<= TQ_MAX_SEGMENTS) segments; every
  *              sequence in [0, batch) must be covered by at least one.
  *  q         : device [batch][n_q_heads][d] in q_dtype.

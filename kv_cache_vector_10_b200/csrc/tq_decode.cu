@@ -157,7 +157,12 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     const int chunk_bytes = TQ_DEC_CHUNK * (krow + vrow);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int half = lane >> 4, slot = lane & 15;
+    const int half = lane >> 4, slot = lane & 15;             // value pass: 16 lanes per token
+    // score pass: lanes per token; 8 for 4 queries per CTA (16-byte table
+    // entries: a quarter-warp of one token reads 8 distinct bank groups)
+    constexpr int LPT = QC == 4 ? 8 : 16;
+    constexpr int TPS = 32 / LPT;                              // tokens per score step
+    const int sl = lane % LPT, tg = lane / LPT;
 
     for (int i = tid; i < vpair_entries<BV>() * VCOP; i += blockDim.x) {
         const int e = i / VCOP;
@@ -280,53 +285,81 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
         const uint8_t *sV = sK + TQ_DEC_CHUNK * krow;
         const int64_t t0 = t_begin + ci * TQ_DEC_CHUNK;
 
-        // scores: step st covers tokens 2*st (lanes 0-15) and 2*st+1 (16-31),
-        // one byte group (8 coordinates / 8 projections) per lane
-        float part[QC][16];
+        // scores: LPT lanes per token (16, or 8 for 4 queries per CTA),
+        // TPS tokens per step; lane (tg, sl) scores token TPS * st + tg, byte
+        // groups sl + LPT * i of each 16-group round
+        float part[QC][LPT];
 #pragma unroll
-        for (int st = 0; st < 16; ++st) {
-            const uint8_t *kr = sK + (2 * st + half) * krow;
-            float am[QC], as[QC];
+        for (int st = 0; st < LPT; ++st) {
+            const uint8_t *kr = sK + (TPS * st + tg) * krow;
+            // query pairs accumulate in packed fp32x2 (one pair when QC == 1)
+            float2 am[(QC + 1) / 2], as[(QC + 1) / 2];
 #pragma unroll
-            for (int qq = 0; qq < QC; ++qq) am[qq] = as[qq] = 0.f;
+            for (int qp = 0; qp < (QC + 1) / 2; ++qp) am[qp] = as[qp] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < RK; ++r) {
-                const int gg = r * 16 + slot;
-                if (gg < NGK) {
-                    uint32_t pb[BK];
 #pragma unroll
-                    for (int pl = 0; pl < BK; ++pl) pb[pl] = kr[pl * (D / 8) + gg];
+                for (int gi = 0; gi < 16 / LPT; ++gi) {
+                    const int gs = sl + LPT * gi, gg = r * 16 + gs;
+                    if (gg < NGK) {
+                        uint32_t pb[BK];
 #pragma unroll
-                    for (int sp = 0; sp < NP; ++sp) {
-                        uint32_t x = 0;
+                        for (int pl = 0; pl < BK; ++pl) pb[pl] = kr[pl * (D / 8) + gg];
 #pragma unroll
-                        for (int pl = 0; pl < BK; ++pl)
-                            if ((sigma_set(BK, sp) >> pl) & 1) x ^= pb[pl];
-                        const VT e = lutq[lut_slot<QC>(r, (int)x, half, slot)];
+                        for (int sp = 0; sp < NP; ++sp) {
+                            uint32_t x = 0;
 #pragma unroll
-                        for (int qq = 0; qq < QC; ++qq) am[qq] = fmaf(alpha[sp], Vec<QC>::get(e, qq), am[qq]);
+                            for (int pl = 0; pl < BK; ++pl)
+                                if ((sigma_set(BK, sp) >> pl) & 1) x ^= pb[pl];
+                            const VT e = lutq[lut_slot<QC>(r, (int)x, tg, gs)];
+                            if constexpr (QC == 1) {
+                                am[0].x = fmaf(alpha[sp], Vec<QC>::get(e, 0), am[0].x);
+                            } else {
+#pragma unroll
+                                for (int qp = 0; qp < QC / 2; ++qp)
+                                    am[qp] = __ffma2_rn(make_float2(alpha[sp], alpha[sp]),
+                                                        make_float2(Vec<QC>::get(e, 2 * qp), Vec<QC>::get(e, 2 * qp + 1)), am[qp]);
+                            }
+                        }
                     }
                 }
             }
-            for (int r = 0; r < RS; ++r) {
-                const int gg = r * 16 + slot;
-                if (gg < NGS) {
-                    const VT e = luts[lut_slot<QC>(r, kr[off_sign + gg], half, slot)];
 #pragma unroll
-                    for (int qq = 0; qq < QC; ++qq) as[qq] += Vec<QC>::get(e, qq);
+            for (int r = 0; r < RS; ++r) {
+#pragma unroll
+                for (int gi = 0; gi < 16 / LPT; ++gi) {
+                    const int gs = sl + LPT * gi, gg = r * 16 + gs;
+                    if (gg < NGS) {
+                        const VT e = luts[lut_slot<QC>(r, kr[off_sign + gg], tg, gs)];
+                        if constexpr (QC == 1) {
+                            as[0].x += Vec<QC>::get(e, 0);
+                        } else {
+#pragma unroll
+                            for (int qp = 0; qp < QC / 2; ++qp)
+                                as[qp] = __fadd2_rn(make_float2(Vec<QC>::get(e, 2 * qp), Vec<QC>::get(e, 2 * qp + 1)), as[qp]);
+                        }
+                    }
                 }
             }
             const float2 nrm = tqdev::key_norms(reinterpret_cast<const uint32_t *>(kr + off_ns), kf16);
             const float a1 = nrm.x * inv_d, a2 = nrm.y * cqs;
+            if constexpr (QC == 1) {
+                part[0][st] = fmaf(a1, am[0].x, a2 * as[0].x);
+            } else {
 #pragma unroll
-            for (int qq = 0; qq < QC; ++qq) part[qq][st] = fmaf(a1, am[qq], a2 * as[qq]);
+                for (int qp = 0; qp < QC / 2; ++qp) {
+                    const float2 v = __ffma2_rn(make_float2(a1, a1), am[qp], __fmul2_rn(make_float2(a2, a2), as[qp]));
+                    part[2 * qp][st] = v.x;
+                    part[2 * qp + 1][st] = v.y;
+                }
+            }
         }
-        // transposing butterfly over the 16 lanes of each half-warp
+        // transposing butterfly over the LPT lanes of each token group
 #pragma unroll
         for (int qq = 0; qq < QC; ++qq) {
 #pragma unroll
-            for (int w = 8; w >= 1; w >>= 1) {
-                const bool up = (slot & w) != 0;
+            for (int w = LPT / 2; w >= 1; w >>= 1) {
+                const bool up = (sl & w) != 0;
 #pragma unroll
                 for (int i = 0; i < w; ++i) {
                     const float send = up ? part[qq][i] : part[qq][i + w];
@@ -335,8 +368,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
                 }
             }
         }
-        // this lane now holds the score of token 2*slot + half
-        const int tok = 2 * slot + half;
+        // this lane now holds the score of token TPS * sl + tg
+        const int tok = TPS * sl + tg;
         const bool valid = t0 + tok < t_end;
         const float nsv = *reinterpret_cast<const float *>(sV + tok * vrow + voff_ns);
         float w_tok[QC];
@@ -364,7 +397,8 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             float2 wq[QC];
 #pragma unroll
             for (int qq = 0; qq < QC; ++qq) {
-                const float wv = __shfl_sync(0xffffffffu, w_tok[qq], half * 16 + st);
+                const int tv = 2 * st + half;   // held by lane (tv % TPS) * LPT + tv / TPS
+                const float wv = __shfl_sync(0xffffffffu, w_tok[qq], (tv % TPS) * LPT + tv / TPS);
                 wq[qq] = make_float2(wv, wv);
             }
             if (vslot) {

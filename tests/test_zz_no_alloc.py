@@ -43,6 +43,31 @@ def test_static_scratch_decode_matches_workspace_decode():
         assert torch.equal(out, ref), (call, float((out - ref).abs().max()))
 
 
+def test_static_scratch_shared_prefix_on_tensor_cores():
+    """A prefix shared by 8 sequences (32 queries per kv head: the tensor-core
+    decode) plus private tails (the byte tables): the same identity."""
+    g = torch.Generator(device="cuda").manual_seed(5)
+    A, Hq, Hkv, d = 8, 8, 2, 128
+    pc, tc = tq.Codec(d, 2, 128, 42), tq.Codec(d, 4, 128, 42)
+    tq.tq_ensure_heads(pc.ctx, Hkv)
+    tq.tq_ensure_heads(tc.ctx, Hkv)
+    pk = torch.randn(1, Hkv, 500, d, generator=g, device="cuda").to(torch.bfloat16)
+    pv = torch.randn(1, Hkv, 500, d, generator=g, device="cuda").to(torch.bfloat16)
+    tk = torch.randn(A, Hkv, 60, d, generator=g, device="cuda").to(torch.bfloat16)
+    tv = torch.randn(A, Hkv, 60, d, generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn(A, Hq, d, generator=g, device="cuda").to(torch.bfloat16)
+    pcache, tcache = pc.alloc(1, Hkv, 512), tc.alloc(A, Hkv, 64)
+    pc.encode_kv(pk, pv, pcache)
+    tc.encode_kv(tk, tv, tcache)
+    segs = [tq.Segment(pcache, 500, 0, A)] + [tq.Segment(tcache, 60, a, 1, codes_batch=a) for a in range(A)]
+    ref = tq.decode_attention(segs, q, Hkv, out_dtype=torch.float32)
+    out = torch.full_like(ref, float("nan"))
+    tq.tq_decode_attention_static(segs, q, A, Hq, Hkv, out)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    assert torch.equal(out, ref), float((out - ref).abs().max())
+
+
 def test_static_scratch_rejects_oversized_calls():
     codec = tq.Codec(128, 2, 128, 1)
     cache = codec.alloc(1, 1, 16)
