@@ -667,18 +667,19 @@ __global__ void __launch_bounds__(D) tq_combine_kernel(const __grid_constant__ D
     tqdev::grid_dep_wait();   // the partials of the decode launches
     const int b = blockIdx.x / P.Hq, j = blockIdx.x % P.Hq;
     const int PF = tq_part_floats(D);
-    // one pass with an online rescale; the (m, l, o_j) of 4 splits are loaded
-    // before any is used, so their latencies overlap
+    // one pass with an online rescale; the (m, l, o_j) of CB splits are
+    // loaded before any is used, so their latencies overlap
+    constexpr int CB = 8;
     float mx = -INFINITY, l = 0.f, o = 0.f;
     for (int s = 0; s < P.n_segs; ++s) {
         const SegDesc &g = P.seg[s];
         if (b < g.first_seq || b >= g.first_seq + g.n_seqs || g.T == 0) continue;
         const float *base = P.part + (g.part_base + (int64_t)(b - g.first_seq) * P.Hq + j) * PF;
         const int64_t stride = (int64_t)g.n_seqs * P.Hq * PF;   // between splits
-        for (int sp0 = 0; sp0 < g.n_splits; sp0 += 4) {
-            float pm[4], pl[4], po[4];
+        for (int sp0 = 0; sp0 < g.n_splits; sp0 += CB) {
+            float pm[CB], pl[CB], po[CB];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < CB; ++k) {
                 const bool in = sp0 + k < g.n_splits;
                 const float *pp = base + (int64_t)(sp0 + k) * stride;
                 pm[k] = in ? pp[0] : -INFINITY;
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(D) tq_combine_kernel(const __grid_constant__ D
                 po[k] = in ? pp[4 + threadIdx.x] : 0.f;
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < CB; ++k) {
                 if (pm[k] == -INFINITY) continue;
                 if (pm[k] > mx) {
                     const float sc = __expf(mx - pm[k]);   // 0 while mx is -inf
