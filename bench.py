@@ -112,21 +112,21 @@ def arm_config(workload):
 # were taken: once one of them changes the entry no longer applies (traffic:
 # null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 330416320),
-    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 320637184),
-    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 148961152),
-    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 298767808),
-    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 292875968),
-    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 80961920),
-    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 629057664),
-    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 616405760),
-    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 43085184),
-    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 42539072),
-    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 27370752),
-    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "0926edfab0563dbfcf287f822c9418bbfd4e3b72", 149602368),
-    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 446450560),
-    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "52c307616b7fe213d21e6c89575df3bdc0692475", 437225984),
-    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "b4267ffe37d4375c1f3ad2780e25487d8149eccf", 152443712),
+    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 330946368),
+    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 320536320),
+    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 148926592),
+    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 299143872),
+    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 292741056),
+    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 81003072),
+    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 629057664),
+    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 616405760),
+    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 43085184),
+    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 42535936),
+    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 27374080),
+    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 149909888),
+    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 444996032),
+    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 436411520),
+    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "58115251d06c1c6cbe58ef71971c963593d86b3b", 152415424),
 }
 
 

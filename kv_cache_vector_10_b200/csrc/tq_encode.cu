@@ -1206,7 +1206,9 @@ struct PipeLayout {
     static constexpr int THREADS = 32 * (4 * NG + 1);    // + the producer warp
     static constexpr int XBOX = ENC_ROWS * 128;          // one 64-column box of a tile (16 KB)
     static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
-    static constexpr int NS = KEYS ? 1 : 4;              // stages of the row ring
+    // stages of the row ring: keys at d = 128 have room for one next to the
+    // two groups' residual buffers
+    static constexpr int NS = KEYS ? (D == 128 ? 1 : 2) : 4;
     static constexpr int OFF_HD = NS * XSTAGE;           // rotation operand [d/64][d][128 B]
     static constexpr int OFF_A = OFF_HD + D * D * 2;     // keys: residual operand hi, lo of each group
     static constexpr int OFF_S = OFF_A + (KEYS ? NG * 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
