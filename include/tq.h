@@ -316,8 +316,7 @@ size_t tq_decode_append_workspace_bytes(const tq_segment *segs, int n_segs, int 
  *    if a segment's context has no tables yet for n_kv_heads heads (building
  *    them allocates; call tq_ensure_heads first).
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.  The address is kept for the life of the
+ *    (cudaGetSymbolAddress) with that device current.  The address is kept for the life of the
  *    process, per device number: only the device's primary context (the
  *    one the CUDA runtime uses) is supported, and the address is not looked
  *    up again after cudaDeviceReset.
