@@ -237,3 +237,40 @@ def test_append_wide_group(monkeypatch):
             for j in range(h * G, (h + 1) * G):
                 ref = oracle.attention(q[b, j].double().numpy(), [(oc, h, ek["rows"], ev["rows"])])
                 assert np.max(np.abs(out[b, j] - ref)) <= pu.ATTN_ABS
+
+
+def test_two_prefixes_different_bits(monkeypatch):
+    """Two prefixes shared by 12 sequences at bits 2 and 3 (two tensor-core
+    launches) plus private tails at bits 4 (the byte tables): every output
+    merges three segments."""
+    g = torch.Generator().manual_seed(33)
+    A, Hq, Hkv, d = 12, 8, 2, 128
+    specs = [dict(bits=2, k=_rand(g, (1, Hkv, 300, d)), v=_rand(g, (1, Hkv, 300, d)), first_seq=0, n_seqs=A),
+             dict(bits=3, k=_rand(g, (1, Hkv, 200, d)), v=_rand(g, (1, Hkv, 200, d)), first_seq=0, n_seqs=A, seed=9),
+             dict(bits=4, k=_rand(g, (A, Hkv, 40, d)), v=_rand(g, (A, Hkv, 40, d)), first_seq=0, n_seqs=1,
+                  stride=1, seed=5)]
+    q = _rand(g, (A, Hq, d))
+    gsegs, osegs, keep = _build(specs, d, 128)
+    _set_path(monkeypatch, None)
+    # query preparation, tails, two tensor-core launches, combine
+    assert tq.tq_decode_launch_count(gsegs, A, Hq, Hkv) == 5
+    out = _decode(gsegs, q, Hkv)
+    pairs = [(b, j) for b in (0, 5, 11) for j in range(Hq)]
+    assert _check(out, q, osegs, Hkv, torch.float32, pairs) <= 1.0
+
+
+def test_two_prefixes_same_bits_one_launch(monkeypatch):
+    """Two prefixes at bits 3 from codecs with different seeds, each shared
+    by a different half of the batch: one tensor-core launch covers both,
+    each CTA with its own segment's rotation signs, codebooks and S."""
+    g = torch.Generator().manual_seed(34)
+    B, Hq, Hkv, d = 16, 8, 2, 128
+    specs = [dict(bits=3, k=_rand(g, (1, Hkv, 250, d)), v=_rand(g, (1, Hkv, 250, d)), first_seq=0, n_seqs=8, seed=1),
+             dict(bits=3, k=_rand(g, (1, Hkv, 180, d)), v=_rand(g, (1, Hkv, 180, d)), first_seq=8, n_seqs=8, seed=2)]
+    q = _rand(g, (B, Hq, d))
+    gsegs, osegs, keep = _build(specs, d, 128)
+    _set_path(monkeypatch, None)
+    assert tq.tq_decode_launch_count(gsegs, B, Hq, Hkv) == 3   # query preparation, one decode, combine
+    out = _decode(gsegs, q, Hkv)
+    pairs = [(b, j) for b in (0, 7, 8, 15) for j in range(Hq)]
+    assert _check(out, q, osegs, Hkv, torch.float32, pairs) <= 1.0
