@@ -1201,8 +1201,8 @@ struct PipeParams {
 template <int D, bool KEYS, int B>
 struct PipeLayout {
     // compute groups of 4 warps: keys hold U and C/P (2 x 128 TMEM columns)
-    // per group; 4-bit values need more registers than four groups leave
-    static constexpr int NG = KEYS ? 2 : (B == 4 ? 3 : 4);
+    // per group; values hold U only (four groups fit 96 registers a thread)
+    static constexpr int NG = KEYS ? 2 : 4;
     static constexpr int THREADS = 32 * (4 * NG + 1);    // + the producer warp
     static constexpr int XBOX = ENC_ROWS * 128;          // one 64-column box of a tile (16 KB)
     static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
