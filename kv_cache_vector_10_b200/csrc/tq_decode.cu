@@ -153,7 +153,10 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
     VT *luts = lutq + lut_entries<QC>(RK);
     float2 *vlut = reinterpret_cast<float2 *>(luts + lut_entries<QC>(RS));
     uint64_t *bars = reinterpret_cast<uint64_t *>(vlut + vpair_entries<BV>() * VCOP);
-    uint8_t *stage = reinterpret_cast<uint8_t *>(bars + NBUF * TQ_DEC_WARPS);
+    // several queries per CTA: the value pass reads each token's softmax
+    // weights (all queries in one entry) from a per-warp array
+    VT *wbuf = reinterpret_cast<VT *>(bars + NBUF * TQ_DEC_WARPS);
+    uint8_t *stage = reinterpret_cast<uint8_t *>(wbuf + (QC > 1 ? TQ_DEC_WARPS * TQ_DEC_CHUNK : 0));
     const int chunk_bytes = TQ_DEC_CHUNK * (krow + vrow);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -389,17 +392,24 @@ __global__ void __launch_bounds__(TQ_DEC_WARPS * 32, 1) tq_decode_kernel(const _
             m_run[qq] = mn;
             w_tok[qq] = valid ? pr * nsv : 0.f;
         }
+        if constexpr (QC > 1) {
+            wbuf[warp * TQ_DEC_CHUNK + tok] = Vec<QC>::make(w_tok);
+            __syncwarp();
+        }
         // values: step st again covers tokens 2*st + half; lane slot g owns
         // coordinates 8g..8g+7 (four value pairs)
 #pragma unroll 4
         for (int st = 0; st < 16; ++st) {
             const uint32_t *vr = reinterpret_cast<const uint32_t *>(sV + (2 * st + half) * vrow);
             float2 wq[QC];
+            if constexpr (QC > 1) {
+                const VT w4 = wbuf[warp * TQ_DEC_CHUNK + 2 * st + half];
 #pragma unroll
-            for (int qq = 0; qq < QC; ++qq) {
+                for (int qq = 0; qq < QC; ++qq) wq[qq] = make_float2(Vec<QC>::get(w4, qq), Vec<QC>::get(w4, qq));
+            } else {
                 const int tv = 2 * st + half;   // held by lane (tv % TPS) * LPT + tv / TPS
-                const float wv = __shfl_sync(0xffffffffu, w_tok[qq], (tv % TPS) * LPT + tv / TPS);
-                wq[qq] = make_float2(wv, wv);
+                const float wv = __shfl_sync(0xffffffffu, w_tok[0], (tv % TPS) * LPT + tv / TPS);
+                wq[0] = make_float2(wv, wv);
             }
             if (vslot) {
 #pragma unroll
@@ -580,7 +590,8 @@ size_t decode_smem_bytes(int d, int bv, int qc, int krow, int vrow, int M, int n
     const size_t vpair = (size_t)(1 << (2 * bv)) * (bv <= 4 ? 16 : 1) * 8;
     const size_t stage = (size_t)TQ_DEC_WARPS * nbuf * TQ_DEC_CHUNK * (krow + vrow);
     const size_t merge = ((size_t)TQ_DEC_WARPS * qc * (d + 2) + qc * d + 2 * qc) * 4;
-    return lut + vpair + (size_t)nbuf * TQ_DEC_WARPS * 8 + std::max(stage, merge);
+    const size_t wbuf = qc > 1 ? (size_t)TQ_DEC_WARPS * TQ_DEC_CHUNK * vt : 0;
+    return lut + vpair + (size_t)nbuf * TQ_DEC_WARPS * 8 + wbuf + std::max(stage, merge);
 }
 
 constexpr size_t kMaxDynSmem = 232448;   // 227 KB per block on sm_100
