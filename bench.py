@@ -112,21 +112,21 @@ def arm_config(workload):
 # were taken: once one of them changes the entry no longer applies (traffic:
 # null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 330946368),
-    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 320536320),
-    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 148926592),
-    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 299143872),
-    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 292741056),
-    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 81003072),
-    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 629057664),
-    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 616405760),
-    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 43085184),
-    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 42535936),
-    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 27374080),
-    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a2626bde09cb68c79b28f33f90695f8682c65722", 149909888),
-    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 444996032),
-    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "378e4478214d0f87b3f61c5dd084724c818bca96", 436411520),
-    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "58115251d06c1c6cbe58ef71971c963593d86b3b", 152415424),
+    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 330933632),
+    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 320983040),
+    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 148838144),
+    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 298906240),
+    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 292800960),
+    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 81011520),
+    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 629141504),
+    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 616230848),
+    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 43086272),
+    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 42973376),
+    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 27370880),
+    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 149732032),
+    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 445050560),
+    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 436104832),
+    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "58115251d06c1c6cbe58ef71971c963593d86b3b", 152447936),
 }
 
 
