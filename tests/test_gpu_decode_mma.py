@@ -274,3 +274,17 @@ def test_two_prefixes_same_bits_one_launch(monkeypatch):
     out = _decode(gsegs, q, Hkv)
     pairs = [(b, j) for b in (0, 7, 8, 15) for j in range(Hq)]
     assert _check(out, q, osegs, Hkv, torch.float32, pairs) <= 1.0
+
+
+@pytest.mark.parametrize("d,m", [(256, 128), (128, 192)])
+def test_many_queries_outside_the_tensor_core_shapes(monkeypatch, d, m):
+    """head_dim 256 or 192 projections with 20 queries per kv head: the
+    planner keeps these segments on the byte tables, same results."""
+    g = torch.Generator().manual_seed(d + m)
+    A, Hq, Hkv = 5, 8, 2
+    specs = [dict(bits=3, k=_rand(g, (1, Hkv, 150, d)), v=_rand(g, (1, Hkv, 150, d)), first_seq=0, n_seqs=A)]
+    q = _rand(g, (A, Hq, d))
+    gsegs, osegs, keep = _build(specs, d, m)
+    _set_path(monkeypatch, None)
+    out = _decode(gsegs, q, Hkv)
+    assert _check(out, q, osegs, Hkv, torch.float32) <= 1.0
