@@ -1,7 +1,8 @@
 """Decode steps captured in a CUDA graph and replayed: the split-K decode
 (including its dependent launches and, for several segments, the combine
-step) and the allocation-free entry point replay to the same bytes as eager
-calls on the same inputs, also after the query is updated in place."""
+step; the shared prefix goes to the tensor-core decode) and the append step
+replay to the same bytes as eager calls on the same inputs, also after the
+query is updated in place."""
 import pytest
 import torch
 
@@ -56,28 +57,6 @@ def test_decode_graph_replay_matches_eager(shared):
     tq.tq_decode_attention(segs, q_static, B, Hq, H, out_static, ws)
     torch.cuda.synchronize()
     assert torch.equal(got, out_static) and not torch.equal(got, ref1)
-
-
-def test_static_decode_graph_replay_matches_eager():
-    B, H, Hq, T = 8, 32, 32, 2048
-    codec, cache = _cache(B, H, T, 4, 9, torch.float16)
-    segs = [tq.Segment(cache, T, b, 1, codes_batch=b) for b in range(B)]
-    q = torch.randn(B, Hq, 128, device=DEV).to(torch.float16)
-    out = torch.empty(B, Hq, 128, dtype=torch.float16, device=DEV)
-    tq.tq_decode_attention_static(segs, q, B, Hq, H, out)   # first call: before capture
-    torch.cuda.synchronize()
-    ref = out.clone()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(graph, stream=s):
-            tq.tq_decode_attention_static(segs, q, B, Hq, H, out)
-    torch.cuda.current_stream().wait_stream(s)
-    out.zero_()
-    graph.replay()
-    torch.cuda.synchronize()
-    assert torch.equal(out, ref)
 
 
 def test_append_graph_replay_appends_like_eager():
