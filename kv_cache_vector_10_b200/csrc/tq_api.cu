@@ -195,6 +195,7 @@ void tq_destroy(tq_ctx *ctx) {
     cudaFree(ctx->d_book);
     cudaFree(ctx->d_Q32);
     cudaFree(ctx->d_Qh);
+    cudaFree(ctx->d_Qbf);
     cudaFree(ctx->d_HD16);
     cudaFree(ctx->d_HDbf);
     delete ctx;
@@ -256,8 +257,10 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
     }
     float *nQ32 = nullptr;
     __half *nQh = nullptr;
-    CUtensorMap qmap;
+    uint16_t *nQbf = nullptr;
+    CUtensorMap qmap, qbfmap;
     std::memset(&qmap, 0, sizeof(qmap));
+    std::memset(&qbfmap, 0, sizeof(qbfmap));
     if (st == TQ_OK && ctx->rotation == TQ_ROT_HAAR) {
         const size_t dd = (size_t)d * d;
         std::vector<double> Q(dd);
@@ -278,6 +281,38 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
         if (st == TQ_OK) st = tq_check_cuda(cudaMalloc(&nQh, qh.size() * 2));
         if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nQ32, q32.data(), q32.size() * 4, cudaMemcpyHostToDevice));
         if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nQh, qh.data(), qh.size() * 2, cudaMemcpyHostToDevice));
+        // bfloat16 hi + mid + lo of sqrt(d) Q for the TMA-fed value encoder
+        // (bfloat16 rows need a bfloat16 operand; three pieces keep 24 bits)
+        if (st == TQ_OK && d <= 128) {
+            auto bf16_bits = [](double v) -> uint16_t {
+                const float f = (float)v;
+                uint32_t u;
+                std::memcpy(&u, &f, 4);
+                u += 0x7FFFu + ((u >> 16) & 1u);   // round to nearest even
+                return (uint16_t)(u >> 16);
+            };
+            auto bf16_val = [](uint16_t b) -> double {
+                const uint32_t u = (uint32_t)b << 16;
+                float f;
+                std::memcpy(&f, &u, 4);
+                return (double)f;
+            };
+            std::vector<uint16_t> qb((size_t)n_heads * 3 * dd);
+            for (int h = 0; h < n_heads; ++h) {
+                tq_host_haar(d, m, ctx->seed, h, Q.data());
+                for (size_t i = 0; i < dd; ++i) {
+                    double r = sd * Q[i];
+                    for (int piece = 0; piece < 3; ++piece) {
+                        const uint16_t b = bf16_bits(r);
+                        qb[((size_t)h * 3 + piece) * dd + i] = b;
+                        r -= bf16_val(b);
+                    }
+                }
+            }
+            st = tq_check_cuda(cudaMalloc(&nQbf, qb.size() * 2));
+            if (st == TQ_OK) st = tq_check_cuda(cudaMemcpy(nQbf, qb.data(), qb.size() * 2, cudaMemcpyHostToDevice));
+            if (st == TQ_OK) st = encode_rows_map(&qbfmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, nQbf, d, (int64_t)n_heads * 3 * d, d);
+        }
         if (st == TQ_OK) {
             PFN_encodeTiled enc = get_encode_tiled();
             cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n_heads * 2 * d};
@@ -322,6 +357,7 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
         cudaFree(nS);
         cudaFree(nQ32);
         cudaFree(nQh);
+        cudaFree(nQbf);
         cudaFree(nHD16);
         cudaFree(nHDbf);
         return st;
@@ -331,6 +367,7 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
     cudaFree(ctx->d_S);
     cudaFree(ctx->d_Q32);
     cudaFree(ctx->d_Qh);
+    cudaFree(ctx->d_Qbf);
     cudaFree(ctx->d_HD16);
     cudaFree(ctx->d_HDbf);
     ctx->d_signs = nsig;
@@ -339,6 +376,8 @@ tq_status tq_ensure_heads(tq_ctx *ctx, int n_heads) {
     ctx->d_Q32 = nQ32;
     ctx->d_Qh = nQh;
     ctx->tmap_Q = qmap;
+    ctx->d_Qbf = nQbf;
+    ctx->tmap_Qbf = qbfmap;
     ctx->d_HD16 = nHD16;
     ctx->d_HDbf = nHDbf;
     ctx->tmap_HD16 = hdmap16;

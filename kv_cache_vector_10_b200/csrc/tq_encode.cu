@@ -1198,7 +1198,9 @@ struct PipeParams {
     int norm_f16;
 };
 
-template <int D, bool KEYS, int B>
+// NP: pieces of the rotation operand (1: the exact +-1 Walsh-Hadamard matrix;
+// Haar values: sqrt(d) Q as binary16 hi + lo (2) or bfloat16 hi + mid + lo (3)).
+template <int D, bool KEYS, int B, int NP = 1>
 struct PipeLayout {
     // compute groups of 4 warps: keys hold U and C/P (2 x 128 TMEM columns)
     // per group; values hold U only (four groups fit 96 registers a thread)
@@ -1208,10 +1210,13 @@ struct PipeLayout {
     static constexpr int XSTAGE = (D / 64) * XBOX;       // one tile of 16-bit rows
     // stages of the row ring: keys at d = 128 have room for one next to the
     // two groups' residual buffers
-    static constexpr int NS = KEYS ? (D == 128 ? 1 : 2) : 4;
-    static constexpr int OFF_HD = NS * XSTAGE;           // rotation operand [d/64][d][128 B]
-    static constexpr int OFF_A = OFF_HD + D * D * 2;     // keys: residual operand hi, lo of each group
-    static constexpr int OFF_S = OFF_A + (KEYS ? NG * 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
+    static constexpr int NS = KEYS ? (D == 128 ? 1 : 2) : (NP == 3 ? 3 : 4);
+    static constexpr int OFF_HD = NS * XSTAGE;           // rotation operand [NP][d/64][d][128 B]
+    static constexpr int OFF_A = OFF_HD + NP * D * D * 2;   // keys: residual operand hi, lo
+    // keys: residual operand buffers, one per group with the Walsh-Hadamard
+    // operand, one shared (taken in tile order) with the larger Haar operand
+    static constexpr int NA = NP == 1 ? NG : 1;
+    static constexpr int OFF_S = OFF_A + (KEYS ? NA * 2 * XSTAGE : 0);   // keys: S [d/64][m][128 B]
     static constexpr int FIXED = 1024 + OFF_S;           // dynamic bytes before S (with alignment slack)
 };
 
@@ -1234,11 +1239,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase) {
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int B, typename Tin, bool KEYS>
-__global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
+template <int D, int B, typename Tin, bool KEYS, int NP = 1>
+__global__ void __launch_bounds__(PipeLayout<D, KEYS, B, NP>::THREADS, 1)
     tq_encode_pipe_kernel(const __grid_constant__ PipeParams p, const __grid_constant__ CUtensorMap tmapX,
                           const __grid_constant__ CUtensorMap tmapHD, const __grid_constant__ CUtensorMap tmapS) {
-    using L = PipeLayout<D, KEYS, B>;
+    using L = PipeLayout<D, KEYS, B, NP>;
     constexpr int NS = L::NS;
     constexpr int NG = L::NG;
     constexpr int HB = (1 << B) / 2;             // magnitude cells of the positive half
@@ -1338,10 +1343,13 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                     if (h != hd_head && !hd_busy) {
                         // the previous rotation (old operand) must be complete
                         if (li == 0 || mbar_test(&bar_xfree[(li - 1) % NS], (uint32_t)(((li - 1) / NS) & 1))) {
-                            tqdev::mbar_expect_tx(&bar_hd, (uint32_t)(D * D * 2));
+                            tqdev::mbar_expect_tx(&bar_hd, (uint32_t)(NP * D * D * 2));
 #pragma unroll
-                            for (int a = 0; a < D / 64; ++a)
-                                tqdev::tma_load_2d(sHD + a * D * 128, &tmapHD, a * 64, h * D, &bar_hd);
+                            for (int piece = 0; piece < NP; ++piece)
+#pragma unroll
+                                for (int a = 0; a < D / 64; ++a)
+                                    tqdev::tma_load_2d(sHD + (piece * (D / 64) + a) * D * 128, &tmapHD, a * 64,
+                                                       (h * NP + piece) * D, &bar_hd);
                             hd_busy = true;
                             hd_head = h;
                             progress = true;
@@ -1358,12 +1366,14 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                         const uint32_t abase = tqdev::smem_u32(sX + (li % NS) * L::XSTAGE);
                         const uint32_t bbase = tqdev::smem_u32(sHD);
 #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t a_addr = abase + (ks / 4) * L::XBOX + (ks % 4) * 32;
-                            const uint32_t b_addr = bbase + (ks / 4) * (D * 128) + (ks % 4) * 32;
-                            tqdev::mma_f16_ss(tmem + (uint32_t)g * GSTRIDE, tqdev::smem_desc_sw128(a_addr),
-                                              tqdev::smem_desc_sw128(b_addr), idesc_rot, ks != 0);
-                        }
+                        for (int piece = 0; piece < NP; ++piece)
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint32_t a_addr = abase + (ks / 4) * L::XBOX + (ks % 4) * 32;
+                                const uint32_t b_addr = bbase + piece * (D / 64) * D * 128 + (ks / 4) * (D * 128) + (ks % 4) * 32;
+                                tqdev::mma_f16_ss(tmem + (uint32_t)g * GSTRIDE, tqdev::smem_desc_sw128(a_addr),
+                                                  tqdev::smem_desc_sw128(b_addr), idesc_rot, (piece | ks) != 0);
+                            }
                         tqdev::mma_commit(&bar_rot[g]);
                         tqdev::mma_commit(&bar_xfree[li % NS]);
                         ++next_rot;
@@ -1375,7 +1385,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                     const int j = next_qjl, h = head_of(j);
                     if (h != s_head && !s_busy) {
                         // the previous projection (old S) must be complete
-                        if (j == 0 || mbar_test(&bar_afree[(j - 1) % NG], (uint32_t)(((j - 1) / NG) & 1))) {
+                        if (j == 0 || mbar_test(&bar_afree[(j - 1) % L::NA], (uint32_t)(((j - 1) / L::NA) & 1))) {
                             tqdev::mbar_expect_tx(&bar_s, p.s_bytes);
 #pragma unroll
                             for (int a = 0; a < D / 64; ++a)
@@ -1390,12 +1400,12 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                         s_busy = false;
                         progress = true;
                     }
-                    if (h == s_head && !s_busy && mbar_test(&bar_afull[j % NG], (uint32_t)((j / NG) & 1))) {
+                    if (h == s_head && !s_busy && mbar_test(&bar_afull[j % L::NA], (uint32_t)((j / L::NA) & 1))) {
                         tqdev::tc_fence_after();
                         const uint32_t col = (uint32_t)(j % NG) * GSTRIDE + (uint32_t)D;
 #pragma unroll
                         for (int pass = 0; pass < 2; ++pass) {
-                            const uint32_t abase = tqdev::smem_u32(sA + ((j % NG) * 2 + pass) * L::XSTAGE);
+                            const uint32_t abase = tqdev::smem_u32(sA + ((j % L::NA) * 2 + pass) * L::XSTAGE);
                             const uint32_t bbase = tqdev::smem_u32(sS);
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
@@ -1406,7 +1416,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                             }
                         }
                         tqdev::mma_commit(&bar_qjl[j % NG]);
-                        tqdev::mma_commit(&bar_afree[j % NG]);
+                        tqdev::mma_commit(&bar_afree[j % L::NA]);
                         ++next_qjl;
                         progress = true;
                     }
@@ -1439,8 +1449,8 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                 tqdev::mbar_wait_bounded(&bar_xfull[li % NS], (uint32_t)((li / NS) & 1));
             for (int li = xfree_seen; li < next_rot; ++li)             // rotations not seen through xfree
                 tqdev::mbar_wait_bounded(&bar_xfree[li % NS], (uint32_t)((li / NS) & 1));
-            for (int j = next_qjl - NG < 0 ? 0 : next_qjl - NG; j < next_qjl; ++j)
-                tqdev::mbar_wait_bounded(&bar_afree[j % NG], (uint32_t)((j / NG) & 1));
+            for (int j = next_qjl - L::NA < 0 ? 0 : next_qjl - L::NA; j < next_qjl; ++j)
+                tqdev::mbar_wait_bounded(&bar_afree[j % L::NA], (uint32_t)((j / L::NA) & 1));
             if (hd_busy) tqdev::mbar_wait_bounded(&bar_hd, hd_ph);
             if (s_busy) tqdev::mbar_wait_bounded(&bar_s, s_ph);
         }
@@ -1450,7 +1460,6 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
         const int row = ((warp & 3) << 5) | lane;               // tile row = TMEM lane
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)g * GSTRIDE;
         const uint32_t tU = tl, tC = tl + (uint32_t)D;          // keys: C, then P, at tC
-        uint8_t *sAg = sA + g * 2 * L::XSTAGE;                  // keys: this group's residual operand
         bool failed = false;
         // keys: the sign plane of the group's previous tile is stored after this
         // tile's |u|^2 pass, so its QJL projection overlaps that pass
@@ -1664,8 +1673,10 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                 float e2a = n2 - 2.f * ns * uc + ns * ns * c2;
                 e2a = fmaxf(e2a, 1e-10f * n2);
                 const float sc = degenerate ? 0.f : sqrtf((float)D / e2a);
-                // ---- residual operand (the group's buffer, free once its previous projection is done)
-                if (k > 0 && !warp_wait(&bar_afree[g], (uint32_t)((k - 1) & 1))) {
+                // ---- residual operand: buffer li % NA, free once the projection
+                // of the tile that used it before is done
+                uint8_t *sAg = sA + (li % L::NA) * 2 * L::XSTAGE;
+                if (li >= L::NA && !warp_wait(&bar_afree[li % L::NA], (uint32_t)(((li / L::NA) - 1) & 1))) {
                     failed = true;
                     break;
                 }
@@ -1703,7 +1714,7 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
                 tqdev::tc_fence_before();
                 tqdev::mbar_arrive(&bar_ufree[g]);                    // U read for the last time
                 tqdev::fence_proxy_async_smem();
-                tqdev::mbar_arrive(&bar_afull[g]);                    // residual operand written
+                tqdev::mbar_arrive(&bar_afull[li % L::NA]);           // residual operand written
                 const float e2 = e2p.x + e2p.y;
                 bool zero_row = degenerate;
                 const int tail = B * NC + M / 32;
@@ -1747,10 +1758,10 @@ __global__ void __launch_bounds__(PipeLayout<D, KEYS, B>::THREADS, 1)
     }
 }
 
-template <int D, typename Tin, bool KEYS>
+template <int D, typename Tin, bool KEYS, int NP = 1>
 cudaError_t launch_pipe(int B, const PipeParams &p, const CUtensorMap &mx, const CUtensorMap &mhd,
                         const CUtensorMap &ms, int grid, cudaStream_t s) {
-    using L = PipeLayout<D, KEYS, 2>;   // the byte layout does not depend on B
+    using L = PipeLayout<D, KEYS, 2, NP>;   // the byte layout does not depend on B
     cudaError_t e = cudaSuccess;
     auto go = [&](auto kern, int threads) {
         size_t smem = (size_t)L::FIXED + (KEYS ? p.s_bytes : 0);
@@ -1766,11 +1777,11 @@ cudaError_t launch_pipe(int B, const PipeParams &p, const CUtensorMap &mx, const
         e = cudaGetLastError();
     };
     switch (B) {
-        case 1: if constexpr (KEYS) go(tq_encode_pipe_kernel<D, 1, Tin, KEYS>, PipeLayout<D, KEYS, 1>::THREADS); else return cudaErrorInvalidValue; break;
-        case 2: go(tq_encode_pipe_kernel<D, 2, Tin, KEYS>, PipeLayout<D, KEYS, 2>::THREADS); break;
-        case 3: go(tq_encode_pipe_kernel<D, 3, Tin, KEYS>, PipeLayout<D, KEYS, 3>::THREADS); break;
-        case 4: go(tq_encode_pipe_kernel<D, 4, Tin, KEYS>, PipeLayout<D, KEYS, 4>::THREADS); break;
-        case 5: if constexpr (!KEYS) go(tq_encode_pipe_kernel<D, 5, Tin, KEYS>, PipeLayout<D, KEYS, 5>::THREADS); else return cudaErrorInvalidValue; break;
+        case 1: if constexpr (KEYS) go(tq_encode_pipe_kernel<D, 1, Tin, KEYS, NP>, PipeLayout<D, KEYS, 1, NP>::THREADS); else return cudaErrorInvalidValue; break;
+        case 2: go(tq_encode_pipe_kernel<D, 2, Tin, KEYS, NP>, PipeLayout<D, KEYS, 2, NP>::THREADS); break;
+        case 3: go(tq_encode_pipe_kernel<D, 3, Tin, KEYS, NP>, PipeLayout<D, KEYS, 3, NP>::THREADS); break;
+        case 4: go(tq_encode_pipe_kernel<D, 4, Tin, KEYS, NP>, PipeLayout<D, KEYS, 4, NP>::THREADS); break;
+        case 5: if constexpr (!KEYS) go(tq_encode_pipe_kernel<D, 5, Tin, KEYS, NP>, PipeLayout<D, KEYS, 5, NP>::THREADS); else return cudaErrorInvalidValue; break;
         default: return cudaErrorInvalidValue;
     }
     return e;
@@ -1906,12 +1917,24 @@ bool tq_rows_map_4d(CUtensorMap *map, bool bf16, const void *base, int d, int64_
 static bool pipe_side(tq_ctx *ctx, bool keys, const void *x, tq_dtype dtype, int batch, int H, int64_t T, int64_t sb,
                       int64_t sh, int64_t st, const tq_codes *codes, int64_t token_offset, cudaStream_t stream,
                       int n_sms, cudaError_t *err) {
-    if (dtype == TQ_F32 || ctx->rotation != TQ_ROT_HADAMARD || (ctx->d != 64 && ctx->d != 128)) return false;
-    if (!ctx->d_HD16 || !ctx->d_HDbf) return false;
+    if (dtype == TQ_F32 || (ctx->d != 64 && ctx->d != 128)) return false;
+    // the Haar rotation: sqrt(d) Q in 2 (binary16 rows) or 3 (bfloat16 rows)
+    // pieces; the key kernel then shares one residual buffer between its groups
+    const bool haar = ctx->rotation == TQ_ROT_HAAR;
+    if (haar) {
+        if (!(dtype == TQ_BF16 ? (void *)ctx->d_Qbf : (void *)ctx->d_Qh)) return false;
+    } else if (ctx->rotation != TQ_ROT_HADAMARD || !ctx->d_HD16 || !ctx->d_HDbf) {
+        return false;
+    }
     const int d = ctx->d, M = ctx->m;
     if (keys) {
         if (2 * (d + std::max(d, M)) > 512) return false;   // two groups' TMEM columns
-        const size_t smem = (d == 128 ? PipeLayout<128, true, 2>::FIXED : PipeLayout<64, true, 2>::FIXED) + (size_t)(d / 64) * M * 128;
+        const int np = haar ? (dtype == TQ_BF16 ? 3 : 2) : 1;
+        const size_t fixed = d == 128 ? (np == 1 ? PipeLayout<128, true, 2, 1>::FIXED
+                                         : np == 2 ? PipeLayout<128, true, 2, 2>::FIXED : PipeLayout<128, true, 2, 3>::FIXED)
+                                      : (np == 1 ? PipeLayout<64, true, 2, 1>::FIXED
+                                         : np == 2 ? PipeLayout<64, true, 2, 2>::FIXED : PipeLayout<64, true, 2, 3>::FIXED);
+        const size_t smem = fixed + (size_t)(d / 64) * M * 128;
         if (smem > 227 * 1024) return false;
     }
     if (T > 0x7FFFFFFF - ENC_ROWS) return false;
@@ -1939,9 +1962,23 @@ static bool pipe_side(tq_ctx *ctx, bool keys, const void *x, tq_dtype dtype, int
     for (int i = 0; i + 1 < HBq; ++i) p.pb[i] = bd[HBq + i];
     if (keys) key_centroid_form(cb, HBq, p.cl);
     const int grid = (int)std::min<int64_t>(p.n_tiles, n_sms > 0 ? n_sms : 148);
-    const CUtensorMap &mhd = dtype == TQ_BF16 ? ctx->tmap_HDbf : ctx->tmap_HD16;
+    const CUtensorMap &mhd = haar ? (dtype == TQ_BF16 ? ctx->tmap_Qbf : ctx->tmap_Q)
+                                  : (dtype == TQ_BF16 ? ctx->tmap_HDbf : ctx->tmap_HD16);
     cudaError_t e;
-    if (d == 128) {
+    if (haar) {
+        // sqrt(d) Q in 2 binary16 or 3 bfloat16 pieces
+        const bool bf = dtype == TQ_BF16;
+        if (d == 128)
+            e = keys ? (bf ? launch_pipe<128, __nv_bfloat16, true, 3>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                           : launch_pipe<128, __half, true, 2>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream))
+                     : (bf ? launch_pipe<128, __nv_bfloat16, false, 3>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                           : launch_pipe<128, __half, false, 2>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream));
+        else
+            e = keys ? (bf ? launch_pipe<64, __nv_bfloat16, true, 3>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                           : launch_pipe<64, __half, true, 2>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream))
+                     : (bf ? launch_pipe<64, __nv_bfloat16, false, 3>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
+                           : launch_pipe<64, __half, false, 2>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream));
+    } else if (d == 128) {
         e = dtype == TQ_BF16 ? (keys ? launch_pipe<128, __nv_bfloat16, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)
                                      : launch_pipe<128, __nv_bfloat16, false>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream))
                              : (keys ? launch_pipe<128, __half, true>(Bq, p, mx, mhd, ctx->tmap_S, grid, stream)

@@ -40,6 +40,10 @@ struct tq_ctx {
     float *d_Q32;
     __half *d_Qh;
     CUtensorMap tmap_Q;
+    // and sqrt(d) Q as bfloat16 hi + mid + lo [heads][3][d][d] (d <= 128) for
+    // the TMA-fed value encoder's bfloat16 rows, same map geometry.
+    uint16_t *d_Qbf;
+    CUtensorMap tmap_Qbf;
     // Walsh-Hadamard rotation as a tensor-core operand: B[h][n][k] = H[n][k] D_h[k]
     // (+-1, exact in both 16-bit types), binary16 and bfloat16 copies
     // [heads][d][d], with TMA maps (inner d, outer heads*d rows, box 64 x d,
