@@ -97,6 +97,33 @@ def test_haar_power_of_two_scaling_tiny_and_nonfinite_rows():
     assert np.array_equal(c.k[0, 1, 5].cpu().numpy(), z.k[0, 1, 5].cpu().numpy())
 
 
+@pytest.mark.parametrize("dtype,scale", [(torch.float16, 2.0 ** -18), (torch.float16, 2.0 ** -10),
+                                         (torch.float16, 2.0 ** 13), (torch.bfloat16, 2.0 ** -40),
+                                         (torch.bfloat16, 2.0 ** 40)])
+def test_haar_encode_16bit_extreme_magnitudes(dtype, scale):
+    """16-bit rows are rotated in their own type against sqrt(d) Q split into
+    16-bit pieces, without a row scale: binary16 subnormals (2^-18), rows
+    mixing subnormal and normal entries (2^-10), rows near the binary16
+    maximum (2^13) and bfloat16 rows far from 1 (2^-40, 2^40) encode like the
+    oracle at d = 128 and d = 64."""
+    g = torch.Generator().manual_seed(int(abs(np.log2(scale))) + 7 * dtype.itemsize)
+    k = (torch.randn(1, 2, 260, 128, generator=g) * scale).to(dtype)
+    v = (torch.randn(1, 2, 260, 128, generator=g) * scale).to(dtype)
+    for d in (128, 64):
+        gc, oc = _pair(d, 4, 64, 21)
+        kd, vd = k[..., :d].contiguous(), v[..., :d].contiguous()
+        cache = gc.alloc(1, 2, 272)
+        gc.encode_kv(kd.to(DEV), vd.to(DEV), cache)
+        torch.cuda.synchronize()
+        assert gc.status() == (0, 0)
+        ek, ev = pu.oracle_encode(oc, kd, True), pu.oracle_encode(oc, vd, False)
+        rep = {}
+        for h in range(2):
+            pu.compare_k(cache.k[0, h, :260].cpu().numpy(), ek[0][h], oc, rep)
+            pu.compare_v(cache.v[0, h, :260].cpu().numpy(), ev[0][h], oc, rep)
+        assert rep["k_rows_flipped"] <= 3 and rep["v_index_flips"] <= 3, rep
+
+
 @pytest.mark.parametrize("bits", [2, 4])
 def test_haar_scores_and_dequant_match_oracle(bits):
     g = torch.Generator().manual_seed(40 + bits)
