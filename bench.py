@@ -112,21 +112,24 @@ def arm_config(workload):
 # were taken: once one of them changes the entry no longer applies (traffic:
 # null).  Summaries: profiles/.
 MEASURED_TRAFFIC = {
-    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 330933632),
-    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 320983040),
-    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 148838144),
-    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 298906240),
-    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 292800960),
-    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 81011520),
-    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 629141504),
-    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 616230848),
-    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 43086272),
-    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 42973376),
-    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 27370880),
-    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "cf099f439fbe227c73a8551fe390511856d10497", 149732032),
-    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 445050560),
-    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "c18571ca65b726ce0c3bb06f492de699369eb29a", 436104832),
-    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "58115251d06c1c6cbe58ef71971c963593d86b3b", 152447936),
+    ("encode_keys", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 330782976),
+    ("encode_values", "mha_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 321204032),
+    ("decode", "mha_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a55d60bb799f47a9fa64595e143b436cb1e3a32a", 149267136),
+    ("encode_keys", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 298793152),
+    ("encode_values", "gqa_decode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 292880512),
+    ("decode", "gqa_decode"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a55d60bb799f47a9fa64595e143b436cb1e3a32a", 81083520),
+    ("encode_keys", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 629477056),
+    ("encode_values", "bulk_encode"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 616778560),
+    ("encode_keys", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 43085248),
+    ("encode_values", "shared_prefix"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 42974656),
+    ("decode", "shared_prefix"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a55d60bb799f47a9fa64595e143b436cb1e3a32a", 27370688),
+    ("decode_append", "mha_append"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a55d60bb799f47a9fa64595e143b436cb1e3a32a", 149690688),
+    ("encode_keys", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 445315968),
+    ("encode_values", "mha_split"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 436353792),
+    ("decode_split", "mha_split"): (('tq_split.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "3deb5480f30ab8588392a6ac1abc822623297177", 152436800),
+    ("encode_keys", "mha_decode_haar"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 333529664),
+    ("encode_values", "mha_decode_haar"): (('tq_encode.cu', 'tq_internal.cuh'), "008f084c694e2a11b023fe06e61a5027e32563c1", 322862464),
+    ("decode", "mha_decode_haar"): (('tq_decode.cu', 'tq_decode_mma.cu', 'tq_aux.cu', 'tq_decode.cuh', 'tq_internal.cuh'), "a55d60bb799f47a9fa64595e143b436cb1e3a32a", 153262400),
 }
 
 
