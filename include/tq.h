@@ -145,14 +145,19 @@ tq_status tq_create(int head_dim, int bits, int projections, uint64_t seed, tq_c
  * matrix of N(0,1) Box-Muller draws that continue head h's SplitMix64
  * stream (seed + h) after the d sign draws and the m*d (rounded up to even)
  * draws of S; Q's columns are signed so that R has a positive diagonal.  The
- * rows are rotated on the tensor cores (sqrt(d) Q as binary16 hi + lo
- * against the row scaled by a power of two into binary16 range: binary16
- * and bfloat16 rows exactly, float32 rows as hi + lo), queries and outputs
- * with fp32 Q.  Not available at head_dim 256 (TQ_ERR_DIM: the two binary16
- * pieces of sqrt(d) Q alone fill 256 KB, above the 227 KB of shared memory a
- * CTA can hold).  Packed formats and every other call are unchanged.  In this
- * mode a row whose largest |x_j| is below 2^-100 is encoded as a zero row.
- * Returns TQ_ERR_DIM for an unknown rotation. */
+ * rows are rotated on the tensor cores: binary16 and bfloat16 rows as they
+ * are, against sqrt(d) Q split into 2 binary16 or 3 bfloat16 pieces of the
+ * row's own type (the TMA-fed encoder); float32 rows, and bfloat16 keys with
+ * more than 136 projections (whose three pieces leave too little shared
+ * memory), scaled by a power of two into binary16 range and split hi + lo,
+ * against sqrt(d) Q as binary16 hi + lo.  Queries and outputs use fp32 Q.
+ * Not available at head_dim 256 (TQ_ERR_DIM: the two binary16 pieces of
+ * sqrt(d) Q alone fill 256 KB, above the 227 KB of shared memory a CTA can
+ * hold).  Packed formats and every other call are unchanged.  In this mode a
+ * row whose largest |x_j| is below 2^-100 is encoded as a zero row, and so is
+ * a 16-bit row on the TMA-fed encoder whose d |x|^2 is below the smallest
+ * normal float (as under the default rotation).  Returns TQ_ERR_DIM for an
+ * unknown rotation. */
 tq_status tq_create_ex(int head_dim, int bits, int projections, uint64_t seed, tq_rotation rotation,
                        tq_ctx **out);
 
