@@ -97,6 +97,34 @@ def test_haar_power_of_two_scaling_tiny_and_nonfinite_rows():
     assert np.array_equal(c.k[0, 1, 5].cpu().numpy(), z.k[0, 1, 5].cpu().numpy())
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_haar_encode_many_tiles_per_cta_strided_offset(d, dtype):
+    """Enough 128-row tiles (16 heads x 33 tiles) that the persistent encoder's
+    CTAs each take several, crossing heads, so the rotation pieces of sqrt(d) Q
+    are reloaded mid-CTA; the input is a [B, T, H, d] tensor viewed as
+    [B, H, T, d] (token stride H d), written at token offset 37 with a ragged
+    last tile.  Sampled heads are compared with the oracle in full, and the
+    rows outside the written range stay zero."""
+    g = torch.Generator().manual_seed(d + 3 * dtype.itemsize)
+    B, H, T, off = 1, 16, 33 * 128 - 51, 37
+    base = torch.randn(B, T, H, d, generator=g).to(dtype)
+    k, v = base.permute(0, 2, 1, 3), (base * 0.5).permute(0, 2, 1, 3)
+    gc, oc = _pair(d, 4, 128, 31)
+    cache = gc.alloc(B, H, _cap(T + off))
+    gc.encode_kv(base.to(DEV).permute(0, 2, 1, 3), (base * 0.5).to(DEV).permute(0, 2, 1, 3), cache, off)
+    torch.cuda.synchronize()
+    assert gc.status() == (0, 0)
+    rep = {}
+    for h in (0, 5, 10, 15):
+        ek = oc.encode(k[0, h].double().numpy(), h, True)
+        ev = oc.encode(v[0, h].double().numpy(), h, False)
+        pu.compare_k(cache.k[0, h, off:off + T].cpu().numpy(), ek, oc, rep)
+        pu.compare_v(cache.v[0, h, off:off + T].cpu().numpy(), ev, oc, rep)
+    assert rep["k_rows_flipped"] <= 12 and rep["v_index_flips"] <= 12, rep
+    assert int(cache.k[:, :, :off].abs().sum()) == 0 and int(cache.v[:, :, off + T:].abs().sum()) == 0
+
+
 @pytest.mark.parametrize("dtype,scale", [(torch.float16, 2.0 ** -18), (torch.float16, 2.0 ** -10),
                                          (torch.float16, 2.0 ** 13), (torch.bfloat16, 2.0 ** -40),
                                          (torch.bfloat16, 2.0 ** 40)])
