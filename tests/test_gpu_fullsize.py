@@ -62,6 +62,34 @@ def test_mha_decode_full_size_sampled_heads():
     print("flips:", rep)
 
 
+@pytest.mark.parametrize("variant", ["haar", "f16norms"])
+def test_mha_decode_variants_full_size_sampled_heads(variant):
+    """The multi-head workload under the Haar-QR rotation (the TMA-fed
+    encoders with sqrt(d) Q in two binary16 pieces) and with binary16 key
+    norms, as bench.py times them; (b, h) = (1, 3) and (7, 30)."""
+    w = workloads.mha_decode(device=DEV, data_seed=4)
+    B, H, T, _ = w["k"].shape
+    kw = dict(rotation="haar") if variant == "haar" else dict(norms="f16")
+    gc = tq.Codec(D, w["bits"], M, w["seed"], **kw)
+    cache = gc.alloc(B, H, T)
+    gc.encode_kv(w["k"], w["v"], cache)
+    segs = [tq.Segment(cache, T, b, 1, codes_batch=b) for b in range(B)]
+    out = torch.empty(B, H, D, dtype=w["q"].dtype, device=DEV)
+    ws = torch.empty(max(tq.tq_decode_workspace_bytes(segs, B, H, H), 16), dtype=torch.uint8, device=DEV)
+    tq.tq_decode_attention(segs, w["q"], B, H, H, out, ws)
+    torch.cuda.synchronize()
+    assert gc.status() == (0, 0)
+    oc = oracle.Codec(D, w["bits"], M, w["seed"], **kw)
+    rep = {}
+    for b, h in ((1, 3), (7, 30)):
+        ek = oc.encode(w["k"][b, h].double().cpu().numpy(), h, True)
+        ev = oc.encode(w["v"][b, h].double().cpu().numpy(), h, False)
+        _check_rows(cache, oc, ek, ev, b, h, T, rep)
+        ref = oracle.attention(w["q"][b, h].double().cpu().numpy(), [(oc, h, ek["rows"], ev["rows"])])
+        _check_out(out, ref, b, h)
+    print("flips:", rep)
+
+
 def test_gqa_decode_full_size_sampled_heads():
     """batch 4, 32 query heads over 8 kv heads, 32768 tokens, bf16, bits 2;
     (b, h_kv) = (0, 0) and (3, 5), all 4 query heads of each."""
