@@ -176,3 +176,63 @@ def test_bulk_encode_full_size_sampled_layers():
         ev = oc.encode(w["v"][layer, h].double().cpu().numpy(), h, False)
         _check_rows(cache, oc, ek, ev, slot, h, T, rep)
     print("flips:", rep)
+
+
+def test_mha_split_full_size_sampled_heads():
+    """The multi-head data with each head's channels ordered by RMS over its
+    keys and split into 64 outlier channels at bits 4 (m 64) and 64 normal
+    channels at bits 3 (m 64), encoded and decoded as bench.py does it;
+    (b, h) = (2, 9) and (5, 26)."""
+    w = workloads.mha_decode(device=DEV, data_seed=2)
+    B, H, T, _ = w["k"].shape
+    order = w["k"].float().pow(2).mean(dim=(0, 2)).argsort(dim=-1, descending=True)
+    idx = order[None, :, None, :]
+    k = torch.gather(w["k"], 3, idx.expand_as(w["k"])).contiguous()
+    v = torch.gather(w["v"], 3, idx.expand_as(w["v"])).contiguous()
+    q = torch.gather(w["q"], 2, order[None].expand_as(w["q"])).contiguous()
+    go, gn = tq.Codec(64, 4, 64, w["seed"]), tq.Codec(64, 3, 64, w["seed"] + 1000)
+    co, cn = go.alloc(B, H, T), gn.alloc(B, H, T)
+    go.encode_kv(k[..., :64], None, co)
+    gn.encode_kv(k[..., 64:], None, cn)
+    go.encode_kv(None, v[..., :64], co)
+    gn.encode_kv(None, v[..., 64:], cn)
+    out = tq.decode_split(go, co, gn, cn, T, q)
+    torch.cuda.synchronize()
+    assert go.status() == (0, 0) and gn.status() == (0, 0)
+    oo, on = oracle.Codec(64, 4, 64, w["seed"]), oracle.Codec(64, 3, 64, w["seed"] + 1000)
+    rep = {}
+    for b, h in ((2, 9), (5, 26)):
+        kb, vb = k[b, h].double().cpu().numpy(), v[b, h].double().cpu().numpy()
+        eko, evo = oo.encode(kb[:, :64], h, True), oo.encode(vb[:, :64], h, False)
+        ekn, evn = on.encode(kb[:, 64:], h, True), on.encode(vb[:, 64:], h, False)
+        _check_rows(co, oo, eko, evo, b, h, T, rep)
+        _check_rows(cn, on, ekn, evn, b, h, T, rep)
+        ref = oracle.attention_split(q[b, h].double().cpu().numpy(), (oo, h, eko["rows"], evo["rows"]),
+                                     (on, h, ekn["rows"], evn["rows"]))
+        _check_out(out, ref, b, h)
+    print("flips:", rep)
+
+
+def test_mha_append_full_size_sampled_heads():
+    """batch 8 x 32 heads, 4096 cached tokens encoded in bulk, then the step
+    that appends token 4096 and attends over 4097, as bench.py times it; the
+    appended rows and the outputs of (b, h) = (3, 4) and (6, 31)."""
+    w = workloads.mha_decode(device=DEV, data_seed=2, n_tokens=4097)
+    B, H, T1, _ = w["k"].shape
+    T = T1 - 1
+    gc = tq.Codec(D, w["bits"], M, w["seed"])
+    cache = gc.alloc(B, H, T + 16)
+    gc.encode_kv(w["k"][:, :, :T], w["v"][:, :, :T], cache)
+    segs = [tq.Segment(cache, T, b, 1, codes_batch=b) for b in range(B)]
+    out = tq.decode_append(segs, w["k"][:, :, T], w["v"][:, :, T], w["q"], H)
+    torch.cuda.synchronize()
+    assert gc.status() == (0, 0)
+    oc = oracle.Codec(D, w["bits"], M, w["seed"])
+    rep = {}
+    for b, h in ((3, 4), (6, 31)):
+        ek = oc.encode(w["k"][b, h].double().cpu().numpy(), h, True)
+        ev = oc.encode(w["v"][b, h].double().cpu().numpy(), h, False)
+        _check_rows(cache, oc, ek, ev, b, h, T1, rep)
+        ref = oracle.attention(w["q"][b, h].double().cpu().numpy(), [(oc, h, ek["rows"], ev["rows"])])
+        _check_out(out, ref, b, h)
+    print("flips:", rep)
